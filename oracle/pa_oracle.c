@@ -1,0 +1,300 @@
+/*
+ * Paged KV-cache append and paged decode attention: fp64 CPU ORACLE.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file; only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline
+ * leg may.  It shares no code, header, helper or constant with the CUDA
+ * library: it is a plain, slow restatement of what the pages define.
+ *
+ * What the pages define, and where:
+ *  - "vLLM — PagedAttention으로 LLM 추론 성능을 2~4배 끌어올린 서빙 엔진" (dev.to),
+ *    section "PagedAttention — OS 가상 메모리에서 영감": the KV cache is cut into
+ *    fixed-size blocks (pages); physical and logical blocks are kept apart so
+ *    that non-contiguous physical memory is used as if it were contiguous.
+ *    Here: logical token j of a sequence lives in physical block
+ *    table[j / Bs] at offset j % Bs (oracle_slot, gather_sequence).
+ *  - same page, section "KV Cache가 왜 병목인가": each generated token's
+ *    self-attention reads the Key and Value of every previous token, which is
+ *    why they are cached (oracle_paged_decode reads all L cached tokens), and
+ *    the cache size is 2 (K and V) x layers x heads x head_dim x tokens x
+ *    bytes per element (oracle_kv_bytes).
+ *  - "[Hacker News 요약] ... Tiny-vLLM ..." (aisleshub), section
+ *    "고성능 추론을 위한 고급 최적화 기법": attention is the basic formula of
+ *    "Attention is all you need" (softmax(q K^T * scale) V), the KV cache keeps
+ *    K/V projections of previous tokens, grouped-query attention lets several
+ *    query heads share one K/V head, and a causal mask lets a token see only
+ *    earlier tokens.  With one decode query at the last position the mask
+ *    keeps every cached token.
+ *  - Readings where the pages are silent (stated, not derived): the pool is
+ *    laid out [num_blocks][num_kv_heads][block_size][head_dim]; query head h
+ *    reads kv head h / (Hq / Hkv) (contiguous groups); a sequence with no
+ *    cached token outputs zeros; a negative slot means "do not write"; a slot
+ *    past the pool is not written either.
+ *
+ * Everything is computed in double.  bf16 inputs are widened exactly
+ * (bits << 16 is the float with the same value; float -> double is exact).
+ * Sums run in logical token order, so the result does not depend on where the
+ * blocks physically are.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---- bf16 (8-bit exponent, 7-bit mantissa: the upper half of an IEEE float) ---- */
+double oracle_bf16_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ---- KV size accounting: 2 (K and V) x layers x heads x head_dim x tokens x bytes ---- */
+int64_t oracle_kv_bytes(int64_t layers, int64_t kv_heads, int64_t head_dim, int64_t tokens,
+                        int64_t bytes_per_element) {
+    return 2 * layers * kv_heads * head_dim * tokens * bytes_per_element;
+}
+
+/* ---- logical -> physical: the slot of logical position p in a sequence's table ---- */
+int64_t oracle_slot(const int32_t* table_row, int64_t position, int64_t block_size) {
+    const int64_t logical_block = position / block_size;
+    const int64_t offset = position % block_size;
+    return (int64_t)table_row[logical_block] * block_size + offset;
+}
+
+/* slots for the newest token of each sequence (position = length - 1) */
+void oracle_slot_mapping(const int32_t* block_tables, int64_t max_blocks_per_seq,
+                         const int32_t* lengths_after_append, int64_t num_seqs,
+                         int64_t block_size, int64_t* slots) {
+    for (int64_t b = 0; b < num_seqs; ++b) {
+        const int64_t p = (int64_t)lengths_after_append[b] - 1;
+        slots[b] = p < 0 ? -1 : oracle_slot(block_tables + b * max_blocks_per_seq, p, block_size);
+    }
+}
+
+/* grouped-query attention: query head h reads kv head h / (Hq / Hkv) */
+static int64_t kv_head_of(int64_t h, int64_t num_q_heads, int64_t num_kv_heads) {
+    return h / (num_q_heads / num_kv_heads);
+}
+
+/* element index of (block, kv head, offset, d) in the [N][Hkv][Bs][D] pool */
+static int64_t pool_index(int64_t block, int64_t kv_head, int64_t offset, int64_t d,
+                          int64_t num_kv_heads, int64_t block_size, int64_t head_dim) {
+    return ((block * num_kv_heads + kv_head) * block_size + offset) * head_dim + d;
+}
+
+/* ---- KV append: write token t's K/V rows into slot slot_mapping[t] ---- */
+void oracle_append_kv(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping,
+                      int64_t num_tokens, int64_t num_kv_heads, int64_t head_dim,
+                      int64_t block_size, int64_t num_blocks, uint16_t* k_cache,
+                      uint16_t* v_cache) {
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0 || slot >= num_blocks * block_size) continue;
+        const int64_t block = slot / block_size;
+        const int64_t offset = slot % block_size;
+        for (int64_t h = 0; h < num_kv_heads; ++h) {
+            for (int64_t d = 0; d < head_dim; ++d) {
+                const int64_t dst = pool_index(block, h, offset, d, num_kv_heads, block_size, head_dim);
+                const int64_t src = (t * num_kv_heads + h) * head_dim + d;
+                k_cache[dst] = k[src];
+                v_cache[dst] = v[src];
+            }
+        }
+    }
+}
+
+/* Gather logical tokens [0, L) of one sequence and kv head into contiguous fp64 rows. */
+static void gather_sequence(const uint16_t* cache, const int32_t* table_row, int64_t L,
+                            int64_t kv_head, int64_t num_kv_heads, int64_t block_size,
+                            int64_t head_dim, double* rows) {
+    for (int64_t j = 0; j < L; ++j) {
+        const int64_t slot = oracle_slot(table_row, j, block_size);
+        const int64_t block = slot / block_size;
+        const int64_t offset = slot % block_size;
+        for (int64_t d = 0; d < head_dim; ++d) {
+            rows[j * head_dim + d] = oracle_bf16_to_double(
+                cache[pool_index(block, kv_head, offset, d, num_kv_heads, block_size, head_dim)]);
+        }
+    }
+}
+
+/*
+ * Textbook attention of one query over contiguous rows [t0, t1):
+ *   s_j = scale * sum_d q_d K_jd,  m = max_j s_j,  e_j = exp(s_j - m),  Z = sum_j e_j,
+ *   p_j = e_j / Z,  o_d = sum_j p_j V_jd,  lse = m + ln Z.
+ * Writes o (head_dim values), returns lse; *psum = sum_j p_j.
+ */
+static double attend(const double* qd, const double* K, const double* V, int64_t t0, int64_t t1,
+                     int64_t head_dim, double scale, double* s, double* o, double* psum) {
+    double m = -INFINITY;
+    for (int64_t j = t0; j < t1; ++j) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < head_dim; ++d) dot += qd[d] * K[j * head_dim + d];
+        s[j - t0] = scale * dot;
+        if (s[j - t0] > m) m = s[j - t0];
+    }
+    double Z = 0.0;
+    for (int64_t j = t0; j < t1; ++j) Z += exp(s[j - t0] - m);
+    double total = 0.0;
+    for (int64_t d = 0; d < head_dim; ++d) o[d] = 0.0;
+    for (int64_t j = t0; j < t1; ++j) {
+        const double p = exp(s[j - t0] - m) / Z;
+        total += p;
+        for (int64_t d = 0; d < head_dim; ++d) o[d] += p * V[j * head_dim + d];
+    }
+    if (psum) *psum = total;
+    return m + log(Z);
+}
+
+static int g_threads = 0; /* 0: OpenMP default */
+
+void oracle_set_num_threads(int n) { g_threads = n; }
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return g_threads > 0 ? g_threads : omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Paged decode attention.
+ *   q            [B][Hq][D] bf16 bits        block_tables [B][MB] int32
+ *   k/v_cache    [N][Hkv][Bs][D] bf16 bits   context_lens [B] int32 (tokens attended)
+ *   out          [B][Hq][D] double           weight_sums  [B][Hq] double or NULL
+ * For each sequence b and query head h: gather the L = context_lens[b] cached
+ * tokens of kv head h / (Hq/Hkv) into contiguous rows, then attend.
+ * Work is spread over (sequence, kv head) pairs so one gather serves the query
+ * heads that read that kv head; each output's arithmetic is the same serial
+ * loop whatever the thread count.
+ */
+int oracle_paged_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                        const int32_t* block_tables, const int32_t* context_lens,
+                        int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                        int64_t head_dim, int64_t block_size, int64_t max_blocks_per_seq,
+                        double scale, double* out, double* weight_sums) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return -1;
+    const int64_t pairs = num_seqs * num_kv_heads;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_num_threads())
+    for (int64_t pair = 0; pair < pairs; ++pair) {
+        const int64_t b = pair / num_kv_heads;
+        const int64_t kvh = pair % num_kv_heads;
+        const int64_t L = context_lens[b];
+        const int32_t* table_row = block_tables + b * max_blocks_per_seq;
+        for (int64_t h = 0; h < num_q_heads; ++h) {
+            if (kv_head_of(h, num_q_heads, num_kv_heads) != kvh) continue;
+            double* o = out + (b * num_q_heads + h) * head_dim;
+            for (int64_t d = 0; d < head_dim; ++d) o[d] = 0.0;
+            if (weight_sums) weight_sums[b * num_q_heads + h] = 0.0;
+        }
+        if (L <= 0) continue;
+        double* K = (double*)malloc(sizeof(double) * (size_t)(L * head_dim));
+        double* V = (double*)malloc(sizeof(double) * (size_t)(L * head_dim));
+        double* s = (double*)malloc(sizeof(double) * (size_t)L);
+        double* qd = (double*)malloc(sizeof(double) * (size_t)head_dim);
+        if (!K || !V || !s || !qd) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            gather_sequence(k_cache, table_row, L, kvh, num_kv_heads, block_size, head_dim, K);
+            gather_sequence(v_cache, table_row, L, kvh, num_kv_heads, block_size, head_dim, V);
+            for (int64_t h = 0; h < num_q_heads; ++h) {
+                if (kv_head_of(h, num_q_heads, num_kv_heads) != kvh) continue;
+                for (int64_t d = 0; d < head_dim; ++d)
+                    qd[d] = oracle_bf16_to_double(q[(b * num_q_heads + h) * head_dim + d]);
+                attend(qd, K, V, 0, L, head_dim, scale, s,
+                       out + (b * num_q_heads + h) * head_dim,
+                       weight_sums ? weight_sums + b * num_q_heads + h : NULL);
+            }
+        }
+        free(K);
+        free(V);
+        free(s);
+        free(qd);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Partial attention of every (sequence, query head) over the logical token
+ * range [t0, min(t1, L)): normalised output o [B][Hq][D] and its natural-log
+ * log-sum-exp lse [B][Hq] (-inf and o = 0 when the range is empty).  This is
+ * the state a split of the context produces before the splits are merged.
+ */
+int oracle_paged_decode_partial(const uint16_t* q, const uint16_t* k_cache,
+                                const uint16_t* v_cache, const int32_t* block_tables,
+                                const int32_t* context_lens, int64_t num_seqs,
+                                int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                                int64_t block_size, int64_t max_blocks_per_seq, double scale,
+                                int64_t t0, int64_t t1, double* o_out, double* lse_out) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return -1;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_num_threads())
+    for (int64_t pair = 0; pair < num_seqs * num_kv_heads; ++pair) {
+        const int64_t b = pair / num_kv_heads;
+        const int64_t kvh = pair % num_kv_heads;
+        const int64_t L = context_lens[b];
+        const int64_t hi = t1 < L ? t1 : L;
+        for (int64_t h = 0; h < num_q_heads; ++h) {
+            if (kv_head_of(h, num_q_heads, num_kv_heads) != kvh) continue;
+            for (int64_t d = 0; d < head_dim; ++d) o_out[(b * num_q_heads + h) * head_dim + d] = 0.0;
+            lse_out[b * num_q_heads + h] = -INFINITY;
+        }
+        if (hi <= t0) continue;
+        double* K = (double*)malloc(sizeof(double) * (size_t)(hi * head_dim));
+        double* V = (double*)malloc(sizeof(double) * (size_t)(hi * head_dim));
+        double* s = (double*)malloc(sizeof(double) * (size_t)(hi - t0));
+        double* qd = (double*)malloc(sizeof(double) * (size_t)head_dim);
+        if (!K || !V || !s || !qd) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            const int32_t* table_row = block_tables + b * max_blocks_per_seq;
+            gather_sequence(k_cache, table_row, hi, kvh, num_kv_heads, block_size, head_dim, K);
+            gather_sequence(v_cache, table_row, hi, kvh, num_kv_heads, block_size, head_dim, V);
+            for (int64_t h = 0; h < num_q_heads; ++h) {
+                if (kv_head_of(h, num_q_heads, num_kv_heads) != kvh) continue;
+                for (int64_t d = 0; d < head_dim; ++d)
+                    qd[d] = oracle_bf16_to_double(q[(b * num_q_heads + h) * head_dim + d]);
+                lse_out[b * num_q_heads + h] =
+                    attend(qd, K, V, t0, hi, head_dim, scale, s,
+                           o_out + (b * num_q_heads + h) * head_dim, NULL);
+            }
+        }
+        free(K);
+        free(V);
+        free(s);
+        free(qd);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Merge S partial states of one query: each split s covers a disjoint token
+ * range with normalised output o_s and lse_s = ln sum_{j in s} exp(score_j).
+ * Softmax over the union: weight of split s is exp(lse_s - M) with
+ * M = max_s lse_s; out = sum_s w_s o_s / sum_s w_s.  Splits with lse = -inf
+ * (empty) get weight 0; if all are empty the output is zero.
+ */
+void oracle_merge_partials(const double* o, const double* lse, int64_t num_splits,
+                           int64_t head_dim, double* out) {
+    double M = -INFINITY;
+    for (int64_t s = 0; s < num_splits; ++s)
+        if (lse[s] > M) M = lse[s];
+    for (int64_t d = 0; d < head_dim; ++d) out[d] = 0.0;
+    if (M == -INFINITY) return;
+    double W = 0.0;
+    for (int64_t s = 0; s < num_splits; ++s) {
+        const double w = exp(lse[s] - M);
+        W += w;
+        for (int64_t d = 0; d < head_dim; ++d) out[d] += w * o[s * head_dim + d];
+    }
+    for (int64_t d = 0; d < head_dim; ++d) out[d] /= W;
+}

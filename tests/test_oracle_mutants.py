@@ -1,0 +1,105 @@
+"""The oracle pins have teeth: each plausible mistake, planted in a copy of the
+oracle's C source and compiled on the CPU, must make at least one pin fail.
+
+The mutant library replaces the oracle's loaded library only for the duration
+of one test; the real oracle source is never modified.
+"""
+import inspect
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from tests import test_oracle as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.c")
+
+MUTANTS = {
+    # query head h reads kv head h % Hkv instead of h / (Hq/Hkv)
+    "gqa_modulo_grouping": ("return h / (num_q_heads / num_kv_heads);",
+                            "return h % num_kv_heads;"),
+    # the softmax scale is dropped
+    "scale_dropped": ("s[j - t0] = scale * dot;", "s[j - t0] = dot;"),
+    # offset inside a block off by one
+    "offset_off_by_one": ("const int64_t offset = position % block_size;",
+                          "const int64_t offset = (position + 1) % block_size;"),
+    # pool read as [N][Bs][Hkv][D] (head and offset axes transposed)
+    "pool_axes_transposed": (
+        "return ((block * num_kv_heads + kv_head) * block_size + offset) * head_dim + d;",
+        "return ((block * block_size + offset) * num_kv_heads + kv_head) * head_dim + d;"),
+    # weights not normalised
+    "softmax_not_normalised": ("const double p = exp(s[j - t0] - m) / Z;",
+                               "const double p = exp(s[j - t0] - m);"),
+    # the newest token is left out of the context
+    "last_token_dropped": ("for (int64_t j = t0; j < t1; ++j) {\n        double dot",
+                           "for (int64_t j = t0; j + 1 < t1; ++j) {\n        double dot"),
+    # log-sum-exp loses the running max
+    "lse_without_max": ("return m + log(Z);", "return log(Z);"),
+    # merge weights with the wrong sign in the exponent
+    "merge_weight_sign": ("const double w = exp(lse[s] - M);", "const double w = exp(M - lse[s]);"),
+    # append writes V's row into the K cache
+    "append_k_from_v": ("k_cache[dst] = k[src];", "k_cache[dst] = v[src];"),
+    # append ignores the skip marker and writes a slot -1 token to slot 0
+    "append_negative_not_skipped": ("const int64_t slot = slot_mapping[t];",
+                                    "const int64_t slot = slot_mapping[t] < 0 ? 0 : slot_mapping[t];"),
+    # K and V swapped in the gather
+    "k_v_swapped": ("gather_sequence(k_cache, table_row, L, kvh", "gather_sequence(v_cache, table_row, L, kvh"),
+}
+
+
+def _pin_calls():
+    """Every pin in test_oracle as a zero-argument callable (parametrised ones expanded)."""
+    calls = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if not params:
+            calls.append((name, fn, {}))
+            continue
+        mark = params[0]
+        argnames = [a.strip() for a in mark.args[0].split(",")] if isinstance(mark.args[0], str) else list(mark.args[0])
+        for values in mark.args[1]:
+            values = values if len(argnames) > 1 else (values,)
+            calls.append((name, fn, dict(zip(argnames, values))))
+    return calls
+
+
+def _build_mutant(old, new, tmpdir):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, "mutation anchor not found: %r" % old
+    src = src.replace(old, new, 1)
+    path_c = os.path.join(tmpdir, "mutant.c")
+    path_so = os.path.join(tmpdir, "mutant.so")
+    open(path_c, "w").write(src)
+    subprocess.check_call(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", path_c,
+                           "-o", path_so, "-lm"])
+    return path_so
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(mutant, monkeypatch):
+    import ctypes
+    old, new = MUTANTS[mutant]
+    real = oracle._lib()
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _build_mutant(old, new, tmp)
+        mut = ctypes.CDLL(so)
+        # reuse the real library's prototypes on the mutant's symbols
+        for sym in ("oracle_bf16_to_double", "oracle_kv_bytes", "oracle_slot", "oracle_slot_mapping",
+                    "oracle_append_kv", "oracle_paged_decode", "oracle_paged_decode_partial",
+                    "oracle_merge_partials", "oracle_set_num_threads", "oracle_num_threads"):
+            f_real, f_mut = getattr(real, sym), getattr(mut, sym)
+            f_mut.argtypes = f_real.argtypes
+            f_mut.restype = f_real.restype
+        monkeypatch.setattr(oracle, "_LIB", mut)
+        caught = []
+        for name, fn, kwargs in _pin_calls():
+            try:
+                fn(**kwargs)
+            except AssertionError:
+                caught.append(name)
+        assert caught, "no pin caught mutant %s" % mutant
