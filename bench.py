@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode step (KV append + paged decode attention).
+
+One step = one decode step of one attention layer for the whole batch:
+append each sequence's new token into its slot (pa_append_kv), then paged
+decode attention over every cached token (pa_decode; long contexts split
+across CTAs and merged in the same launch).  The default workload is the
+Llama-3.2-1B-shaped layer: 64 sequences, Hq=32, Hkv=8, head_dim 64, block
+size 16, cached lengths uniform in [128, 2048], blocks scattered over a pool
+10 % larger than needed.  Successive steps rotate over independent copies of
+the layer's pool (different addresses, > 1 GB together) so that the 126 MB L2
+cannot serve the K/V reads.
+
+Prints one JSON line (rank 0).  `value` is seq-steps/s over all ranks with
+inputs resident in HBM; `e2e` repeats the measurement with each step's inputs
+copied from pinned host memory and the output copied back inside the timed
+region.  `roofline` reports the decode kernel's KV-read bandwidth against the
+measured HBM copy bandwidth.  `cpu_baseline` times the fp64 CPU oracle on a
+bounded sample.  With --impl reference the oracle alone is timed.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+path has no exchange step); the timed region is bracketed by barriers and the
+max over ranks is reported (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged-decode seq-steps/s and KV-read HBM GB/s (fraction of B200 peak)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD_TEXT = {
+    "c1": "tiny: B=2, L=5/37 (+1 appended), Hq=2, Hkv=1, D=64, Bs=16, 8 blocks",
+    "c2": "Llama-3.2-1B-shaped decode layer: B=64, Hq=32, Hkv=8, D=64, Bs=16, cached L~U[128,2048] (+1 appended), pool=needed+10%",
+    "c3": "shared 1024-token prefix (4 blocks in every table) + suffix~U[256,7168] (+1), B=32, Hq=32, Hkv=8, D=64, Bs=256",
+    "c4": "long context split-KV: B=4, L=32768/65536/98304/131072 (+1), Hq=64, Hkv=8, D=128, Bs=16",
+}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4"], default="c2")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--split-tokens", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------------------------
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kv_read_bytes(lens, num_kv_heads, head_dim):
+    """Algorithmic K+V bytes one decode launch must read: 2 (K,V) x L x Hkv x D x 2 B per sequence."""
+    return int(2 * int(np.sum(lens, dtype=np.int64)) * num_kv_heads * head_dim * 2)
+
+
+def kernel_source_hash(kernel_name):
+    files = {"tensor": ["decode_tensor.cu"], "simt": ["decode_simt.cu"]}[kernel_name]
+    files = files + ["pa_device.cuh", "pa_internal.h", "api.cu"]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "pagedattention_kv_cache_pa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config, kernel_name):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+    prof = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(prof):
+        return None
+    pat = re.compile(r"^traffic\[%s,%s\]:\s*([0-9]+)\s+bytes/launch\s+source=([0-9a-f]+)"
+                     % (re.escape(config), re.escape(kernel_name)), re.M)
+    want = kernel_source_hash(kernel_name)
+    for name in sorted(os.listdir(prof)):
+        if not name.endswith((".txt", ".md")):
+            continue
+        m = pat.search(open(os.path.join(prof, name)).read())
+        if m and m.group(2) == want:
+            return int(m.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index, enabled=True):
+        self.proc = None
+        self.device_index = device_index
+        if not enabled:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# the reference arm: the fp64 CPU oracle
+# ---------------------------------------------------------------------------------------------
+def run_reference(args, rank):
+    import oracle
+    if rank != 0:
+        return None
+    b = wl.CONFIGS[args.config]()
+    B, Bs = b.batch, b.block_size
+    model = oracle.BlockManagerModel(b.num_blocks, Bs, B, b.max_blocks_per_seq, b.free_order)
+    for s in range(B):
+        L = int(b.context_lens[s])
+        model.import_seq(s, L, b.block_tables[s, : -(-L // Bs)])
+    slots = np.array(model.append_tokens(list(range(B))), dtype=np.int64)
+    tables = np.array([model.table_array(s) for s in range(B)], dtype=np.int32)
+    lens = np.array(model.lens, dtype=np.int32)
+    kc, vc = b.k_cache.copy(), b.v_cache.copy()
+
+    def one(i):
+        s = i % B   # one step = one sequence's append + decode (all its heads)
+        oracle.append_kv(b.k_new[s:s + 1], b.v_new[s:s + 1], slots[s:s + 1], kc, vc, in_place=True)
+        oracle.paged_decode(b.q[s:s + 1], kc, vc, tables[s:s + 1], lens[s:s + 1], b.scale)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    cores = oracle.num_threads()
+    sample = "%d steps, each one sequence (cycling over the %d of %s) appended and decoded over all %d query heads" % (
+        args.steps, B, args.config.upper(), b.num_q_heads)
+    return {"metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD_TEXT[args.config], "config": args.config,
+                       "batch": B},
+            "cpu_baseline": {"value": value, "unit": "seq-steps/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "seq-steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def cpu_baseline(b, slots, tables, lens, budget_s):
+    """The oracle as it stands on the host's cores, on whole-batch steps until the budget is spent."""
+    import oracle
+    kc, vc = b.k_cache.copy(), b.v_cache.copy()
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.append_kv(b.k_new, b.v_new, slots, kc, vc, in_place=True)
+        oracle.paged_decode(b.q, kc, vc, tables, lens, b.scale)
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n >= 1000:
+            break
+    return {"value": n * b.batch / dt, "unit": "seq-steps/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d whole-batch steps of %s (append + decode of all %d sequences x %d heads), %.1f s"
+                      % (n, b.name, b.batch, b.num_q_heads, dt)}
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+def run_ours(args, rank, world, dist):
+    import torch
+    import pagedattention_kv_cache_pa_b200 as pa
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    b = wl.CONFIGS[args.config]()
+    B, Bs, MB = b.batch, b.block_size, b.max_blocks_per_seq
+    Hq, Hkv, D = b.num_q_heads, b.num_kv_heads, b.head_dim
+
+    # (a1, a2) on the host: give each sequence its new token's slot
+    bm = pa.BlockManager(b.num_blocks, Bs, B, MB, b.free_order)
+    for s in range(B):
+        L = int(b.context_lens[s])
+        bm.import_seq(s, L, b.block_tables[s, : -(-L // Bs)])
+    slots = bm.append_tokens(np.arange(B, dtype=np.int32))
+    tables = bm.block_tables().copy()
+    lens = bm.context_lens().copy()
+    bm.close()
+    max_len = int(lens.max())
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    pool_bytes = 2 * b.k_cache.nbytes
+    layers = max(1, min(8, math.ceil(1.0e9 / pool_bytes)))
+    kcs = [to_dev(b.k_cache) for _ in range(layers)]
+    vcs = [to_dev(b.v_cache) for _ in range(layers)]
+    q, k_new, v_new = to_dev(b.q), to_dev(b.k_new), to_dev(b.v_new)
+    slots_d = torch.from_numpy(slots).to(dev)
+    tables_d = torch.from_numpy(tables).to(dev)
+    lens_d = torch.from_numpy(lens).to(dev)
+    out = torch.empty_like(q)
+    desc = pa.CacheDesc.make(num_blocks=b.num_blocks, block_size=Bs, num_kv_heads=Hkv,
+                             num_q_heads=Hq, head_dim=D, max_blocks_per_seq=MB)
+    kernel = {"auto": pa.PA_KERNEL_AUTO, "simt": pa.PA_KERNEL_SIMT,
+              "tensor": pa.PA_KERNEL_TENSOR}[args.kernel]
+    opts = pa.DecodeOptions(split_tokens=args.split_tokens, kernel=kernel)
+    wsb = pa.pa_decode_workspace_size(B, max_len, desc, opts)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    splits = pa.pa_decode_max_splits(B, max_len, desc, opts)
+
+    def step(i):
+        L = i % layers
+        pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
+        pa.pa_decode(q, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts,
+                     stream=stream)
+
+    # correctness guard before timing: the kernel must not report device errors
+    step(0)
+    torch.cuda.synchronize()
+    rc = pa.pa_decode_status(ws)
+    if rc != 0:
+        raise RuntimeError("decode reported %s" % pa.pa_status_string(rc))
+
+    for i in range(args.warmup):
+        step(i)
+    K = args.steps
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
+    t_start.record(stream)
+    for i in range(K):
+        L = i % layers
+        pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
+        ev_dec[i][0].record(stream)
+        pa.pa_decode(q, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts,
+                     stream=stream)
+        ev_dec[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = [s.elapsed_time(e) for s, e in ev_dec]
+    dec_avg_ms = float(np.mean(dec_ms))
+    if dist is not None:
+        t = torch.tensor([elapsed_ms, dec_avg_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, dec_avg_ms = float(t[0]), float(t[1])
+    rc = pa.pa_decode_status(ws)
+    if rc != 0:
+        raise RuntimeError("decode reported %s during timing" % pa.pa_status_string(rc))
+
+    value = world * B * K / (elapsed_ms / 1e3)
+
+    # ---- e2e: host buffers in, result out, every step -----------------------------------
+    E = args.e2e_steps
+    h_q = torch.from_numpy(b.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_k = torch.from_numpy(b.k_new.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_v = torch.from_numpy(b.v_new.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_slots = torch.from_numpy(slots).pin_memory()
+    h_tables = torch.from_numpy(tables).pin_memory()
+    h_lens = torch.from_numpy(lens).pin_memory()
+    h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+    d_slots, d_tables, d_lens = (torch.empty_like(slots_d), torch.empty_like(tables_d),
+                                 torch.empty_like(lens_d))
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_tables, h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step(i):
+        L = i % layers
+        for dst, src in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_slots, h_slots),
+                         (d_tables, h_tables), (d_lens, h_lens)):
+            dst.copy_(src, non_blocking=True)
+        pa.pa_append_kv(d_k, d_v, d_slots, kcs[L], vcs[L], desc, stream=stream)
+        pa.pa_decode(d_q, kcs[L], vcs[L], d_tables, d_lens, max_len, b.scale, out, ws, desc, opts,
+                     stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    for i in range(min(args.warmup, 20)):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(E):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = world * B * E / (e2e_ms / 1e3)
+
+    if rank != 0:
+        return None
+
+    kernel_name = "tensor" if kernel == pa.PA_KERNEL_TENSOR else "simt"
+    if kernel == pa.PA_KERNEL_AUTO:
+        kernel_name = os.environ.get("PA_DECODE_KERNEL", "simt")
+    peak, peak_kind = measured_peaks()
+    kv_bytes = kv_read_bytes(lens, Hkv, D)
+    achieved = kv_bytes / (dec_avg_ms / 1e3) / 1e9
+    res = {
+        "metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[args.config], "config": args.config,
+                   "batch": B, "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
+                   "block_size": Bs, "num_blocks": b.num_blocks, "mean_context": float(lens.mean()),
+                   "max_context": max_len, "decode_kernel": kernel_name,
+                   "split_tokens": args.split_tokens or "auto", "max_splits": splits,
+                   "l2": "inputs larger than L2: %d rotating layer pools of %.0f MB" % (layers, pool_bytes / 1e6),
+                   "parallelism": "replicas x%d" % world},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
+                     "traffic": profiled_traffic(args.config, kernel_name),
+                     "kernel": "pa_decode (%s)" % kernel_name,
+                     "algorithmic_bytes_per_launch": kv_bytes,
+                     "avg_launch_ms": dec_avg_ms},
+        "kv_read_gbs_step": kv_bytes * K / (elapsed_ms / 1e3) / 1e9,
+        "e2e": {"value": e2e_value, "unit": "seq-steps/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": E},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline(b, slots, tables, lens, args.cpu_seconds)
+    return res
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist_mod
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_mod
+    try:
+        res = run_ours(args, rank, world, dist)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,224 @@
+/*
+ * pa.h — C ABI of libpa: paged KV-cache append and paged decode attention
+ * for NVIDIA B200 (sm_100a), plus the host-side block manager that feeds them.
+ *
+ * Every entry point takes plain pointers and sizes.  Device pointers are
+ * CUDA device addresses owned by the caller; the library never allocates,
+ * frees or keeps device memory, and never synchronises unless a function says
+ * so.  `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ * stream); work is enqueued on it asynchronously.  Functions return a status
+ * code (PA_OK or a negative PA_ERR_*); no C++ exception crosses this ABI.
+ *
+ * bf16 tensors are passed as pa_bf16 (the raw 16-bit pattern: sign, 8-bit
+ * exponent, 7-bit mantissa — the upper half of an IEEE-754 float, as the
+ * Tiny-vLLM summary page "[Hacker News 요약] ... Tiny-vLLM ..." (aisleshub)
+ * describes bfloat16 in its section "모델 로딩 및 데이터 형식 심층 이해").
+ *
+ * Where the operations come from:
+ *  - Paging: page "vLLM — PagedAttention으로 LLM 추론 성능을 2~4배 끌어올린 서빙
+ *    엔진" (dev.to), section "PagedAttention — OS 가상 메모리에서 영감": the KV
+ *    cache is divided into fixed-size blocks handed out only as tokens arrive,
+ *    and logical blocks are mapped to non-contiguous physical blocks.
+ *  - KV cache and attention: same page, section "KV Cache가 왜 병목인가", and
+ *    the Tiny-vLLM summary page, section "고성능 추론을 위한 고급 최적화 기법":
+ *    K/V of earlier tokens are stored and re-read at every decode step;
+ *    attention is softmax(q K^T * scale) V; grouped-query attention lets
+ *    several query heads share one K/V head; the causal mask lets the decode
+ *    query (the newest position) see every cached token.
+ *  - Block manager: page "Nano-vLLM로 배우는 vLLM 추론 엔진 작동 원리 한눈에
+ *    정리" (tilnote.io), section "KV 캐시와 Block Manager": fixed-size blocks,
+ *    metadata on the CPU, K/V tensors on the GPU, shared prefix blocks.
+ *  - Decode is memory-bound (dev.to page, section "Prefill vs Decode"), which
+ *    is why the decode kernel streams each K/V page from HBM once per kv head
+ *    and splits long contexts across CTAs.
+ *
+ * Layouts (all row-major, contiguous):
+ *   k_cache, v_cache  [num_blocks][num_kv_heads][block_size][head_dim] bf16
+ *   q, out            [num_seqs][num_q_heads][head_dim]               bf16
+ *   k, v (append)     [num_tokens][num_kv_heads][head_dim]            bf16
+ *   slot_mapping      [num_tokens] int64: slot = block * block_size + offset
+ *   block_tables      [num_seqs][max_blocks_per_seq] int32: physical block of
+ *                     logical block i; entries past a sequence's last block
+ *                     are never read
+ *   context_lens      [num_seqs] int32: tokens the decode query attends to,
+ *                     the token appended this step included
+ * Query head h reads kv head h / (num_q_heads / num_kv_heads).
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+typedef uint16_t pa_bf16;
+
+/* ---- status codes ---------------------------------------------------------------------- */
+#define PA_OK                 0
+#define PA_ERR_INVALID       -1  /* null pointer, bad size, misaligned pointer, Hq % Hkv != 0 */
+#define PA_ERR_UNSUPPORTED   -2  /* well-formed but outside the built shapes (see pa_decode) */
+#define PA_ERR_CUDA          -3  /* a CUDA runtime call or kernel launch failed */
+#define PA_ERR_WORKSPACE     -4  /* workspace missing, misaligned or smaller than required */
+#define PA_ERR_OOM_BLOCKS    -5  /* block manager: not enough free blocks */
+#define PA_ERR_SHARED_BLOCK  -6  /* block manager: append into a block that several tables hold */
+#define PA_ERR_BAD_BLOCK     -7  /* decode saw a block id outside [0, num_blocks) */
+#define PA_ERR_BAD_LENGTH    -8  /* decode saw a context length above max_context_len or the table */
+#define PA_ERR_TIMEOUT       -9  /* a bounded wait inside a kernel gave up */
+
+/* Human-readable name of a status code (static string, never NULL). */
+PA_API const char* pa_status_string(int status);
+
+/* ---- pool geometry ---------------------------------------------------------------------- */
+typedef struct pa_cache_desc {
+    int32_t num_blocks;          /* N: physical blocks in each cache tensor                   */
+    int32_t block_size;          /* Bs: tokens per block                                       */
+    int32_t num_kv_heads;        /* Hkv                                                        */
+    int32_t num_q_heads;         /* Hq, a multiple of Hkv                                      */
+    int32_t head_dim;            /* D                                                          */
+    int32_t max_blocks_per_seq;  /* MB: row stride of block_tables                             */
+} pa_cache_desc;
+
+/* ---- KV append ------------------------------------------------------------------------- */
+/*
+ * Writes token t's K and V rows (all kv heads) into slot slot_mapping[t] of
+ * k_cache / v_cache: block s / Bs, offset s % Bs.  A negative slot, or one
+ * at or past num_blocks * block_size, writes nothing.  The copy is bit-exact;
+ * no other byte of the caches changes.  Two tokens mapped to the same slot
+ * race (the survivor is unspecified).
+ * Requirements: head_dim a multiple of 8; k, v, k_cache, v_cache 16-byte
+ * aligned.  num_tokens == 0 is a no-op.
+ * Errors: PA_ERR_INVALID (arguments), PA_ERR_CUDA (launch).
+ */
+PA_API int pa_append_kv(const pa_bf16* k, const pa_bf16* v, const int64_t* slot_mapping,
+                 int32_t num_tokens, pa_bf16* k_cache, pa_bf16* v_cache,
+                 const pa_cache_desc* desc, void* stream);
+
+/* ---- paged decode attention ------------------------------------------------------------ */
+#define PA_KERNEL_AUTO    0   /* the fastest built kernel for the shape                         */
+#define PA_KERNEL_SIMT    1   /* CUDA-core kernel: plain loads, fp32 FMA                         */
+#define PA_KERNEL_TENSOR  2   /* TMA-staged pages, q.K and p.V on tensor cores (mma.sync bf16)   */
+
+#define PA_FLAG_CHECK     1   /* synchronise after the launch and report device-side errors     */
+
+typedef struct pa_decode_options {
+    int32_t split_tokens;  /* 0: automatic; else tokens per KV split, a positive multiple of 64 */
+    int32_t kernel;        /* PA_KERNEL_*                                                        */
+    int32_t flags;         /* PA_FLAG_*                                                          */
+    int32_t reserved;      /* must be 0                                                          */
+} pa_decode_options;
+
+/*
+ * Bytes of device workspace pa_decode needs for this batch shape (0 on bad
+ * arguments).  max_context_len is an upper bound of every context_lens[b].
+ * Needs a current CUDA device (the split plan depends on its SM count).
+ */
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t max_context_len,
+                                const pa_cache_desc* desc);
+PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_len,
+                                   const pa_cache_desc* desc, const pa_decode_options* options);
+
+/*
+ * Paged decode attention: for every sequence b and query head h,
+ *   out[b][h] = bf16( sum_j p_j V_j ),  p = softmax_j(scale * q[b][h] . K_j),
+ * over the context_lens[b] tokens the table row block_tables[b] reaches,
+ * with K_j, V_j the rows of kv head h / (Hq/Hkv).  fp32 accumulation, online
+ * softmax, the result rounded to nearest-even bf16.  A sequence with
+ * context_lens[b] == 0 outputs zeros.  Long contexts are split across CTAs;
+ * the partial states are merged (log-sum-exp) inside the same launch.
+ *
+ * workspace: caller-owned device buffer of at least
+ * pa_decode_workspace_size(...) bytes, 256-byte aligned, ZERO-FILLED BEFORE
+ * ITS FIRST USE.  The kernel leaves its counters at zero when it completes,
+ * so the buffer can be reused by later calls without clearing; calls that
+ * may overlap on the GPU need separate workspaces.
+ *
+ * Built shapes: head_dim 64 or 128; block_size 8, 16, 32, 64, 128 or 256;
+ * Hq / Hkv <= 16.  Others return PA_ERR_UNSUPPORTED.  Pointers q, out,
+ * k_cache, v_cache must be 16-byte aligned.
+ * A block id outside [0, num_blocks) is read as zeros and a length above
+ * max_context_len or the table is clipped; both raise a bit in the
+ * workspace's status word, which pa_decode_status reports (PA_FLAG_CHECK
+ * does so before returning).
+ */
+PA_API int pa_decode(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
+              const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+              int32_t max_context_len, float scale, pa_bf16* out, void* workspace,
+              size_t workspace_bytes, const pa_cache_desc* desc, void* stream);
+PA_API int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
+                 const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+                 int32_t max_context_len, float scale, pa_bf16* out, void* workspace,
+                 size_t workspace_bytes, const pa_cache_desc* desc,
+                 const pa_decode_options* options, void* stream);
+
+/*
+ * Synchronises `stream`, reads and clears the workspace's device status word.
+ * Returns PA_OK, PA_ERR_BAD_BLOCK, PA_ERR_BAD_LENGTH or PA_ERR_TIMEOUT (the
+ * first set, in that order), or PA_ERR_CUDA if the read fails.
+ */
+PA_API int pa_decode_status(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Number of KV splits pa_decode uses per (sequence, kv head) at most for this shape. */
+PA_API int32_t pa_decode_max_splits(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc* desc,
+                             const pa_decode_options* options);
+
+/* ---- host slot mapping ----------------------------------------------------------------- */
+/*
+ * slots[b] = block_tables[b][p / Bs] * Bs + p % Bs with p = lengths[b] - 1
+ * (the newest token's slot), or -1 when lengths[b] <= 0.  Host memory only.
+ */
+PA_API int pa_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* lengths, int32_t num_seqs, int32_t block_size, int64_t* slots);
+
+/* ---- host block manager ---------------------------------------------------------------- */
+/*
+ * Host-memory bookkeeping of a block pool shared by up to max_seqs sequence
+ * rows.  Policy: free blocks form a stack, free_order[0] handed out first; a
+ * block's reference count is the number of tables holding it and it returns
+ * to the top of the stack when the count reaches zero; releasing a sequence
+ * walks its table from logical block 0; appending a token at position p takes
+ * a block when p % Bs == 0; a batch append is all-or-nothing; an append into
+ * a block held by more than one table is refused (PA_ERR_SHARED_BLOCK).
+ * Not thread-safe: one manager per thread.
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+PA_API int pa_bm_create(int32_t num_blocks, int32_t block_size, int32_t max_seqs,
+                 int32_t max_blocks_per_seq, const int32_t* free_order, int32_t num_free,
+                 pa_block_manager** out);
+PA_API void pa_bm_destroy(pa_block_manager* bm);
+/* Adopt a sequence whose num_tokens tokens already sit in `blocks` (ceil(num_tokens/Bs)
+ * ids that are not on the free stack); each block's count rises by one. */
+PA_API int pa_bm_import_seq(pa_block_manager* bm, int32_t seq, int32_t num_tokens, const int32_t* blocks);
+/* Admit a sequence of num_tokens cached tokens into fresh blocks. */
+PA_API int pa_bm_add_seq(pa_block_manager* bm, int32_t seq, int32_t num_tokens);
+/* Admit a sequence that shares the first num_shared_blocks blocks of src (which must be
+ * full) and gets fresh blocks for the rest of its num_tokens tokens. */
+PA_API int pa_bm_fork_seq(pa_block_manager* bm, int32_t seq, int32_t src, int32_t num_shared_blocks,
+                   int32_t num_tokens);
+/* Release a sequence's blocks. */
+PA_API int pa_bm_free_seq(pa_block_manager* bm, int32_t seq);
+/* One new token for each of the n (distinct) listed sequences; slots[i] receives its slot. */
+PA_API int pa_bm_append_tokens(pa_block_manager* bm, const int32_t* seqs, int32_t n, int64_t* slots);
+PA_API int32_t pa_bm_num_free(const pa_block_manager* bm);
+PA_API int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
+/* Host views, valid until the manager is destroyed: [max_seqs][max_blocks_per_seq] (-1
+ * past each sequence's blocks) and [max_seqs] (0 for rows without a sequence). */
+PA_API const int32_t* pa_bm_block_tables(const pa_block_manager* bm);
+PA_API const int32_t* pa_bm_context_lens(const pa_block_manager* bm);
+/* Rows whose table changed since the last call (up to cap, ascending); returns the count. */
+PA_API int32_t pa_bm_take_dirty_rows(pa_block_manager* bm, int32_t* rows, int32_t cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

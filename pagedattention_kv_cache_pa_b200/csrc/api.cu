@@ -1,0 +1,270 @@
+// C-ABI entry points of libpa: argument checks, the split plan, dispatch.
+// The kernels themselves live in append.cu, decode_simt.cu and decode_tensor.cu.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool supported_block_size(int32_t bs) {
+    return bs == 8 || bs == 16 || bs == 32 || bs == 64 || bs == 128 || bs == 256;
+}
+
+int check_desc(const pa_cache_desc* d) {
+    if (!d) return PA_ERR_INVALID;
+    if (d->num_blocks <= 0 || d->block_size <= 0 || d->num_kv_heads <= 0 ||
+        d->num_q_heads <= 0 || d->head_dim <= 0 || d->max_blocks_per_seq <= 0)
+        return PA_ERR_INVALID;
+    if (d->num_q_heads % d->num_kv_heads != 0) return PA_ERR_INVALID;
+    if ((int64_t)d->num_blocks * d->num_kv_heads * d->block_size > (int64_t)INT32_MAX)
+        return PA_ERR_UNSUPPORTED;  // row index of the pool must fit in 32 bits
+    return PA_OK;
+}
+
+// Optional override of the automatic split size, for tuning sweeps.
+int32_t env_split_tokens() {
+    static int32_t v = [] {
+        const char* s = getenv("PA_SPLIT_TOKENS");
+        return s ? (int32_t)atoi(s) : 0;
+    }();
+    return v;
+}
+
+int32_t env_kernel() {
+    static int32_t v = [] {
+        const char* s = getenv("PA_DECODE_KERNEL");
+        if (!s) return (int32_t)PA_KERNEL_AUTO;
+        if (!strcmp(s, "simt")) return (int32_t)PA_KERNEL_SIMT;
+        if (!strcmp(s, "tensor")) return (int32_t)PA_KERNEL_TENSOR;
+        return (int32_t)PA_KERNEL_AUTO;
+    }();
+    return v;
+}
+
+}  // namespace
+
+int num_sms_current_device(int* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int cached = g_sm_count[dev].load(std::memory_order_relaxed);
+        if (cached > 0) {
+            *out = cached;
+            return PA_OK;
+        }
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return PA_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(n, std::memory_order_relaxed);
+    *out = n;
+    return PA_OK;
+}
+
+// Split plan: tokens per split C (a multiple of 64) and the grid's split count.
+// Automatic choice: enough (sequence, kv head, split) work items for about
+// 32 per SM if every sequence were max_context_len long, never below 128
+// tokens per split.
+int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc& d,
+                     const pa_decode_options* opt, DecodePlan* plan) {
+    int32_t C = opt ? opt->split_tokens : 0;
+    if (C == 0) C = env_split_tokens();
+    if (C < 0 || C % 64 != 0) return PA_ERR_INVALID;
+    if (C == 0) {
+        int sms = 0;
+        const int rc = num_sms_current_device(&sms);
+        if (rc != PA_OK) return rc;
+        const int64_t work = (int64_t)num_seqs * d.num_kv_heads * (max_context_len > 0 ? max_context_len : 1);
+        int64_t c = ceil_div(work, (int64_t)sms * 32);
+        c = ceil_div(c, 64) * 64;
+        if (c < 128) c = 128;
+        C = (int32_t)(c > (1 << 30) ? (1 << 30) : c);
+    }
+    int32_t kernel = opt ? opt->kernel : PA_KERNEL_AUTO;
+    if (kernel == PA_KERNEL_AUTO) kernel = env_kernel();
+    if (kernel == PA_KERNEL_AUTO) kernel = PA_KERNEL_SIMT;
+    plan->kernel = kernel;
+    plan->split_tokens = C;
+    plan->max_splits = (int32_t)(max_context_len > 0 ? ceil_div(max_context_len, C) : 1);
+    const int32_t G = d.num_q_heads / d.num_kv_heads;
+    const size_t pairs = (size_t)num_seqs * d.num_kv_heads;
+    auto up = [](size_t x) { return (x + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign; };
+    plan->off_counters = kWorkspaceAlign;  // [0, 256): status word
+    size_t off = plan->off_counters + up(pairs * sizeof(int32_t));
+    plan->off_lse = off;
+    if (plan->max_splits > 1) {
+        off += up(pairs * plan->max_splits * G * sizeof(float));
+        plan->off_o = off;
+        off += up(pairs * plan->max_splits * G * (size_t)d.head_dim * sizeof(float));
+    } else {
+        plan->off_o = off;
+    }
+    plan->bytes = off;
+    return PA_OK;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" const char* pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID: return "PA_ERR_INVALID: invalid argument";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: shape not built";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime error";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case PA_ERR_OOM_BLOCKS: return "PA_ERR_OOM_BLOCKS: not enough free blocks";
+        case PA_ERR_SHARED_BLOCK: return "PA_ERR_SHARED_BLOCK: append into a shared block";
+        case PA_ERR_BAD_BLOCK: return "PA_ERR_BAD_BLOCK: block id outside the pool";
+        case PA_ERR_BAD_LENGTH: return "PA_ERR_BAD_LENGTH: context length beyond the bound";
+        case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT: a bounded wait in a kernel gave up";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int pa_append_kv(const pa_bf16* k, const pa_bf16* v, const int64_t* slot_mapping,
+                            int32_t num_tokens, pa_bf16* k_cache, pa_bf16* v_cache,
+                            const pa_cache_desc* desc, void* stream) {
+    int rc = check_desc(desc);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0) return PA_ERR_INVALID;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID;
+    if (desc->head_dim % 8 != 0) return PA_ERR_INVALID;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 8))
+        return PA_ERR_INVALID;
+    const cudaError_t e = launch_append(k, v, slot_mapping, num_tokens, k_cache, v_cache, *desc,
+                                        (cudaStream_t)stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+static int check_decode_shape(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc* d) {
+    int rc = check_desc(d);
+    if (rc != PA_OK) return rc;
+    if (num_seqs < 0 || num_seqs > 65535 || max_context_len < 0) return PA_ERR_INVALID;
+    if (d->head_dim != 64 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (!supported_block_size(d->block_size)) return PA_ERR_UNSUPPORTED;
+    if (d->num_q_heads / d->num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+    if (d->num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+extern "C" size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_len,
+                                              const pa_cache_desc* desc,
+                                              const pa_decode_options* options) {
+    if (check_decode_shape(num_seqs, max_context_len, desc) != PA_OK) return 0;
+    DecodePlan plan;
+    if (make_decode_plan(num_seqs, max_context_len, *desc, options, &plan) != PA_OK) return 0;
+    return plan.bytes;
+}
+
+extern "C" size_t pa_decode_workspace_size(int32_t num_seqs, int32_t max_context_len,
+                                           const pa_cache_desc* desc) {
+    return pa_decode_workspace_size_ex(num_seqs, max_context_len, desc, nullptr);
+}
+
+extern "C" int32_t pa_decode_max_splits(int32_t num_seqs, int32_t max_context_len,
+                                        const pa_cache_desc* desc,
+                                        const pa_decode_options* options) {
+    if (check_decode_shape(num_seqs, max_context_len, desc) != PA_OK) return -1;
+    DecodePlan plan;
+    if (make_decode_plan(num_seqs, max_context_len, *desc, options, &plan) != PA_OK) return -1;
+    return plan.max_splits;
+}
+
+extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            int32_t num_seqs, int32_t max_context_len, float scale, pa_bf16* out,
+                            void* workspace, size_t workspace_bytes, const pa_cache_desc* desc,
+                            const pa_decode_options* options, void* stream) {
+    int rc = check_decode_shape(num_seqs, max_context_len, desc);
+    if (rc != PA_OK) return rc;
+    if (options && (options->reserved != 0 || options->kernel < 0 || options->kernel > 2))
+        return PA_ERR_INVALID;
+    if (num_seqs == 0) return PA_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+        return PA_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4))
+        return PA_ERR_INVALID;
+    DecodePlan plan;
+    rc = make_decode_plan(num_seqs, max_context_len, *desc, options, &plan);
+    if (rc != PA_OK) return rc;
+    if (!workspace || !aligned(workspace, kWorkspaceAlign) || workspace_bytes < plan.bytes)
+        return PA_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    DecodeParams p;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = out;
+    p.status = reinterpret_cast<int32_t*>(ws);
+    p.counters = reinterpret_cast<int32_t*>(ws + plan.off_counters);
+    p.part_lse = reinterpret_cast<float*>(ws + plan.off_lse);
+    p.part_o = reinterpret_cast<float*>(ws + plan.off_o);
+    p.num_seqs = num_seqs;
+    p.num_blocks = desc->num_blocks;
+    p.block_size = desc->block_size;
+    p.num_kv_heads = desc->num_kv_heads;
+    p.num_q_heads = desc->num_q_heads;
+    p.head_dim = desc->head_dim;
+    p.group = desc->num_q_heads / desc->num_kv_heads;
+    p.max_blocks_per_seq = desc->max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.split_tokens = plan.split_tokens;
+    p.max_splits = plan.max_splits;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    cudaError_t e;
+    if (plan.kernel == PA_KERNEL_TENSOR && tensor_kernel_supports(p)) {
+        e = launch_decode_tensor(p, (cudaStream_t)stream);
+    } else {
+        e = launch_decode_simt(p, (cudaStream_t)stream);
+    }
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    if (options && (options->flags & PA_FLAG_CHECK))
+        return pa_decode_status(workspace, workspace_bytes, stream);
+    return PA_OK;
+}
+
+extern "C" int pa_decode(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens,
+                         int32_t num_seqs, int32_t max_context_len, float scale, pa_bf16* out,
+                         void* workspace, size_t workspace_bytes, const pa_cache_desc* desc,
+                         void* stream) {
+    return pa_decode_ex(q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                        max_context_len, scale, out, workspace, workspace_bytes, desc, nullptr,
+                        stream);
+}
+
+extern "C" int pa_decode_status(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < sizeof(int32_t)) return PA_ERR_WORKSPACE;
+    int32_t word = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof word, s) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+    if (word & kStatusBadBlock) return PA_ERR_BAD_BLOCK;
+    if (word & kStatusBadLength) return PA_ERR_BAD_LENGTH;
+    if (word & kStatusTimeout) return PA_ERR_TIMEOUT;
+    return PA_OK;
+}

@@ -1,0 +1,61 @@
+// KV-cache append: scatter each new token's K/V rows into its slot.
+//
+// The KV cache keeps the K/V projections of earlier tokens so a decode step
+// does not recompute them (Tiny-vLLM summary page, section "고성능 추론을 위한
+// 고급 최적화 기법"; dev.to vLLM page, section "KV Cache가 왜 병목인가").  With
+// paging, a token's storage is a slot: block s / Bs, offset s % Bs of the pool
+// (dev.to page, section "PagedAttention — OS 가상 메모리에서 영감").
+//
+// One thread moves one 16-byte chunk of K and the same chunk of V, so a warp
+// writes whole 128-byte rows (D = 64) with coalesced 16-byte stores.  Pure
+// copy: the result is bit-identical to the input rows.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+__global__ void __launch_bounds__(256) append_kv_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, const int64_t* __restrict__ slots,
+    int64_t chunks, int32_t chunks_per_row, int32_t num_kv_heads, int32_t block_size,
+    int64_t num_slots, uint4* __restrict__ k_cache, uint4* __restrict__ v_cache) {
+    const int64_t per_token = (int64_t)num_kv_heads * chunks_per_row;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / per_token;
+        const int64_t within = i - t * per_token;          // h * chunks_per_row + c
+        const int64_t slot = slots[t];
+        if (slot < 0 || slot >= num_slots) continue;
+        const int64_t blk = slot / block_size;
+        const int64_t off = slot - blk * block_size;
+        const int64_t h = within / chunks_per_row;
+        const int64_t c = within - h * chunks_per_row;
+        const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * chunks_per_row + c;
+        const uint4 kk = __ldg(k + i);
+        const uint4 vv = __ldg(v + i);
+        k_cache[dst] = kk;
+        v_cache[dst] = vv;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const pa_bf16* k, const pa_bf16* v, const int64_t* slots, int32_t T,
+                          pa_bf16* k_cache, pa_bf16* v_cache, const pa_cache_desc& d,
+                          cudaStream_t stream) {
+    const int32_t chunks_per_row = d.head_dim / 8;
+    const int64_t chunks = (int64_t)T * d.num_kv_heads * chunks_per_row;
+    if (chunks == 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t blocks = (chunks + threads - 1) / threads;
+    if (blocks > 148 * 32) blocks = 148 * 32;  // grid-stride beyond 32 CTAs per SM
+    append_kv_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), slots, chunks,
+        chunks_per_row, d.num_kv_heads, d.block_size, (int64_t)d.num_blocks * d.block_size,
+        reinterpret_cast<uint4*>(k_cache), reinterpret_cast<uint4*>(v_cache));
+    return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,65 @@
+// Internal declarations shared by the libpa translation units (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+// Bits of the device status word (first int32 of the decode workspace).
+enum : int32_t {
+    kStatusBadBlock = 1,
+    kStatusBadLength = 2,
+    kStatusTimeout = 4,
+};
+
+// Everything a decode kernel reads; passed by value as the kernel parameter.
+struct DecodeParams {
+    const uint16_t* q;             // [B][Hq][D]
+    const uint16_t* k_cache;       // [N][Hkv][Bs][D]
+    const uint16_t* v_cache;
+    const int32_t* block_tables;   // [B][MB]
+    const int32_t* context_lens;   // [B]
+    uint16_t* out;                 // [B][Hq][D]
+    int32_t* status;               // device status word
+    int32_t* counters;             // [B][Hkv] split arrival counters (self-resetting)
+    float* part_lse;               // [B][Hkv][S][G] log2-domain log-sum-exp
+    float* part_o;                 // [B][Hkv][S][G][D] normalised partial outputs
+    int32_t num_seqs;
+    int32_t num_blocks;
+    int32_t block_size;
+    int32_t num_kv_heads;
+    int32_t num_q_heads;
+    int32_t head_dim;
+    int32_t group;                 // Hq / Hkv
+    int32_t max_blocks_per_seq;
+    int32_t max_context_len;
+    int32_t split_tokens;          // C: tokens per split (multiple of 64)
+    int32_t max_splits;            // S = ceil(max_context_len / C)
+    float scale_log2;              // scale * log2(e): scores are kept in the log2 domain
+};
+
+struct DecodePlan {
+    int32_t split_tokens;
+    int32_t max_splits;
+    int32_t kernel;                // PA_KERNEL_SIMT or PA_KERNEL_TENSOR
+    size_t off_counters, off_lse, off_o, bytes;
+};
+
+constexpr size_t kWorkspaceAlign = 256;
+
+int num_sms_current_device(int* out);
+int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc& d,
+                     const pa_decode_options* opt, DecodePlan* plan);
+
+cudaError_t launch_append(const pa_bf16* k, const pa_bf16* v, const int64_t* slots, int32_t T,
+                          pa_bf16* k_cache, pa_bf16* v_cache, const pa_cache_desc& d,
+                          cudaStream_t stream);
+cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_decode_tensor(const DecodeParams& p, cudaStream_t stream);
+bool tensor_kernel_supports(const DecodeParams& p);
+
+}  // namespace pa

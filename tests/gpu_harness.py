@@ -1,0 +1,95 @@
+"""Shared plumbing of the GPU parity tests: one decode step through the C ABI
+next to the same step through the oracle, on identical seeded inputs.
+
+Step = (a1) the host block manager gives each sequence a block if its last one
+is full, (a2) the newest token's slot, (a3) KV append, (a4-a10) paged decode.
+The product side uses libpa (C++ block manager + CUDA kernels); the oracle side
+uses oracle.BlockManagerModel + the C oracle.  Nothing flows from the product
+side into the oracle side.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import workloads as wl
+import pagedattention_kv_cache_pa_b200 as pa
+
+DEV = torch.device("cuda:0")
+
+
+def to_dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(DEV)
+
+
+def to_host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def desc_of(b: wl.DecodeBatch, max_blocks_per_seq=None) -> pa.CacheDesc:
+    return pa.CacheDesc.make(num_blocks=b.num_blocks, block_size=b.block_size,
+                             num_kv_heads=b.num_kv_heads, num_q_heads=b.num_q_heads,
+                             head_dim=b.head_dim,
+                             max_blocks_per_seq=max_blocks_per_seq or b.max_blocks_per_seq)
+
+
+def host_step(b: wl.DecodeBatch):
+    """(a1, a2) on both sides; returns product (slots, tables, lens) and oracle ones."""
+    B, Bs, MB = b.batch, b.block_size, b.max_blocks_per_seq
+    bm = pa.BlockManager(b.num_blocks, Bs, B, MB, b.free_order)
+    model = oracle.BlockManagerModel(b.num_blocks, Bs, B, MB, b.free_order)
+    for s in range(B):
+        L = int(b.context_lens[s])
+        blocks = b.block_tables[s, : -(-L // Bs)]
+        bm.import_seq(s, L, blocks)
+        model.import_seq(s, L, blocks)
+    slots = bm.append_tokens(np.arange(B, dtype=np.int32))
+    tables = bm.block_tables().copy()
+    lens = bm.context_lens().copy()
+    bm.close()
+    o_slots = np.array(model.append_tokens(list(range(B))), dtype=np.int64)
+    o_tables = np.array([model.table_array(s) for s in range(B)], dtype=np.int32)
+    o_lens = np.array(model.lens, dtype=np.int32)
+    return (slots, tables, lens), (o_slots, o_tables, o_lens)
+
+
+def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int = 0,
+             check_pool: bool = True, sample=None):
+    """Runs one step on both sides; returns a dict of results and checks."""
+    (slots, tables, lens), (o_slots, o_tables, o_lens) = host_step(b)
+    assert np.array_equal(slots, o_slots), "slot mapping differs from the model"
+    assert np.array_equal(tables, o_tables), "block tables differ from the model"
+    assert np.array_equal(lens, o_lens)
+    assert np.array_equal(slots, oracle.slot_mapping(o_tables, o_lens, b.block_size))
+
+    desc = desc_of(b)
+    k_cache, v_cache = to_dev(b.k_cache), to_dev(b.v_cache)
+    q = to_dev(b.q)
+    out = torch.empty_like(q)
+    max_len = int(lens.max()) if lens.size else 0
+    opts = pa.DecodeOptions(split_tokens=split_tokens, kernel=kernel, flags=pa.PA_FLAG_CHECK)
+    ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, max_len, desc, opts), dtype=torch.uint8,
+                     device=DEV)
+    pa.pa_append_kv(to_dev(b.k_new), to_dev(b.v_new), torch.from_numpy(slots).to(DEV), k_cache,
+                    v_cache, desc)
+    pa.pa_decode(q, k_cache, v_cache, torch.from_numpy(tables).to(DEV),
+                 torch.from_numpy(lens).to(DEV), max_len, b.scale, out, ws, desc, opts)
+    torch.cuda.synchronize()
+
+    ref_k, ref_v = oracle.append_kv(b.k_new, b.v_new, o_slots, b.k_cache, b.v_cache)
+    res = {"splits": pa.pa_decode_max_splits(b.batch, max_len, desc, opts)}
+    if check_pool:
+        res["pool_equal"] = (np.array_equal(to_host_bits(k_cache), ref_k) and
+                             np.array_equal(to_host_bits(v_cache), ref_v))
+    got = out.float().cpu().numpy().astype(np.float64)
+    if sample is None:
+        ref = oracle.paged_decode(b.q, ref_k, ref_v, o_tables, o_lens, b.scale)
+        res["ok"], res["excess"] = oracle.within_tolerance(got, ref)
+    else:
+        idx = np.asarray(sample)
+        ref = oracle.paged_decode(b.q[idx], ref_k, ref_v, o_tables[idx], o_lens[idx], b.scale)
+        res["ok"], res["excess"] = oracle.within_tolerance(got[idx], ref)
+    res["out"] = got
+    res["finite"] = bool(np.isfinite(got).all())
+    return res

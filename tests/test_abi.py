@@ -1,0 +1,83 @@
+"""The C-ABI library loads, exports what include/pa.h declares, and rejects bad
+arguments before touching a GPU (CPU only: no compute call runs here)."""
+import ctypes
+import subprocess
+
+import numpy as np
+import pytest
+
+import pagedattention_kv_cache_pa_b200 as pa
+from pagedattention_kv_cache_pa_b200 import binding
+
+
+def test_every_declared_symbol_is_exported():
+    declared = pa.declared_symbols()
+    assert len(declared) >= 20
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [s for s in declared if s not in exported]
+    assert not missing, missing
+    for s in declared:
+        assert hasattr(binding.lib, s)
+    # nothing beyond the declared ABI leaks out
+    assert exported == set(declared), sorted(exported - set(declared))
+
+
+def test_status_strings():
+    for code in range(-9, 1):
+        assert binding.STATUS[code] in pa.pa_status_string(code)
+    assert "unknown" in pa.pa_status_string(-1234)
+
+
+def _desc(**kw):
+    base = dict(num_blocks=8, block_size=16, num_kv_heads=1, num_q_heads=2, head_dim=64,
+                max_blocks_per_seq=4)
+    base.update(kw)
+    return pa.CacheDesc.make(**base)
+
+
+def test_append_rejects_bad_arguments_without_a_gpu():
+    lib = binding.lib
+    d = _desc()
+    fake = ctypes.c_void_p(0x10000)          # never dereferenced: validation fails first
+    assert lib.pa_append_kv(None, fake, fake, 1, fake, fake, ctypes.byref(d), None) == -1
+    assert lib.pa_append_kv(fake, fake, fake, -1, fake, fake, ctypes.byref(d), None) == -1
+    assert lib.pa_append_kv(fake, fake, fake, 0, fake, fake, ctypes.byref(d), None) == 0  # no-op
+    assert lib.pa_append_kv(fake, fake, fake, 1, fake, fake, None, None) == -1
+    bad = _desc(num_q_heads=3, num_kv_heads=2)
+    assert lib.pa_append_kv(fake, fake, fake, 1, fake, fake, ctypes.byref(bad), None) == -1
+    odd = _desc(head_dim=60)
+    assert lib.pa_append_kv(fake, fake, fake, 1, fake, fake, ctypes.byref(odd), None) == -1
+    mis = ctypes.c_void_p(0x10002)
+    assert lib.pa_append_kv(mis, fake, fake, 1, fake, fake, ctypes.byref(d), None) == -1
+
+
+def test_decode_rejects_unsupported_shapes_without_a_gpu():
+    lib = binding.lib
+    fake = ctypes.c_void_p(0x10000)
+    for kw, want in ((dict(head_dim=96), -2), (dict(block_size=12), -2),
+                     (dict(num_q_heads=34, num_kv_heads=2), -2), (dict(num_q_heads=3, num_kv_heads=2), -1)):
+        d = _desc(**kw)
+        rc = lib.pa_decode(fake, fake, fake, fake, fake, 1, 16, ctypes.c_float(0.1), fake, fake, 1 << 20,
+                           ctypes.byref(d), None)
+        assert rc == want, (kw, rc)
+    d = _desc()
+    assert lib.pa_decode(fake, fake, fake, fake, fake, -1, 16, ctypes.c_float(0.1), fake, fake, 0,
+                         ctypes.byref(d), None) == -1
+    assert lib.pa_decode(fake, fake, fake, fake, fake, 0, 16, ctypes.c_float(0.1), fake, fake, 0,
+                         ctypes.byref(d), None) == 0   # empty batch: nothing to do
+    opts = pa.DecodeOptions(split_tokens=100)          # not a multiple of 64
+    assert lib.pa_decode_max_splits(1, 16, ctypes.byref(d), ctypes.byref(opts)) == -1
+    opts = pa.DecodeOptions(split_tokens=128)          # explicit: no device query needed
+    assert lib.pa_decode_max_splits(1, 1000, ctypes.byref(d), ctypes.byref(opts)) == 8
+    assert pa.pa_decode_workspace_size(2, 1000, d, opts) > 0
+
+
+def test_slot_mapping_entry_matches_oracle():
+    import oracle
+    rng = np.random.default_rng(0)
+    tables = rng.integers(0, 1000, size=(50, 20)).astype(np.int32)
+    lens = rng.integers(0, 20 * 16 + 1, size=50).astype(np.int32)
+    np.testing.assert_array_equal(pa.pa_slot_mapping(tables, lens, 16),
+                                  oracle.slot_mapping(tables, lens, 16))

@@ -1,0 +1,201 @@
+"""CUDA path vs fp64 oracle through the C ABI (needs a B200).
+
+Append: bit-exact, everywhere in the pool.  Decode: |gpu - oracle| <= 1e-2 +
+1e-2 * |oracle| elementwise (the tolerance the workload statement fixes).
+Both decode kernels (CUDA-core and tensor-core) are checked on every case.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+import pagedattention_kv_cache_pa_b200 as pa
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = [pa.PA_KERNEL_SIMT, pa.PA_KERNEL_TENSOR]
+KNAMES = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR: "tensor"}
+
+
+@pytest.fixture(scope="module")
+def h():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tests import gpu_harness
+    return gpu_harness
+
+
+def _assert(res):
+    assert res["pool_equal"], "append is not bit-exact"
+    assert res["finite"]
+    assert res["ok"], "decode outside tolerance by %g" % res["excess"]
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+def test_c1_tiny(h, kernel):
+    _assert(h.run_step(wl.config1(), kernel=kernel))
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+@pytest.mark.parametrize("split", [0, 64, 256])
+def test_c2_llama_1b_layer(h, kernel, split):
+    res = h.run_step(wl.config2(), kernel=kernel, split_tokens=split)
+    _assert(res)
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+def test_c3_shared_prefix_bs256(h, kernel):
+    _assert(h.run_step(wl.config3(), kernel=kernel))
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+def test_c4_long_context_split(h, kernel):
+    res = h.run_step(wl.config4(), kernel=kernel)
+    assert res["splits"] > 1
+    _assert(res)
+
+
+EDGE_SHAPES = [
+    # (Hq, Hkv, D, Bs)
+    (4, 2, 64, 16), (8, 1, 128, 16), (3, 1, 64, 8), (16, 1, 64, 32), (6, 3, 128, 64),
+    (32, 8, 64, 128), (2, 2, 64, 256), (16, 2, 128, 8),
+]
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+@pytest.mark.parametrize("shape", EDGE_SHAPES, ids=lambda s: "Hq%d-Hkv%d-D%d-Bs%d" % s)
+def test_edge_lengths(h, kernel, shape):
+    Hq, Hkv, D, Bs = shape
+    # cached lengths around block and split edges (appended token makes +1)
+    lens = sorted({0, 1, Bs - 2, Bs - 1, Bs, 62, 63, 64, 65, 127, 128, 129, 300, 511, 777})
+    lens = [x for x in lens if x >= 0]
+    b = wl.small_batch(1000 + Bs + D + Hq, lens, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                       block_size=Bs)
+    for split in (64, 128, 0):
+        _assert(h.run_step(b, kernel=kernel, split_tokens=split))
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+def test_empty_context_outputs_zero(h, kernel):
+    # a sequence with no cached tokens and a negative slot (nothing appended)
+    b = wl.small_batch(77, [40, 3], num_q_heads=4, num_kv_heads=2)
+    desc = h.desc_of(b)
+    q = h.to_dev(b.q)
+    out = torch.full_like(q, 7.0)
+    lens = torch.tensor([40, 0], dtype=torch.int32, device=h.DEV)
+    tables = torch.from_numpy(b.block_tables).to(h.DEV)
+    opts = pa.DecodeOptions(split_tokens=64, kernel=kernel, flags=pa.PA_FLAG_CHECK)
+    ws = torch.zeros(pa.pa_decode_workspace_size(2, 40, desc, opts), dtype=torch.uint8, device=h.DEV)
+    pa.pa_decode(q, h.to_dev(b.k_cache), h.to_dev(b.v_cache), tables, lens, 40, b.scale, out, ws,
+                 desc, opts)
+    torch.cuda.synchronize()
+    assert torch.all(out[1] == 0)
+    ref = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables,
+                              np.array([40, 0], np.int32), b.scale)
+    ok, ex = oracle.within_tolerance(out.float().cpu().numpy(), ref)
+    assert ok, ex
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+def test_physical_permutation_is_bitwise_invisible(h, kernel):
+    b = wl.small_batch(88, [100, 17, 640, 33], num_q_heads=8, num_kv_heads=2)
+    desc = h.desc_of(b)
+    lens = torch.from_numpy(b.context_lens).to(h.DEV)
+    opts = pa.DecodeOptions(split_tokens=128, kernel=kernel)
+    wsb = pa.pa_decode_workspace_size(b.batch, 640, desc, opts)
+
+    def run(kc, vc, tables):
+        out = torch.empty_like(h.to_dev(b.q))
+        ws = torch.zeros(wsb, dtype=torch.uint8, device=h.DEV)
+        pa.pa_decode(h.to_dev(b.q), h.to_dev(kc), h.to_dev(vc), torch.from_numpy(tables).to(h.DEV),
+                     lens, 640, b.scale, out, ws, desc, opts)
+        torch.cuda.synchronize()
+        return h.to_host_bits(out)
+
+    ref = run(b.k_cache, b.v_cache, b.block_tables)
+    perm = np.random.default_rng(5).permutation(b.num_blocks).astype(np.int32)
+    kc = np.empty_like(b.k_cache); vc = np.empty_like(b.v_cache)
+    kc[perm] = b.k_cache; vc[perm] = b.v_cache
+    tables = np.where(b.block_tables >= 0, perm[np.maximum(b.block_tables, 0)], -1).astype(np.int32)
+    np.testing.assert_array_equal(run(kc, vc, tables), ref)
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+def test_workspace_reused_without_clearing(h, kernel):
+    b = wl.small_batch(99, [1000, 513, 64], num_q_heads=4, num_kv_heads=1)
+    desc = h.desc_of(b)
+    lens = torch.from_numpy(b.context_lens).to(h.DEV)
+    tables = torch.from_numpy(b.block_tables).to(h.DEV)
+    opts = pa.DecodeOptions(split_tokens=64, kernel=kernel, flags=pa.PA_FLAG_CHECK)
+    ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, 1000, desc, opts), dtype=torch.uint8,
+                     device=h.DEV)
+    ref = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale)
+    kc, vc, q = h.to_dev(b.k_cache), h.to_dev(b.v_cache), h.to_dev(b.q)
+    outs = []
+    for _ in range(3):
+        out = torch.empty_like(q)
+        pa.pa_decode(q, kc, vc, tables, lens, 1000, b.scale, out, ws, desc, opts)
+        torch.cuda.synchronize()
+        outs.append(h.to_host_bits(out))
+        ok, ex = oracle.within_tolerance(out.float().cpu().numpy(), ref)
+        assert ok, ex
+    np.testing.assert_array_equal(outs[0], outs[1])
+    np.testing.assert_array_equal(outs[0], outs[2])
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+def test_bad_block_id_reported_not_faulted(h, kernel):
+    b = wl.small_batch(111, [50, 20], num_q_heads=4, num_kv_heads=2)
+    desc = h.desc_of(b)
+    tables = b.block_tables.copy()
+    tables[0, 1] = b.num_blocks + 5      # outside the pool
+    opts = pa.DecodeOptions(split_tokens=64, kernel=kernel, flags=pa.PA_FLAG_CHECK)
+    ws = torch.zeros(pa.pa_decode_workspace_size(2, 50, desc, opts), dtype=torch.uint8, device=h.DEV)
+    out = torch.empty_like(h.to_dev(b.q))
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode(h.to_dev(b.q), h.to_dev(b.k_cache), h.to_dev(b.v_cache),
+                     torch.from_numpy(tables).to(h.DEV), torch.from_numpy(b.context_lens).to(h.DEV),
+                     50, b.scale, out, ws, desc, opts)
+    assert e.value.status == -7
+    # the untouched sequence is still right, and the status word was cleared
+    ref = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale)
+    ok, ex = oracle.within_tolerance(out.float().cpu().numpy()[1], ref[1])
+    assert ok, ex
+    assert pa.pa_decode_status(ws) == 0
+
+
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+def test_length_beyond_bound_reported(h, kernel):
+    b = wl.small_batch(112, [50, 20], num_q_heads=4, num_kv_heads=2)
+    desc = h.desc_of(b)
+    opts = pa.DecodeOptions(split_tokens=64, kernel=kernel, flags=pa.PA_FLAG_CHECK)
+    ws = torch.zeros(pa.pa_decode_workspace_size(2, 40, desc, opts), dtype=torch.uint8, device=h.DEV)
+    out = torch.empty_like(h.to_dev(b.q))
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode(h.to_dev(b.q), h.to_dev(b.k_cache), h.to_dev(b.v_cache),
+                     torch.from_numpy(b.block_tables).to(h.DEV),
+                     torch.from_numpy(b.context_lens).to(h.DEV), 40, b.scale, out, ws, desc, opts)
+    assert e.value.status == -8
+
+
+def test_argument_errors(h):
+    b = wl.config1()
+    desc = h.desc_of(b)
+    q = h.to_dev(b.q)
+    kc = h.to_dev(b.k_cache)
+    tables = torch.from_numpy(b.block_tables).to(h.DEV)
+    lens = torch.from_numpy(b.context_lens).to(h.DEV)
+    out = torch.empty_like(q)
+    ws = torch.zeros(pa.pa_decode_workspace_size(2, 37, desc), dtype=torch.uint8, device=h.DEV)
+    with pytest.raises(pa.PaError) as e:   # workspace too small
+        pa.pa_decode(q, kc, kc, tables, lens, 37, b.scale, out, ws, desc, workspace_bytes=16)
+    assert e.value.status == -4
+    bad = pa.CacheDesc.make(num_blocks=8, block_size=16, num_kv_heads=1, num_q_heads=2, head_dim=96,
+                            max_blocks_per_seq=3)
+    with pytest.raises(pa.PaError) as e:   # head_dim 96 not built
+        pa.pa_decode(q, kc, kc, tables, lens, 37, b.scale, out, ws, bad)
+    assert e.value.status == -2
+    with pytest.raises(pa.PaError) as e:   # misaligned output pointer
+        pa.pa_decode(q, kc, kc, tables, lens, 37, b.scale, out.data_ptr() + 2, ws, desc)
+    assert e.value.status == -1
