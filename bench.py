@@ -375,9 +375,9 @@ def run_ours(args, rank, world, dist):
     if rank != 0:
         return None
 
-    kernel_name = "tensor" if kernel == pa.PA_KERNEL_TENSOR else "simt"
-    if kernel == pa.PA_KERNEL_AUTO:
-        kernel_name = os.environ.get("PA_DECODE_KERNEL", "simt")
+    # PA_KERNEL_AUTO runs the tensor-core kernel on every shape this bench builds
+    kernel_name = "simt" if (kernel == pa.PA_KERNEL_SIMT or
+                             os.environ.get("PA_DECODE_KERNEL") == "simt") else "tensor"
     peak, peak_kind = measured_peaks()
     kv_bytes = kv_read_bytes(lens, Hkv, D)
     achieved = kv_bytes / (dec_avg_ms / 1e3) / 1e9

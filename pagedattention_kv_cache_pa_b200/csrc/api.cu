@@ -97,8 +97,7 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
     }
     int32_t kernel = opt ? opt->kernel : PA_KERNEL_AUTO;
     if (kernel == PA_KERNEL_AUTO) kernel = env_kernel();
-    if (kernel == PA_KERNEL_AUTO) kernel = PA_KERNEL_SIMT;
-    plan->kernel = kernel;
+    plan->kernel = kernel;  // PA_KERNEL_AUTO resolves at launch
     plan->split_tokens = C;
     plan->max_splits = (int32_t)(max_context_len > 0 ? ceil_div(max_context_len, C) : 1);
     const int32_t G = d.num_q_heads / d.num_kv_heads;
@@ -234,10 +233,12 @@ extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_b
     p.max_splits = plan.max_splits;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaError_t e;
-    if (plan.kernel == PA_KERNEL_TENSOR && tensor_kernel_supports(p)) {
-        e = launch_decode_tensor(p, (cudaStream_t)stream);
-    } else {
+    const bool tensor_ok = tensor_kernel_supports(p);
+    if (plan.kernel == PA_KERNEL_TENSOR && !tensor_ok) return PA_ERR_UNSUPPORTED;
+    if (plan.kernel == PA_KERNEL_SIMT || !tensor_ok) {
         e = launch_decode_simt(p, (cudaStream_t)stream);
+    } else {
+        e = launch_decode_tensor(p, (cudaStream_t)stream);
     }
     if (e != cudaSuccess) return PA_ERR_CUDA;
     if (options && (options->flags & PA_FLAG_CHECK))
