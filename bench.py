@@ -62,7 +62,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=["c1", "c2", "c3", "c4"], default="c2")
-    ap.add_argument("--kernel", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "split"], default="auto")
+    ap.add_argument("--max-ctas", type=int, default=0)
     ap.add_argument("--split-tokens", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -91,7 +92,9 @@ def kv_read_bytes(lens, num_kv_heads, head_dim):
 
 
 def kernel_source_hash(kernel_name):
-    files = {"tensor": ["decode_tensor.cu"], "simt": ["decode_simt.cu"]}[kernel_name]
+    files = {"tensor": ["decode_stream.cu", "pa_ptx.cuh", "merge.cu"],
+             "split": ["decode_tensor.cu", "pa_ptx.cuh", "merge.cu"],
+             "simt": ["decode_simt.cu", "merge.cu"]}[kernel_name]
     files = files + ["pa_device.cuh", "pa_internal.h", "api.cu"]
     h = hashlib.sha256()
     for f in files:
@@ -272,8 +275,8 @@ def run_ours(args, rank, world, dist):
     desc = pa.CacheDesc.make(num_blocks=b.num_blocks, block_size=Bs, num_kv_heads=Hkv,
                              num_q_heads=Hq, head_dim=D, max_blocks_per_seq=MB)
     kernel = {"auto": pa.PA_KERNEL_AUTO, "simt": pa.PA_KERNEL_SIMT,
-              "tensor": pa.PA_KERNEL_TENSOR}[args.kernel]
-    opts = pa.DecodeOptions(split_tokens=args.split_tokens, kernel=kernel)
+              "tensor": pa.PA_KERNEL_TENSOR, "split": pa.PA_KERNEL_TENSOR_SPLIT}[args.kernel]
+    opts = pa.DecodeOptions(split_tokens=args.split_tokens, kernel=kernel, max_ctas=args.max_ctas)
     wsb = pa.pa_decode_workspace_size(B, max_len, desc, opts)
     ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
     splits = pa.pa_decode_max_splits(B, max_len, desc, opts)
@@ -375,9 +378,9 @@ def run_ours(args, rank, world, dist):
     if rank != 0:
         return None
 
-    # PA_KERNEL_AUTO runs the tensor-core kernel on every shape this bench builds
-    kernel_name = "simt" if (kernel == pa.PA_KERNEL_SIMT or
-                             os.environ.get("PA_DECODE_KERNEL") == "simt") else "tensor"
+    # PA_KERNEL_AUTO runs the tensor-core kernel; with Hkv a multiple of 8 (every
+    # workload here) that is the whole-group, stream-partitioned one
+    kernel_name = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR_SPLIT: "split"}.get(kernel, "tensor")
     peak, peak_kind = measured_peaks()
     kv_bytes = kv_read_bytes(lens, Hkv, D)
     achieved = kv_bytes / (dec_avg_ms / 1e3) / 1e9
@@ -402,7 +405,9 @@ def run_ours(args, rank, world, dist):
         "kv_read_gbs_step": kv_bytes * K / (elapsed_ms / 1e3) / 1e9,
         "e2e": {"value": e2e_value, "unit": "seq-steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": E},
-        "gpu_launches": 2 * K,
+        # per step: the append kernel, the decode kernel and (when any sequence can be cut)
+        # the merge kernel
+        "gpu_launches": K * (2 + (1 if (kernel_name == "tensor" or splits > 1) else 0)),
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:

@@ -103,17 +103,20 @@ PA_API int pa_append_kv(const pa_bf16* k, const pa_bf16* v, const int64_t* slot_
                  const pa_cache_desc* desc, void* stream);
 
 /* ---- paged decode attention ------------------------------------------------------------ */
-#define PA_KERNEL_AUTO    0   /* the fastest built kernel for the shape                         */
-#define PA_KERNEL_SIMT    1   /* CUDA-core kernel: plain loads, fp32 FMA                         */
-#define PA_KERNEL_TENSOR  2   /* TMA-staged pages, q.K and p.V on tensor cores (mma.sync bf16)   */
+#define PA_KERNEL_AUTO          0  /* the fastest built kernel for the shape                    */
+#define PA_KERNEL_SIMT          1  /* CUDA cores: plain loads, fp32 FMA                         */
+#define PA_KERNEL_TENSOR        2  /* tensor cores (mma.sync bf16), TMA-staged pages; whole kv-  */
+                                   /* head groups of 8 per CTA when Hkv % 8 == 0, else per head */
+#define PA_KERNEL_TENSOR_SPLIT  3  /* tensor cores, one (sequence, kv head, split) per work item */
 
 #define PA_FLAG_CHECK     1   /* synchronise after the launch and report device-side errors     */
 
 typedef struct pa_decode_options {
-    int32_t split_tokens;  /* 0: automatic; else tokens per KV split, a positive multiple of 64 */
+    int32_t split_tokens;  /* SIMT / TENSOR_SPLIT: 0 automatic, else tokens per KV split, a      */
+                           /* positive multiple of 64                                           */
     int32_t kernel;        /* PA_KERNEL_*                                                        */
     int32_t flags;         /* PA_FLAG_*                                                          */
-    int32_t reserved;      /* must be 0                                                          */
+    int32_t max_ctas;      /* TENSOR: 0 = one CTA per resident slot, else at most this many      */
 } pa_decode_options;
 
 /*
@@ -142,7 +145,10 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * may overlap on the GPU need separate workspaces.
  *
  * Built shapes: head_dim 64 or 128; block_size 8, 16, 32, 64, 128 or 256;
- * Hq / Hkv <= 16.  Others return PA_ERR_UNSUPPORTED.  Pointers q, out,
+ * Hq / Hkv <= 16.  Others return PA_ERR_UNSUPPORTED.  The tensor-core
+ * kernels need the CUDA driver's tensor-map encoder; an explicit
+ * PA_KERNEL_TENSOR(_SPLIT) request that cannot be served returns
+ * PA_ERR_UNSUPPORTED (no silent fallback).  Pointers q, out,
  * k_cache, v_cache must be 16-byte aligned.
  * A block id outside [0, num_blocks) is read as zeros and a length above
  * max_context_len or the table is clipped; both raise a bit in the

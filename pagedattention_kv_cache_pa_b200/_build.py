@@ -12,9 +12,9 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpa.so")
 
-CUDA_SOURCES = ["api.cu", "append.cu", "decode_simt.cu", "decode_tensor.cu"]
+CUDA_SOURCES = ["api.cu", "append.cu", "decode_simt.cu", "decode_tensor.cu", "decode_stream.cu", "merge.cu"]
 CXX_SOURCES = ["block_manager.cpp"]
-HEADERS = ["pa_internal.h", "pa_device.cuh"]
+HEADERS = ["pa_internal.h", "pa_device.cuh", "pa_ptx.cuh"]
 
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

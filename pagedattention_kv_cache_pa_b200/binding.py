@@ -15,7 +15,8 @@ import re
 import numpy as np
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libpa.so")
+# PA_LIBRARY points the binding at another build of the same ABI (e.g. a tuning variant)
+LIB_PATH = os.environ.get("PA_LIBRARY") or os.path.join(PKG, "libpa.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "pa.h")
 
 if not os.path.exists(LIB_PATH):
@@ -28,7 +29,7 @@ PA_OK = 0
 STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_CUDA",
           -4: "PA_ERR_WORKSPACE", -5: "PA_ERR_OOM_BLOCKS", -6: "PA_ERR_SHARED_BLOCK",
           -7: "PA_ERR_BAD_BLOCK", -8: "PA_ERR_BAD_LENGTH", -9: "PA_ERR_TIMEOUT"}
-PA_KERNEL_AUTO, PA_KERNEL_SIMT, PA_KERNEL_TENSOR = 0, 1, 2
+PA_KERNEL_AUTO, PA_KERNEL_SIMT, PA_KERNEL_TENSOR, PA_KERNEL_TENSOR_SPLIT = 0, 1, 2, 3
 PA_FLAG_CHECK = 1
 
 
@@ -51,7 +52,7 @@ class CacheDesc(ctypes.Structure):
 
 class DecodeOptions(ctypes.Structure):
     _fields_ = [("split_tokens", ctypes.c_int32), ("kernel", ctypes.c_int32),
-                ("flags", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("flags", ctypes.c_int32), ("max_ctas", ctypes.c_int32)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t

@@ -51,6 +51,7 @@ int32_t env_kernel() {
         if (!s) return (int32_t)PA_KERNEL_AUTO;
         if (!strcmp(s, "simt")) return (int32_t)PA_KERNEL_SIMT;
         if (!strcmp(s, "tensor")) return (int32_t)PA_KERNEL_TENSOR;
+        if (!strcmp(s, "split")) return (int32_t)PA_KERNEL_TENSOR_SPLIT;
         return (int32_t)PA_KERNEL_AUTO;
     }();
     return v;
@@ -76,12 +77,47 @@ int num_sms_current_device(int* out) {
     return PA_OK;
 }
 
-// Split plan: tokens per split C (a multiple of 64) and the grid's split count.
-// Automatic choice: enough (sequence, kv head, split) work items for about
-// 32 per SM if every sequence were max_context_len long, never below 128
-// tokens per split.
+// Decode plan: which kernel runs and how its workspace is laid out.
+//  * kStream (tensor cores, Hkv a multiple of 8): persistent grid of every
+//    resident CTA slot (or options->max_ctas); partial states: 2 per CTA.
+//  * kSplit / kSimt: C tokens per split (a multiple of 64), a split grid of
+//    ceil(max_context_len / C) per (sequence, kv head).  Automatic C: enough
+//    work items for about 32 per SM if every sequence were max_context_len
+//    long, never below 128 tokens.
+// Workspace: [0, 256) status word and work counters; (kStream) one piece
+// descriptor per (kv group, sequence); partial log-sum-exps; partial outputs.
 int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc& d,
                      const pa_decode_options* opt, DecodePlan* plan) {
+    int32_t kernel = opt ? opt->kernel : PA_KERNEL_AUTO;
+    if (kernel == PA_KERNEL_AUTO) kernel = env_kernel();
+    if (kernel == PA_KERNEL_AUTO) kernel = PA_KERNEL_TENSOR;
+    const int32_t G = d.num_q_heads / d.num_kv_heads;
+    const size_t pairs = (size_t)num_seqs * d.num_kv_heads;
+    auto up = [](size_t x) { return (x + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign; };
+    plan->off_desc = kWorkspaceAlign;
+    plan->off_lse = plan->off_desc;
+    plan->grid = 0;
+    plan->split_tokens = 0;
+    plan->max_splits = 1;
+
+    if (kernel == PA_KERNEL_TENSOR && stream_kernel_supports(d)) {
+        plan->kernel = DecodeKernel::kStream;
+        plan->grid = stream_kernel_grid(d, opt ? opt->max_ctas : 0);
+        if (plan->grid <= 0) return PA_ERR_CUDA;
+        plan->off_lse = plan->off_desc + up((size_t)(d.num_kv_heads / 8) * num_seqs * 16);
+        const size_t rows = (size_t)plan->grid * 2 * d.num_kv_heads * G;
+        plan->off_o = plan->off_lse + up(rows * sizeof(float));
+        plan->bytes = plan->off_o + up(rows * (size_t)d.head_dim * sizeof(float));
+        return PA_OK;
+    }
+    if (kernel == PA_KERNEL_TENSOR || kernel == PA_KERNEL_TENSOR_SPLIT) {
+        if (!tensor_kernel_supports(d)) return PA_ERR_UNSUPPORTED;
+        plan->kernel = DecodeKernel::kSplit;
+    } else if (kernel == PA_KERNEL_SIMT) {
+        plan->kernel = DecodeKernel::kSimt;
+    } else {
+        return PA_ERR_INVALID;
+    }
     int32_t C = opt ? opt->split_tokens : 0;
     if (C == 0) C = env_split_tokens();
     if (C < 0 || C % 64 != 0) return PA_ERR_INVALID;
@@ -95,25 +131,15 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
         if (c < 128) c = 128;
         C = (int32_t)(c > (1 << 30) ? (1 << 30) : c);
     }
-    int32_t kernel = opt ? opt->kernel : PA_KERNEL_AUTO;
-    if (kernel == PA_KERNEL_AUTO) kernel = env_kernel();
-    plan->kernel = kernel;  // PA_KERNEL_AUTO resolves at launch
     plan->split_tokens = C;
     plan->max_splits = (int32_t)(max_context_len > 0 ? ceil_div(max_context_len, C) : 1);
-    const int32_t G = d.num_q_heads / d.num_kv_heads;
-    const size_t pairs = (size_t)num_seqs * d.num_kv_heads;
-    auto up = [](size_t x) { return (x + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign; };
-    plan->off_counters = kWorkspaceAlign;  // [0, 256): status word
-    size_t off = plan->off_counters + up(pairs * sizeof(int32_t));
-    plan->off_lse = off;
     if (plan->max_splits > 1) {
-        off += up(pairs * plan->max_splits * G * sizeof(float));
-        plan->off_o = off;
-        off += up(pairs * plan->max_splits * G * (size_t)d.head_dim * sizeof(float));
+        plan->off_o = plan->off_lse + up(pairs * plan->max_splits * G * sizeof(float));
+        plan->bytes = plan->off_o + up(pairs * plan->max_splits * G * (size_t)d.head_dim * sizeof(float));
     } else {
-        plan->off_o = off;
+        plan->off_o = plan->off_lse;
+        plan->bytes = plan->off_lse;
     }
-    plan->bytes = off;
     return PA_OK;
 }
 
@@ -195,7 +221,7 @@ extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_b
                             const pa_decode_options* options, void* stream) {
     int rc = check_decode_shape(num_seqs, max_context_len, desc);
     if (rc != PA_OK) return rc;
-    if (options && (options->reserved != 0 || options->kernel < 0 || options->kernel > 2))
+    if (options && (options->max_ctas < 0 || options->kernel < 0 || options->kernel > 3))
         return PA_ERR_INVALID;
     if (num_seqs == 0) return PA_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
@@ -217,7 +243,9 @@ extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_b
     p.context_lens = context_lens;
     p.out = out;
     p.status = reinterpret_cast<int32_t*>(ws);
-    p.counters = reinterpret_cast<int32_t*>(ws + plan.off_counters);
+    p.work_counter = reinterpret_cast<int32_t*>(ws) + 1;
+    p.done_counter = reinterpret_cast<int32_t*>(ws) + 2;
+    p.seq_desc = reinterpret_cast<int32_t*>(ws + plan.off_desc);
     p.part_lse = reinterpret_cast<float*>(ws + plan.off_lse);
     p.part_o = reinterpret_cast<float*>(ws + plan.off_o);
     p.num_seqs = num_seqs;
@@ -233,13 +261,16 @@ extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_b
     p.max_splits = plan.max_splits;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaError_t e;
-    const bool tensor_ok = tensor_kernel_supports(p);
-    if (plan.kernel == PA_KERNEL_TENSOR && !tensor_ok) return PA_ERR_UNSUPPORTED;
-    if (plan.kernel == PA_KERNEL_SIMT || !tensor_ok) {
-        e = launch_decode_simt(p, (cudaStream_t)stream);
-    } else {
-        e = launch_decode_tensor(p, (cudaStream_t)stream);
+    const cudaStream_t st = (cudaStream_t)stream;
+    switch (plan.kernel) {
+        case DecodeKernel::kStream: e = launch_decode_stream(p, plan.grid, st); break;
+        case DecodeKernel::kSplit: e = launch_decode_tensor(p, st); break;
+        default: e = launch_decode_simt(p, st); break;
     }
+    // second pass: merge the pieces of every sequence that was cut
+    if (e == cudaSuccess && (plan.kernel == DecodeKernel::kStream || plan.max_splits > 1))
+        e = launch_merge(p, plan.kernel == DecodeKernel::kStream,
+                         plan.kernel != DecodeKernel::kSimt, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;
     if (options && (options->flags & PA_FLAG_CHECK))
         return pa_decode_status(workspace, workspace_bytes, stream);

@@ -8,7 +8,7 @@
 // that head's running max / sum / output (online softmax, fp32, log2 domain),
 // and accumulates p * V the same way.  The four warps' states are combined in
 // shared memory, then either stored (one split) or written as a partial state
-// that the last split to arrive merges.
+// for the merge kernel.
 //
 // It serves as the CUDA-core reference for the tensor-core kernel: every K/V
 // element is widened to fp32 once, but the per-token shuffle reductions make
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_simt_kernel(const DecodePa
     const int32_t split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int32_t L = clipped_length(p, b);
     if (L == 0) {
-        if (split == 0) store_zero_group(p, b, kvh);
+        if (split == 0) store_zero_group(p, b, kvh, threadIdx.x, blockDim.x);
         return;
     }
     const int32_t C = p.split_tokens;
@@ -148,7 +148,6 @@ __global__ void __launch_bounds__(kWarps * 32) decode_simt_kernel(const DecodePa
             if (d == 0) p.part_lse[part + h] = M + __log2f(lsum);
         }
     }
-    if (nsplit > 1) arrive_and_maybe_merge(p, b, kvh, nsplit);
 }
 
 template <int D>

@@ -1,0 +1,573 @@
+// Paged decode attention, stream-partitioned: the main tensor-core kernel.
+//
+// Shaped by two facts measured on the B200: HBM streams at full rate through
+// TMA only when each request is large (about 16 KB; a CTA retires roughly one
+// request every 0.4 us whatever its size), and a decode step is short, so any
+// imbalance between CTAs is paid in full.
+//
+//  * A CTA covers a group of 8 kv heads at once.  In the pool layout
+//    [block][kv head][token][head dim], the 16 tokens x 8 heads of a block are
+//    one 16 KB (D=64) region, fetched by a single 3-D tiled TMA box (dims
+//    head_dim x block_size x blocks*kv_heads, 128-byte swizzle, no multicast)
+//    for K and one for V.  Eight consumer warps each own one kv head; one
+//    producer warp feeds a ring of stages (16 tokens each) on mbarriers.
+//  * Work is the concatenation, over kv groups and sequences, of 16-token
+//    slabs (an empty sequence counts one slab).  The persistent grid (every
+//    resident CTA slot) cuts that stream into equal slices, so CTAs differ by
+//    at most one slab whatever the length mix.  A CTA walks its slice; each
+//    maximal run of one sequence inside it is a segment.  A sequence lying in
+//    one CTA is written out directly; one shared by several CTAs leaves one
+//    fp32 partial state per CTA (at most two per CTA: the run it starts in and
+//    the run it ends in), which the merge kernel (merge.cu) combines.
+//  * Per warp and stage: q.K^T for the group's query heads as m16n8k16 bf16
+//    MMAs (16 tokens = M, up to 8 heads = N per n-tile), fp32 online softmax
+//    in the log2 domain on the accumulator, probabilities rounded to bf16 and
+//    transposed in registers (movmatrix) into the B operand of V^T P.
+//  * q rows of a segment arrive by a 1-D bulk copy into a two-slot ring.
+//  * Every wait is bounded (2 s, then a status bit), so nothing can hang.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "pa_device.cuh"
+#include "pa_ptx.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int kGroup = 8;                    // kv heads per CTA = consumer warps
+constexpr int kThreads = (kGroup + 1) * 32;
+constexpr int kSlab = 16;                    // tokens per stage
+constexpr int kRowBytes = 128;               // 64 bf16 of head dim, one swizzled row
+constexpr int kQSlots = 2;
+
+template <int D, int NT>
+struct SCfg {
+    static constexpr int kHalves = D / 64;
+    static constexpr int kHalfBytes = kGroup * kSlab * kRowBytes;   // 16 KB
+    static constexpr int kTileBytes = kHalves * kHalfBytes;         // K (or V) of a stage
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kStages = (D == 128 && NT == 2) ? 2 : 3;
+    static constexpr int kKSteps = D / 16;
+    static constexpr int kMTiles = D / 16;
+    static constexpr int kMinBlocks = (D == 64 && NT == 1) ? 2 : 1;
+    // dynamic shared memory for query group size g
+    static constexpr size_t smem_bytes(int g) {
+        return (size_t)kStages * kStageBytes + (size_t)kQSlots * kGroup * g * D * 2 + 1024;
+    }
+};
+
+enum : int32_t { kFirst = 1, kLast = 2, kEmpty = 4, kEnd = 8 };
+
+struct Hdr {
+    int32_t b, kvh0, t0, valid;   // sequence, first kv head of the group, stage tokens [t0, t0+valid)
+    int32_t flags, qslot;         // kFirst / kLast / kEmpty / kEnd; q ring slot of the segment
+    int32_t nsplit, slot;         // CTAs sharing the sequence; this CTA's partial slot (0/1)
+    int32_t i_first, first_slot;  // first CTA of the sequence and the slot it used
+    int32_t pad0, pad1;
+};
+
+// Row of (kv head hl, token t) inside a stage half-tile filled by boxes of tb tokens x 8 heads.
+__device__ __forceinline__ int stage_row(int hl, int t, int tb) {
+    return (t / tb) * (kGroup * tb) + hl * tb + (t % tb);
+}
+
+__device__ __forceinline__ uint32_t swz(uint32_t half_tile, int row, int chunk) {
+    return half_tile + row * kRowBytes + (((chunk & 7) ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ int32_t nslabs(const DecodeParams& p, int32_t b) {
+    const int32_t L = clipped_length(p, b);
+    return L == 0 ? 1 : (L + kSlab - 1) / kSlab;
+}
+
+// CTA whose slice holds slab s (slices: [floor(i S / G), floor((i+1) S / G)) ).
+__device__ __forceinline__ int32_t cta_of(int64_t s, int64_t S, int64_t G) {
+    return (int32_t)(((s + 1) * G - 1) / S);
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
+    decode_stream_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
+                         const __grid_constant__ CUtensorMap vmap) {
+    using C = SCfg<D, NT>;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ Hdr s_hdr[C::kStages];
+    __shared__ __align__(8) uint64_t full_bar[C::kStages];
+    __shared__ __align__(8) uint64_t empty_bar[C::kStages];
+    __shared__ __align__(8) uint64_t qfull_bar[kQSlots];
+    __shared__ __align__(8) uint64_t qempty_bar[kQSlots];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int32_t G = p.group;
+    const int32_t Hkv = p.num_kv_heads;
+    const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
+    const uint32_t q_base = smem_base + C::kStages * C::kStageBytes;   // q ring after the stages
+    const uint32_t q_slot_bytes = (uint32_t)(kGroup * G * D * 2);
+    allow_dependents();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), kGroup);
+        }
+        for (int s = 0; s < kQSlots; ++s) {
+            mbar_init(smem_u32(&qfull_bar[s]), 1);
+            mbar_init(smem_u32(&qempty_bar[s]), kGroup);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == kGroup) {
+        // ================================ producer ================================
+        const int32_t B = p.num_seqs, Bs = p.block_size;
+        const int32_t tb = Bs < kSlab ? Bs : kSlab;             // tokens per TMA box
+        const int32_t groups = Hkv / kGroup;
+        const int32_t zmax = p.num_blocks * Hkv;                // z extent of the maps
+        // slabs per group of kv heads: S_seq = sum_b nslabs(b)
+        int64_t part = 0;
+        for (int32_t b = lane; b < B; b += 32) part += nslabs(p, b);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        const int64_t S_seq = part;
+        const int64_t S = S_seq * groups;
+        // slices: CTA i < Gc takes slabs [i S / Gc, (i+1) S / Gc); never more slices than slabs,
+        // so that every slice a sequence spans holds at least one of its slabs
+        const int64_t Gc = S < (int64_t)gridDim.x ? S : (int64_t)gridDim.x, ci = blockIdx.x;
+        const int64_t lo = ci < Gc ? ci * S / Gc : S, hi = ci < Gc ? (ci + 1) * S / Gc : S;
+        uint32_t gtile = 0, qk = 0;
+        bool alive = true;
+        auto acquire = [&](uint64_t* bars, uint32_t k, uint32_t n, int& slot) -> bool {
+            slot = (int)(k % n);
+            if (k >= n) {
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(smem_u32(&bars[slot]), ((k / n) - 1) & 1, p.status);
+                return __shfl_sync(0xffffffffu, ok, 0);
+            }
+            return true;
+        };
+        if (lo < hi) {
+            // locate slab lo: kv group gi, sequence b, slab j of b; P = stream index of b's slab 0
+            int32_t gi = (int32_t)(lo / S_seq);
+            const int64_t r = lo - (int64_t)gi * S_seq;
+            int32_t b = 0, j = 0;
+            int64_t P = 0, cum = 0;
+            for (int32_t base = 0; base < B; base += 32) {
+                const int32_t n = base + lane < B ? nslabs(p, base + lane) : 0;
+                int32_t incl = n;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                const int32_t total = __shfl_sync(0xffffffffu, incl, 31);
+                if (r < cum + total) {
+                    const unsigned hit = __ballot_sync(0xffffffffu, r < cum + incl);
+                    const int k = __ffs(hit) - 1;
+                    const int32_t excl = __shfl_sync(0xffffffffu, incl - n, k);
+                    b = base + k;
+                    j = (int32_t)(r - (cum + excl));
+                    P = (int64_t)gi * S_seq + cum + excl;
+                    break;
+                }
+                cum += total;
+            }
+            int32_t L = clipped_length(p, b);
+            int32_t nb = L == 0 ? 1 : (L + kSlab - 1) / kSlab;
+            // segment state
+            int32_t seg_nsplit = 1, seg_slot = 0, seg_ifirst = 0, seg_fslot = 0, seg_q = 0;
+            const int32_t* table = nullptr;
+            int32_t win_base = -1, win_entry = -1;
+            for (int64_t s = lo; s < hi && alive; ++s) {
+                const bool first = (s == lo) || (j == 0);
+                const bool last = (s == hi - 1) || (j == nb - 1);
+                if (first) {
+                    const int32_t i_first = cta_of(P, S, Gc), i_last = cta_of(P + nb - 1, S, Gc);
+                    seg_nsplit = i_last - i_first + 1;
+                    seg_slot = P < lo ? 0 : 1;
+                    seg_ifirst = i_first;
+                    seg_fslot = P < (int64_t)i_first * S / Gc ? 0 : 1;
+                    if (P >= lo && lane == 0)   // this CTA holds the sequence's first slab
+                        reinterpret_cast<int4*>(p.seq_desc)[(size_t)gi * B + b] =
+                            make_int4(seg_nsplit, i_first, seg_fslot, 0);
+                    table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+                    win_base = -1;
+                    if (L > 0) {
+                        int qs;
+                        if (!acquire(qempty_bar, qk, kQSlots, qs)) { alive = false; break; }
+                        seg_q = qs;
+                        if (lane == 0) {
+                            const uint32_t bar = smem_u32(&qfull_bar[qs]);
+                            mbar_arrive_expect_tx(bar, q_slot_bytes);
+                            bulk_load(q_base + qs * q_slot_bytes,
+                                      p.q + ((size_t)b * p.num_q_heads + (size_t)gi * kGroup * G) * D,
+                                      q_slot_bytes, bar);
+                        }
+                        ++qk;
+                    }
+                }
+                int st;
+                if (!acquire(empty_bar, gtile, C::kStages, st)) { alive = false; break; }
+                const int32_t t0 = j * kSlab;
+                const int32_t valid = L == 0 ? 0 : min(kSlab, L - t0);
+                const uint32_t fbar = smem_u32(&full_bar[st]);
+                if (lane == 0) {
+                    s_hdr[st] = Hdr{b, gi * kGroup, t0, valid,
+                                    (first ? kFirst : 0) | (last ? kLast : 0) | (L == 0 ? kEmpty : 0),
+                                    seg_q, seg_nsplit, seg_slot, seg_ifirst, seg_fslot, 0, 0};
+                }
+                if (valid > 0) {
+                    const int32_t nbox = (valid + tb - 1) / tb;
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(fbar, (uint32_t)(nbox * kGroup * tb * kRowBytes * C::kHalves * 2));
+                    const uint32_t k_tile = smem_base + st * C::kStageBytes;
+                    const uint32_t v_tile = k_tile + C::kTileBytes;
+                    for (int32_t x = 0; x < nbox; ++x) {
+                        const int32_t tok = t0 + x * tb;
+                        const int32_t lbk = tok / Bs;
+                        if (win_base < 0 || lbk >= win_base + 32) {      // warp-uniform refill
+                            win_base = lbk;
+                            const int32_t idx = win_base + lane;
+                            win_entry = idx < p.max_blocks_per_seq ? __ldg(table + idx) : -1;
+                        }
+                        const int32_t blk = __shfl_sync(0xffffffffu, win_entry, lbk - win_base);
+                        if (lane == 0) {
+                            int32_t z;
+                            if (blk < 0 || blk >= p.num_blocks) {
+                                raise_status(p.status, kStatusBadBlock);
+                                z = zmax;                                // outside the map: zeros
+                            } else {
+                                z = blk * Hkv + gi * kGroup;
+                            }
+                            const int32_t y = tok - lbk * Bs;
+                            const uint32_t off = (uint32_t)(x * kGroup * tb * kRowBytes);
+#pragma unroll
+                            for (int h = 0; h < C::kHalves; ++h) {
+                                tma_load_3d(k_tile + h * C::kHalfBytes + off, &kmap, h * 64, y, z, fbar);
+                                tma_load_3d(v_tile + h * C::kHalfBytes + off, &vmap, h * 64, y, z, fbar);
+                            }
+                        }
+                    }
+                } else if (lane == 0) {
+                    mbar_arrive(fbar);
+                }
+                ++gtile;
+                // advance to the next slab of the stream
+                if (++j == nb) {
+                    j = 0;
+                    P += nb;
+                    if (++b == B) {
+                        b = 0;
+                        ++gi;
+                    }
+                    if (s + 1 < hi) {
+                        L = clipped_length(p, b);
+                        nb = L == 0 ? 1 : (L + kSlab - 1) / kSlab;
+                    }
+                }
+            }
+        }
+        int st;
+        if (acquire(empty_bar, gtile, C::kStages, st) && lane == 0) {
+            s_hdr[st].flags = kEnd;
+            mbar_arrive(smem_u32(&full_bar[st]));
+        }
+    } else {
+        // ================================ consumers ===============================
+        // warp w owns kv head kvh0 + w of every stage
+        const int r = lane >> 2, c = lane & 3;
+        const int mi = lane >> 3, rr = lane & 7;
+        const int32_t tb = p.block_size < kSlab ? p.block_size : kSlab;
+        const float sl2 = p.scale_log2;
+        uint32_t qf[NT][C::kKSteps][2];
+        float m_run[NT][2], l_run[NT][2];
+        float o_acc[NT][C::kMTiles][4];
+        uint32_t qk = 0;
+        // rows of this warp's 16 tokens: lane-provided ldmatrix row addresses
+        const int row_a = stage_row(warp, rr + ((mi & 1) << 3), tb);     // K: tokens rr (+8)
+        const int row_b = stage_row(warp, rr + ((mi >> 1) << 3), tb);    // V: tokens rr (+8)
+        for (uint32_t gtile = 0;; ++gtile) {
+            const int st = gtile % C::kStages;
+            if (!warp_wait(smem_u32(&full_bar[st]), (gtile / C::kStages) & 1, p.status)) break;
+            const Hdr hd = s_hdr[st];
+            if (hd.flags & kEnd) break;
+            const int32_t kvh = hd.kvh0 + warp;
+            if (hd.flags & kEmpty) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+                store_zero_group(p, hd.b, kvh, lane, 32);
+                continue;
+            }
+            if (hd.flags & kFirst) {
+                const int qs = qk % kQSlots;
+                if (!warp_wait(smem_u32(&qfull_bar[qs]), (qk / kQSlots) & 1, p.status)) break;
+                const uint16_t* qsm = reinterpret_cast<const uint16_t*>(
+                    smem_gen + (q_base - smem_base) + qs * (size_t)(kGroup * G * D * 2)) + (size_t)warp * G * D;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int h = nt * 8 + r;
+#pragma unroll
+                    for (int ks = 0; ks < C::kKSteps; ++ks) {
+                        const uint32_t* qr = reinterpret_cast<const uint32_t*>(qsm + h * D + ks * 16);
+                        qf[nt][ks][0] = h < G ? qr[c] : 0u;
+                        qf[nt][ks][1] = h < G ? qr[c + 4] : 0u;
+                    }
+                    m_run[nt][0] = m_run[nt][1] = -INFINITY;
+                    l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+                    for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o_acc[nt][mt][e] = 0.f;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&qempty_bar[qs]));
+                ++qk;
+            }
+            const int valid = hd.valid;
+            const uint32_t k_tile = smem_base + st * C::kStageBytes;
+            const uint32_t v_tile = k_tile + C::kTileBytes;
+            if (valid < kSlab) {
+                // tokens past the sequence: zero V so that 0-probability rows add nothing
+                for (int i = lane; i < (kSlab - valid) * 8 * C::kHalves; i += 32) {
+                    const int t = valid + i / (8 * C::kHalves);
+                    const int ch = i % (8 * C::kHalves);
+                    const int row = stage_row(warp, t, tb);
+                    *reinterpret_cast<uint4*>(smem_gen + (v_tile - smem_base) + (ch >> 3) * C::kHalfBytes +
+                                              row * kRowBytes + (((ch & 7) ^ (row & 7)) << 4)) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+            }
+            // ---- S = K q^T : 16 tokens x 8 heads per n-tile ----
+            float sacc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < C::kKSteps; ++ks) {
+                const int ch = 2 * ks + (mi >> 1);
+                uint32_t a[4];
+                ldmatrix_x4(swz(k_tile + (ch >> 3) * C::kHalfBytes, row_a, ch), a);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+            }
+            // ---- online softmax over the 16 rows (tokens) per head column ----
+            const bool v_lo = r < valid, v_hi = (r + 8) < valid;
+            uint32_t pb[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float s0 = v_lo ? sacc[nt][0] * sl2 : -INFINITY;
+                const float s1 = v_lo ? sacc[nt][1] * sl2 : -INFINITY;
+                const float s2 = v_hi ? sacc[nt][2] * sl2 : -INFINITY;
+                const float s3 = v_hi ? sacc[nt][3] * sl2 : -INFINITY;
+                float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+                const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
+                m_run[nt][0] = mn0;
+                m_run[nt][1] = mn1;
+                const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
+                const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
+                l_run[nt][0] = l_run[nt][0] * al0 + (p0 + p2);
+                l_run[nt][1] = l_run[nt][1] * al1 + (p1 + p3);
+#pragma unroll
+                for (int mt = 0; mt < C::kMTiles; ++mt) {
+                    o_acc[nt][mt][0] *= al0;
+                    o_acc[nt][mt][1] *= al1;
+                    o_acc[nt][mt][2] *= al0;
+                    o_acc[nt][mt][3] *= al1;
+                }
+                pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));   // tokens 0-7
+                pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));   // tokens 8-15
+            }
+            // ---- O^T += V^T P : 16 head-dim rows x 8 heads per (m-tile, n-tile) ----
+#pragma unroll
+            for (int mt = 0; mt < C::kMTiles; ++mt) {
+                const int ch = 2 * mt + (mi & 1);
+                uint32_t a[4];
+                ldmatrix_x4_trans(swz(v_tile + (ch >> 3) * C::kHalfBytes, row_b, ch), a);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o_acc[nt][mt], a, pb[nt][0], pb[nt][1]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+            if (!(hd.flags & kLast)) continue;
+
+            // ======== end of this warp's segment: store, or publish a partial ========
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1)
+                        l_run[nt][jj] += __shfl_xor_sync(0xffffffffu, l_run[nt][jj], off);
+            const int32_t b = hd.b;
+            if (hd.nsplit == 1) {
+                uint16_t* out = p.out + ((size_t)b * p.num_q_heads + (size_t)kvh * G) * D;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int h = nt * 8 + 2 * c + jj;
+                        if (h >= G) continue;
+                        const float inv = 1.f / l_run[nt][jj];
+#pragma unroll
+                        for (int mt = 0; mt < C::kMTiles; ++mt) {
+                            out[(size_t)h * D + mt * 16 + r] = f32_to_bf16_rn(o_acc[nt][mt][jj] * inv);
+                            out[(size_t)h * D + mt * 16 + r + 8] = f32_to_bf16_rn(o_acc[nt][mt][jj + 2] * inv);
+                        }
+                    }
+                continue;
+            }
+            const size_t prow = (((size_t)blockIdx.x * 2 + hd.slot) * Hkv + kvh) * G;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int h = nt * 8 + 2 * c + jj;
+                    if (h >= G) continue;
+                    const float inv = 1.f / l_run[nt][jj];
+                    float* po = p.part_o + (prow + h) * D;
+#pragma unroll
+                    for (int mt = 0; mt < C::kMTiles; ++mt) {
+                        po[mt * 16 + r] = o_acc[nt][mt][jj] * inv;
+                        po[mt * 16 + r + 8] = o_acc[nt][mt][jj + 2] * inv;
+                    }
+                    if (r == 0) p.part_lse[prow + h] = m_run[nt][jj] + __log2f(l_run[nt][jj]);
+                }
+        }
+    }
+    __syncthreads();
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            f = reinterpret_cast<EncodeTiledFn>(ptr);
+            fn.store(f, std::memory_order_release);
+        }
+    }
+    return f;
+}
+
+// 3-D view [blocks * Hkv][block_size][head_dim]; box = 64 dims x tb tokens x 8 kv heads.
+bool make_map(CUtensorMap* map, const void* base, const DecodeParams& p) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)p.head_dim, (cuuint64_t)p.block_size,
+                                (cuuint64_t)p.num_blocks * p.num_kv_heads};
+    const cuuint64_t strides[2] = {(cuuint64_t)p.head_dim * 2,
+                                   (cuuint64_t)p.block_size * p.head_dim * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)(p.block_size < kSlab ? p.block_size : kSlab),
+                               (cuuint32_t)kGroup};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int NT>
+auto kernel_ptr() {
+    return decode_stream_kernel<D, NT>;
+}
+
+// The dynamic shared-memory opt-in is a per-kernel attribute: set it once per
+// device to the instantiation's largest need (its largest query group), then
+// size every launch by its own group.
+template <int D, int NT>
+bool ensure_smem_attr() {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const uint64_t bit = 1ull << dev;
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    if (cudaFuncSetAttribute(kernel_ptr<D, NT>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SCfg<D, NT>::smem_bytes(NT * 8)) != cudaSuccess)
+        return false;
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return true;
+}
+
+// Resident CTAs per SM for this instantiation and query group size (cached per device).
+template <int D, int NT>
+int occupancy(int g) {
+    static std::atomic<int> cache[64][17];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || g < 1 || g > NT * 8) return 0;
+    int occ = cache[dev][g].load(std::memory_order_acquire);
+    if (occ > 0) return occ;
+    if (!ensure_smem_attr<D, NT>()) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel_ptr<D, NT>(), kThreads,
+                                                      SCfg<D, NT>::smem_bytes(g)) != cudaSuccess)
+        return 0;
+    cache[dev][g].store(occ, std::memory_order_release);
+    return occ;
+}
+
+int occupancy_for(int D, int g) {
+    const bool two = g > 8;
+    if (D == 64) return two ? occupancy<64, 2>(g) : occupancy<64, 1>(g);
+    if (D == 128) return two ? occupancy<128, 2>(g) : occupancy<128, 1>(g);
+    return 0;
+}
+
+template <int D, int NT>
+cudaError_t launch_s(const DecodeParams& p, int grid, const CUtensorMap& km, const CUtensorMap& vm,
+                     cudaStream_t stream) {
+    if (!ensure_smem_attr<D, NT>() || occupancy<D, NT>(p.group) <= 0) return cudaErrorInvalidConfiguration;
+    decode_stream_kernel<D, NT><<<grid, kThreads, SCfg<D, NT>::smem_bytes(p.group), stream>>>(p, km, vm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool stream_kernel_supports(const pa_cache_desc& d) {
+    const int g = d.num_q_heads / d.num_kv_heads;
+    return (d.head_dim == 64 || d.head_dim == 128) && d.num_kv_heads % kGroup == 0 && g >= 1 &&
+           g <= 16 && encode_fn() != nullptr;
+}
+
+int stream_kernel_grid(const pa_cache_desc& d, int max_ctas) {
+    int sms = 0;
+    if (num_sms_current_device(&sms) != PA_OK) return 0;
+    const int occ = occupancy_for(d.head_dim, d.num_q_heads / d.num_kv_heads);
+    if (occ <= 0) return 0;
+    int grid = sms * occ;
+    if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
+    return grid;
+}
+
+cudaError_t launch_decode_stream(const DecodeParams& p, int grid, cudaStream_t stream) {
+    CUtensorMap km, vm;
+    if (!make_map(&km, p.k_cache, p) || !make_map(&vm, p.v_cache, p)) return cudaErrorInvalidValue;
+    const bool two = p.group > 8;
+    if (p.head_dim == 64)
+        return two ? launch_s<64, 2>(p, grid, km, vm, stream) : launch_s<64, 1>(p, grid, km, vm, stream);
+    if (p.head_dim == 128)
+        return two ? launch_s<128, 2>(p, grid, km, vm, stream) : launch_s<128, 1>(p, grid, km, vm, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pa

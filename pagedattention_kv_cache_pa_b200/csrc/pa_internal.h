@@ -24,8 +24,10 @@ struct DecodeParams {
     const int32_t* block_tables;   // [B][MB]
     const int32_t* context_lens;   // [B]
     uint16_t* out;                 // [B][Hq][D]
-    int32_t* status;               // device status word
-    int32_t* counters;             // [B][Hkv] split arrival counters (self-resetting)
+    int32_t* status;               // device status word (workspace word 0)
+    int32_t* work_counter;         // next work item to hand out (word 1, self-resetting)
+    int32_t* done_counter;         // CTAs that have finished (word 2, self-resetting)
+    int32_t* seq_desc;             // stream kernel: [Hkv/8][B] int4 {pieces, first CTA, first slot, 0}
     float* part_lse;               // [B][Hkv][S][G] log2-domain log-sum-exp
     float* part_o;                 // [B][Hkv][S][G][D] normalised partial outputs
     int32_t num_seqs;
@@ -42,11 +44,19 @@ struct DecodeParams {
     float scale_log2;              // scale * log2(e): scores are kept in the log2 domain
 };
 
+// Which decode kernel a plan runs.
+enum class DecodeKernel : int32_t {
+    kSimt = 0,     // CUDA cores, one CTA per (sequence, kv head, split)
+    kSplit = 1,    // tensor cores, persistent CTAs over (sequence, kv head, split) items
+    kStream = 2,   // tensor cores, 8 kv heads per CTA, stream-partitioned slabs
+};
+
 struct DecodePlan {
-    int32_t split_tokens;
-    int32_t max_splits;
-    int32_t kernel;                // PA_KERNEL_SIMT or PA_KERNEL_TENSOR
-    size_t off_counters, off_lse, off_o, bytes;
+    DecodeKernel kernel;
+    int32_t split_tokens;          // kSimt / kSplit: tokens per split
+    int32_t max_splits;            // kSimt / kSplit: splits per (sequence, kv head) at most
+    int32_t grid;                  // kStream: persistent CTAs (partial slots: 2 per CTA)
+    size_t off_desc, off_lse, off_o, bytes;
 };
 
 constexpr size_t kWorkspaceAlign = 256;
@@ -60,6 +70,10 @@ cudaError_t launch_append(const pa_bf16* k, const pa_bf16* v, const int64_t* slo
                           cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_tensor(const DecodeParams& p, cudaStream_t stream);
-bool tensor_kernel_supports(const DecodeParams& p);
+bool tensor_kernel_supports(const pa_cache_desc& d);
+cudaError_t launch_decode_stream(const DecodeParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_merge(const DecodeParams& p, bool stream_layout, bool pdl, cudaStream_t stream);
+bool stream_kernel_supports(const pa_cache_desc& d);
+int stream_kernel_grid(const pa_cache_desc& d, int max_ctas);
 
 }  // namespace pa

@@ -55,7 +55,7 @@ def host_step(b: wl.DecodeBatch):
 
 
 def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int = 0,
-             check_pool: bool = True, sample=None):
+             max_ctas: int = 0, check_pool: bool = True, sample=None):
     """Runs one step on both sides; returns a dict of results and checks."""
     (slots, tables, lens), (o_slots, o_tables, o_lens) = host_step(b)
     assert np.array_equal(slots, o_slots), "slot mapping differs from the model"
@@ -68,7 +68,8 @@ def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int =
     q = to_dev(b.q)
     out = torch.empty_like(q)
     max_len = int(lens.max()) if lens.size else 0
-    opts = pa.DecodeOptions(split_tokens=split_tokens, kernel=kernel, flags=pa.PA_FLAG_CHECK)
+    opts = pa.DecodeOptions(split_tokens=split_tokens, kernel=kernel, flags=pa.PA_FLAG_CHECK,
+                            max_ctas=max_ctas)
     ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, max_len, desc, opts), dtype=torch.uint8,
                      device=DEV)
     pa.pa_append_kv(to_dev(b.k_new), to_dev(b.v_new), torch.from_numpy(slots).to(DEV), k_cache,

@@ -69,7 +69,7 @@ def test_decode_rejects_unsupported_shapes_without_a_gpu():
                          ctypes.byref(d), None) == 0   # empty batch: nothing to do
     opts = pa.DecodeOptions(split_tokens=100)          # not a multiple of 64
     assert lib.pa_decode_max_splits(1, 16, ctypes.byref(d), ctypes.byref(opts)) == -1
-    opts = pa.DecodeOptions(split_tokens=128)          # explicit: no device query needed
+    opts = pa.DecodeOptions(split_tokens=128, kernel=pa.PA_KERNEL_SIMT)  # no device query needed
     assert lib.pa_decode_max_splits(1, 1000, ctypes.byref(d), ctypes.byref(opts)) == 8
     assert pa.pa_decode_workspace_size(2, 1000, d, opts) > 0
 

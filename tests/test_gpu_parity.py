@@ -14,8 +14,9 @@ import pagedattention_kv_cache_pa_b200 as pa
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = [pa.PA_KERNEL_SIMT, pa.PA_KERNEL_TENSOR]
-KNAMES = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR: "tensor"}
+KERNELS = [pa.PA_KERNEL_SIMT, pa.PA_KERNEL_TENSOR, pa.PA_KERNEL_TENSOR_SPLIT]
+KNAMES = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR: "tensor",
+          pa.PA_KERNEL_TENSOR_SPLIT: "split"}
 
 
 @pytest.fixture(scope="module")
@@ -44,6 +45,13 @@ def test_c2_llama_1b_layer(h, kernel, split):
     _assert(res)
 
 
+@pytest.mark.parametrize("ctas", [1, 2, 5, 64, 1000])
+def test_c2_stream_partitions(h, ctas):
+    # the tensor kernel's slices of the token stream: one CTA (no merge), a few (long
+    # merges), many (every sequence cut several times)
+    _assert(h.run_step(wl.config2(), kernel=pa.PA_KERNEL_TENSOR, max_ctas=ctas))
+
+
 @pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
 def test_c3_shared_prefix_bs256(h, kernel):
     _assert(h.run_step(wl.config3(), kernel=kernel))
@@ -52,7 +60,8 @@ def test_c3_shared_prefix_bs256(h, kernel):
 @pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
 def test_c4_long_context_split(h, kernel):
     res = h.run_step(wl.config4(), kernel=kernel)
-    assert res["splits"] > 1
+    if kernel != pa.PA_KERNEL_TENSOR:        # the stream kernel has no fixed split grid
+        assert res["splits"] > 1
     _assert(res)
 
 
@@ -60,6 +69,9 @@ EDGE_SHAPES = [
     # (Hq, Hkv, D, Bs)
     (4, 2, 64, 16), (8, 1, 128, 16), (3, 1, 64, 8), (16, 1, 64, 32), (6, 3, 128, 64),
     (32, 8, 64, 128), (2, 2, 64, 256), (16, 2, 128, 8),
+    # kv heads in groups of 8 (the tensor kernel's whole-group path)
+    (8, 8, 64, 8), (16, 8, 128, 16), (64, 8, 128, 16), (128, 8, 64, 16), (32, 16, 64, 32),
+    (24, 8, 64, 256), (96, 8, 128, 32),
 ]
 
 
@@ -72,8 +84,8 @@ def test_edge_lengths(h, kernel, shape):
     lens = [x for x in lens if x >= 0]
     b = wl.small_batch(1000 + Bs + D + Hq, lens, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
                        block_size=Bs)
-    for split in (64, 128, 0):
-        _assert(h.run_step(b, kernel=kernel, split_tokens=split))
+    for split, ctas in ((64, 3), (128, 17), (0, 0), (0, 1)):
+        _assert(h.run_step(b, kernel=kernel, split_tokens=split, max_ctas=ctas))
 
 
 @pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
