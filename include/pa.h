@@ -176,6 +176,36 @@ PA_API int pa_decode_status(void* workspace, size_t workspace_bytes, void* strea
 PA_API int32_t pa_decode_max_splits(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc* desc,
                              const pa_decode_options* options);
 
+/* ---- paged decode without allocation ------------------------------------------------------ */
+/*
+ * (The pages have no counterpart: this is a deployment convenience.)
+ *
+ * pa_decode for callers that cannot allocate device memory: code that runs
+ * under a memory planner which owns every device allocation in advance (an
+ * inference runtime that gives a plugin only its inputs and outputs), code on
+ * a latency-bound path where a cudaMalloc could synchronise the device or fail
+ * at the wrong moment, or C callers without an allocator.  Same arguments,
+ * result and errors as pa_decode_ex, minus the workspace: the scratch comes
+ * from a fixed array of PA_NOALLOC_SCRATCH_BYTES in the library's device image,
+ * which every GPU that loads the library holds until the process exits.  The
+ * call allocates nothing.
+ *  - A shape whose workspace (pa_decode_workspace_size_ex) exceeds
+ *    PA_NOALLOC_SCRATCH_BYTES returns PA_ERR_WORKSPACE and launches nothing.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array and it keeps the previous call's
+ *    contents (the words that must start at zero are cleared on `stream`), so
+ *    calls that may overlap on the GPU race: serialise them (one stream).
+ */
+#define PA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+PA_API int pa_decode_noalloc(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             int32_t num_seqs, int32_t max_context_len, float scale, pa_bf16* out,
+                             const pa_cache_desc* desc, const pa_decode_options* options,
+                             void* stream);
+
 /* ---- host slot mapping ----------------------------------------------------------------- */
 /*
  * slots[b] = block_tables[b][p / Bs] * Bs + p % Bs with p = lengths[b] - 1

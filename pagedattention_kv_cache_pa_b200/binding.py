@@ -73,6 +73,9 @@ lib.pa_decode.restype = ctypes.c_int
 lib.pa_decode_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _vp, _sz,
                              _DESC, _OPTS, _vp]
 lib.pa_decode_ex.restype = ctypes.c_int
+lib.pa_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _DESC,
+                                  _OPTS, _vp]
+lib.pa_decode_noalloc.restype = ctypes.c_int
 lib.pa_decode_status.argtypes = [_vp, _sz, _vp]
 lib.pa_decode_status.restype = ctypes.c_int
 lib.pa_decode_max_splits.argtypes = [_i32, _i32, _DESC, _OPTS]
@@ -193,6 +196,21 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: 
                             ctypes.byref(desc),
                             ctypes.byref(options) if options is not None else None,
                             _stream(stream)), "pa_decode")
+
+
+def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+                      scale: float, out, desc: CacheDesc, options: DecodeOptions | None = None,
+                      stream=None, num_seqs: int | None = None) -> None:
+    """pa_decode with the library's fixed scratch array instead of a caller workspace."""
+    n = int(context_lens.shape[0]) if num_seqs is None else int(num_seqs)
+    _check(lib.pa_decode_noalloc(_dev(q, "bfloat16", "q"), _dev(k_cache, "bfloat16", "k_cache"),
+                                 _dev(v_cache, "bfloat16", "v_cache"),
+                                 _dev(block_tables, "int32", "block_tables"),
+                                 _dev(context_lens, "int32", "context_lens"), n,
+                                 int(max_context_len), float(scale), _dev(out, "bfloat16", "out"),
+                                 ctypes.byref(desc),
+                                 ctypes.byref(options) if options is not None else None,
+                                 _stream(stream)), "pa_decode_noalloc")
 
 
 def pa_decode_status(workspace, stream=None, workspace_bytes: int | None = None) -> int:
