@@ -52,6 +52,9 @@ WORKLOAD_TEXT = {
     "c2": "Llama-3.2-1B-shaped decode layer: B=64, Hq=32, Hkv=8, D=64, Bs=16, cached L~U[128,2048] (+1 appended), pool=needed+10%",
     "c3": "shared 1024-token prefix (4 blocks in every table) + suffix~U[256,7168] (+1), B=32, Hq=32, Hkv=8, D=64, Bs=256",
     "c4": "long context split-KV: B=4, L=32768/65536/98304/131072 (+1), Hq=64, Hkv=8, D=128, Bs=16",
+    "c5": "continuous-batching trace: 16 layers (own pools), 256 live sequences, lognormal L (median 512, "
+          "sigma 1, <=16384), 100 decode steps, finish p=0.01 per step with replacement, Hq=32, Hkv=8, "
+          "D=64, Bs=16",
 }
 
 
@@ -61,9 +64,13 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4"], default="c2")
+    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4", "c5"], default="c2")
+    ap.add_argument("--trace-steps", type=int, default=200,
+                    help="c5: decode steps timed (the 100-step trace replayed as needed)")
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "split"], default="auto")
     ap.add_argument("--max-ctas", type=int, default=0)
+    ap.add_argument("--path", choices=["fused", "separate"], default="fused",
+                    help="fused: pa_append_decode; separate: pa_append_kv then pa_decode")
     ap.add_argument("--split-tokens", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -176,6 +183,25 @@ def run_reference(args, rank):
     import oracle
     if rank != 0:
         return None
+    if args.config == "c5":
+        t = wl.Trace5()
+        bm = oracle.BlockManagerModel(t.num_blocks, t.block_size, t.batch, t.max_blocks_per_seq,
+                                      t.free_order)
+        for s in range(t.batch):
+            bm.add_seq(s, int(t.initial_lens[s]))
+        bm.append_tokens(list(range(t.batch)))
+        tables = np.array([[bm.table_array(s) for s in range(t.batch)]], dtype=np.int32)
+        lens = np.array([bm.lens], dtype=np.int32)
+        t.steps = 1
+        cb = cpu_baseline_c5(t, tables, lens, max(1.0, args.cpu_seconds))
+        return {"metric": METRIC, "value": cb["value"], "unit": "seq-steps/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / cb["value"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": WORKLOAD_TEXT["c5"], "config": "c5", "batch": t.batch},
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "seq-steps/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     b = wl.CONFIGS[args.config]()
     B, Bs = b.batch, b.block_size
     model = oracle.BlockManagerModel(b.num_blocks, Bs, B, b.max_blocks_per_seq, b.free_order)
@@ -281,11 +307,17 @@ def run_ours(args, rank, world, dist):
     ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
     splits = pa.pa_decode_max_splits(B, max_len, desc, opts)
 
+    fused = args.path == "fused"
+
     def step(i):
         L = i % layers
-        pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
-        pa.pa_decode(q, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts,
-                     stream=stream)
+        if fused:
+            pa.pa_append_decode(q, k_new, v_new, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale,
+                                out, ws, desc, opts, stream=stream)
+        else:
+            pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
+            pa.pa_decode(q, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts,
+                         stream=stream)
 
     # correctness guard before timing: the kernel must not report device errors
     step(0)
@@ -308,11 +340,17 @@ def run_ours(args, rank, world, dist):
     t_start.record(stream)
     for i in range(K):
         L = i % layers
-        pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
-        ev_dec[i][0].record(stream)
-        pa.pa_decode(q, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts,
-                     stream=stream)
-        ev_dec[i][1].record(stream)
+        if fused:
+            ev_dec[i][0].record(stream)
+            pa.pa_append_decode(q, k_new, v_new, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale,
+                                out, ws, desc, opts, stream=stream)
+            ev_dec[i][1].record(stream)
+        else:
+            pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
+            ev_dec[i][0].record(stream)
+            pa.pa_decode(q, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts,
+                         stream=stream)
+            ev_dec[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -351,9 +389,13 @@ def run_ours(args, rank, world, dist):
         for dst, src in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_slots, h_slots),
                          (d_tables, h_tables), (d_lens, h_lens)):
             dst.copy_(src, non_blocking=True)
-        pa.pa_append_kv(d_k, d_v, d_slots, kcs[L], vcs[L], desc, stream=stream)
-        pa.pa_decode(d_q, kcs[L], vcs[L], d_tables, d_lens, max_len, b.scale, out, ws, desc, opts,
-                     stream=stream)
+        if fused:
+            pa.pa_append_decode(d_q, d_k, d_v, kcs[L], vcs[L], d_tables, d_lens, max_len, b.scale,
+                                out, ws, desc, opts, stream=stream)
+        else:
+            pa.pa_append_kv(d_k, d_v, d_slots, kcs[L], vcs[L], desc, stream=stream)
+            pa.pa_decode(d_q, kcs[L], vcs[L], d_tables, d_lens, max_len, b.scale, out, ws, desc, opts,
+                         stream=stream)
         h_out.copy_(out, non_blocking=True)
 
     for i in range(min(args.warmup, 20)):
@@ -393,26 +435,223 @@ def run_ours(args, rank, world, dist):
                    "block_size": Bs, "num_blocks": b.num_blocks, "mean_context": float(lens.mean()),
                    "max_context": max_len, "decode_kernel": kernel_name,
                    "split_tokens": args.split_tokens or "auto", "max_splits": splits,
+                   "call": "pa_append_decode" if fused else "pa_append_kv + pa_decode",
                    "l2": "inputs larger than L2: %d rotating layer pools of %.0f MB" % (layers, pool_bytes / 1e6),
                    "parallelism": "replicas x%d" % world},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
                      "traffic": profiled_traffic(args.config, kernel_name),
-                     "kernel": "pa_decode (%s)" % kernel_name,
+                     "kernel": ("pa_append_decode (%s)" if fused else "pa_decode (%s)") % kernel_name,
                      "algorithmic_bytes_per_launch": kv_bytes,
                      "avg_launch_ms": dec_avg_ms},
         "kv_read_gbs_step": kv_bytes * K / (elapsed_ms / 1e3) / 1e9,
         "e2e": {"value": e2e_value, "unit": "seq-steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": E},
-        # per step: the append kernel, the decode kernel and (when any sequence can be cut)
-        # the merge kernel
-        "gpu_launches": K * (2 + (1 if (kernel_name == "tensor" or splits > 1) else 0)),
+        # per step: the append (its own kernel unless the tensor kernel fuses it), the decode
+        # kernel and (when any sequence can be cut) the merge kernel
+        "gpu_launches": K * ((0 if (fused and kernel_name == "tensor") else 1) + 1 +
+                             (1 if (kernel_name == "tensor" or splits > 1) else 0)),
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(b, slots, tables, lens, args.cpu_seconds)
     return res
+
+
+def run_c5(args, rank, world, dist):
+    """C5: the continuous-batching trace.  One step = one decode step of all 16 layers for the
+    256 live sequences (host block manager, then pa_append_decode per layer)."""
+    import torch
+    import pagedattention_kv_cache_pa_b200 as pa
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    t = wl.Trace5()
+    B, Bs, MB, N = t.batch, t.block_size, t.max_blocks_per_seq, t.num_blocks
+    Hq, Hkv, D, NL, S = t.num_q_heads, t.num_kv_heads, t.head_dim, t.layers, t.steps
+    seqs = np.arange(B, dtype=np.int32)
+
+    def replay():
+        bm = pa.BlockManager(N, Bs, B, MB, t.free_order)
+        for s in range(B):
+            bm.add_seq(s, int(t.initial_lens[s]))
+        for step, retired, admitted in t.events():
+            for s in retired:
+                bm.free_seq(s)
+            for s, n in admitted:
+                bm.add_seq(s, n)
+            bm.append_tokens(seqs)
+            yield step, bm
+        bm.close()
+
+    tables = np.empty((S, B, MB), dtype=np.int32)
+    lens = np.empty((S, B), dtype=np.int32)
+    for step, bm in replay():
+        tables[step] = bm.block_tables()
+        lens[step] = bm.context_lens()
+    tables_d = torch.from_numpy(tables).to(dev)
+    lens_d = torch.from_numpy(lens).to(dev)
+    step_max = [int(x) for x in lens.max(axis=1)]
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    kcs, vcs, qs, ks, vs, outs = [], [], [], [], [], []
+    for layer in range(NL):
+        kc, vc = t.pool(layer)
+        kcs.append(to_dev(kc))
+        vcs.append(to_dev(vc))
+        del kc, vc
+        q, k, v = t.token_inputs(layer, 0)
+        qs.append(to_dev(q))
+        ks.append(to_dev(k))
+        vs.append(to_dev(v))
+        outs.append(torch.empty_like(qs[-1]))
+    desc = pa.CacheDesc.make(num_blocks=N, block_size=Bs, num_kv_heads=Hkv, num_q_heads=Hq,
+                             head_dim=D, max_blocks_per_seq=MB)
+    kernel = {"auto": pa.PA_KERNEL_AUTO, "simt": pa.PA_KERNEL_SIMT,
+              "tensor": pa.PA_KERNEL_TENSOR, "split": pa.PA_KERNEL_TENSOR_SPLIT}[args.kernel]
+    opts = pa.DecodeOptions(split_tokens=args.split_tokens, kernel=kernel, max_ctas=args.max_ctas)
+    ws = torch.zeros(pa.pa_decode_workspace_size(B, int(lens.max()), desc, opts), dtype=torch.uint8,
+                     device=dev)
+
+    def call(s, layer):
+        pa.pa_append_decode(qs[layer], ks[layer], vs[layer], kcs[layer], vcs[layer], tables_d[s],
+                            lens_d[s], step_max[s], t.scale, outs[layer], ws, desc, opts,
+                            stream=stream)
+
+    for s in range(3):
+        for layer in range(NL):
+            call(s, layer)
+    torch.cuda.synchronize()
+    rc = pa.pa_decode_status(ws)
+    if rc != 0:
+        raise RuntimeError("decode reported %s" % pa.pa_status_string(rc))
+    K = args.trace_steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K * NL)]
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
+    t0e.record(stream)
+    for i in range(K):
+        s = i % S
+        for layer in range(NL):
+            ev[i * NL + layer][0].record(stream)
+            call(s, layer)
+            ev[i * NL + layer][1].record(stream)
+    t1e.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    elapsed_ms = t0e.elapsed_time(t1e)
+    call_ms = np.array([a.elapsed_time(b) for a, b in ev])
+    kv_per_call = np.array([kv_read_bytes(lens[i % S], Hkv, D) for i in range(K) for _ in range(NL)],
+                           dtype=np.float64)
+    gbs = float(kv_per_call.sum() / (call_ms.sum() / 1e3) / 1e9)
+    if dist is not None:
+        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt[0])
+    value = world * B * K / (elapsed_ms / 1e3)
+
+    # e2e: the host block manager replays the trace inside the timed region; per step the
+    # table rows and lengths go up, per layer q/k/v go up and the output comes back
+    E = min(args.e2e_steps, S)
+    h_q = [torch.from_numpy(np.ascontiguousarray(t.token_inputs(l, 0)[0]).view(np.int16)).view(torch.bfloat16).pin_memory() for l in range(NL)]
+    h_k = [torch.from_numpy(np.ascontiguousarray(t.token_inputs(l, 0)[1]).view(np.int16)).view(torch.bfloat16).pin_memory() for l in range(NL)]
+    h_v = [torch.from_numpy(np.ascontiguousarray(t.token_inputs(l, 0)[2]).view(np.int16)).view(torch.bfloat16).pin_memory() for l in range(NL)]
+    h_out = torch.empty(outs[0].shape, dtype=torch.bfloat16).pin_memory()
+    h_tab = torch.empty((B, MB), dtype=torch.int32).pin_memory()
+    h_len = torch.empty((B,), dtype=torch.int32).pin_memory()
+    d_q, d_k, d_v = torch.empty_like(qs[0]), torch.empty_like(ks[0]), torch.empty_like(vs[0])
+    d_tab, d_len = torch.empty((B, MB), dtype=torch.int32, device=dev), torch.empty((B,), dtype=torch.int32, device=dev)
+    h2d = h_tab.numel() * 4 + h_len.numel() * 4 + NL * (h_q[0].numel() + h_k[0].numel() + h_v[0].numel()) * 2
+    d2h = NL * h_out.numel() * 2
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for step, bm in replay():
+        if step >= E:
+            break
+        torch.cuda.current_stream().synchronize()   # pinned staging is reused each step
+        h_tab.numpy()[:] = bm.block_tables()
+        h_len.numpy()[:] = bm.context_lens()
+        d_tab.copy_(h_tab, non_blocking=True)
+        d_len.copy_(h_len, non_blocking=True)
+        mx = int(h_len.numpy().max())
+        for layer in range(NL):
+            d_q.copy_(h_q[layer], non_blocking=True)
+            d_k.copy_(h_k[layer], non_blocking=True)
+            d_v.copy_(h_v[layer], non_blocking=True)
+            pa.pa_append_decode(d_q, d_k, d_v, kcs[layer], vcs[layer], d_tab, d_len, mx, t.scale,
+                                outs[layer], ws, desc, opts, stream=stream)
+            h_out.copy_(outs[layer], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt[0])
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks()
+    kernel_name = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR_SPLIT: "split"}.get(kernel, "tensor")
+    res = {
+        "metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": world, "steps": K,
+        "warmup": 3, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT["c5"], "config": "c5", "batch": B, "layers": NL,
+                   "trace_steps": S, "num_blocks": N, "mean_context": float(lens.mean()),
+                   "decode_kernel": kernel_name, "call": "pa_append_decode per layer",
+                   "l2": "inputs larger than L2: 16 layer pools of %.0f MB" % (2 * kcs[0].numel() * 2 / 1e6),
+                   "parallelism": "replicas x%d" % world},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                     "frac": gbs / peak, "peak_kind": peak_kind,
+                     "frac_of_nominal_8000": gbs / NOMINAL_HBM_GBS,
+                     "traffic": profiled_traffic("c5", kernel_name),
+                     "kernel": "pa_append_decode (%s)" % kernel_name,
+                     "algorithmic_bytes_per_launch": float(kv_per_call.mean()),
+                     "avg_launch_ms": float(call_ms.mean())},
+        "e2e": {"value": world * B * E / (e2e_ms / 1e3), "unit": "seq-steps/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": E,
+                "includes": "host block manager (retire, admit, append) per step"},
+        "gpu_launches": K * NL * 2,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline_c5(t, tables, lens, args.cpu_seconds)
+    return res
+
+
+def cpu_baseline_c5(t, tables, lens, budget_s):
+    """The oracle on layer 0 of successive trace steps (whole batch), until the budget is spent."""
+    import oracle
+    kc, vc = t.pool(0)
+    q, _, _ = t.token_inputs(0, 0)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        s = n % t.steps
+        oracle.paged_decode(q, kc, vc, tables[s], lens[s], t.scale)
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            break
+    # one seq-step = one sequence through all layers: the sample covers 1 of the 16 layers
+    return {"value": n * t.batch / dt / t.layers, "unit": "seq-steps/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d trace steps of layer 0 only (256 sequences x 32 heads each), %.1f s; "
+                      "value scaled to all %d layers" % (n, dt, t.layers)}
 
 
 def main(argv=None):
@@ -434,7 +673,7 @@ def main(argv=None):
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = dist_mod
     try:
-        res = run_ours(args, rank, world, dist)
+        res = (run_c5 if args.config == "c5" else run_ours)(args, rank, world, dist)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

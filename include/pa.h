@@ -166,6 +166,23 @@ PA_API int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16*
                  const pa_decode_options* options, void* stream);
 
 /*
+ * One decode step in one call: for every sequence b with L = context_lens[b] > 0,
+ * writes k[b], v[b] ([num_seqs][Hkv][D] bf16, all kv heads) into position L-1 of
+ * its table row (slot = block_tables[b][(L-1)/Bs]*Bs + (L-1)%Bs), then runs
+ * pa_decode over the L tokens.  The same result as pa_slot_mapping +
+ * pa_append_kv + pa_decode; the tensor-core kernel writes the new rows itself,
+ * just before it loads the block that holds them, which saves a launch and a
+ * pass.  Same arguments and errors as pa_decode_ex plus k and v (16-byte
+ * aligned); k_cache and v_cache are written.
+ */
+PA_API int pa_append_decode(const pa_bf16* q, const pa_bf16* k, const pa_bf16* v,
+                            pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, int32_t num_seqs, int32_t max_context_len,
+                            float scale, pa_bf16* out, void* workspace, size_t workspace_bytes,
+                            const pa_cache_desc* desc, const pa_decode_options* options,
+                            void* stream);
+
+/*
  * Synchronises `stream`, reads and clears the workspace's device status word.
  * Returns PA_OK, PA_ERR_BAD_BLOCK, PA_ERR_BAD_LENGTH or PA_ERR_TIMEOUT (the
  * first set, in that order), or PA_ERR_CUDA if the read fails.

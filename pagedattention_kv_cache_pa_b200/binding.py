@@ -73,6 +73,9 @@ lib.pa_decode.restype = ctypes.c_int
 lib.pa_decode_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _vp, _sz,
                              _DESC, _OPTS, _vp]
 lib.pa_decode_ex.restype = ctypes.c_int
+lib.pa_append_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp,
+                                 _vp, _sz, _DESC, _OPTS, _vp]
+lib.pa_append_decode.restype = ctypes.c_int
 lib.pa_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _DESC,
                                   _OPTS, _vp]
 lib.pa_decode_noalloc.restype = ctypes.c_int
@@ -196,6 +199,25 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: 
                             ctypes.byref(desc),
                             ctypes.byref(options) if options is not None else None,
                             _stream(stream)), "pa_decode")
+
+
+def pa_append_decode(q, k, v, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+                     scale: float, out, workspace, desc: CacheDesc,
+                     options: DecodeOptions | None = None, stream=None, num_seqs: int | None = None,
+                     workspace_bytes: int | None = None) -> None:
+    """Append each sequence's newest token at position context_lens-1, then decode."""
+    n = int(context_lens.shape[0]) if num_seqs is None else int(num_seqs)
+    wbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else int(workspace_bytes)
+    ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
+    _check(lib.pa_append_decode(_dev(q, "bfloat16", "q"), _dev(k, "bfloat16", "k"),
+                                _dev(v, "bfloat16", "v"), _dev(k_cache, "bfloat16", "k_cache"),
+                                _dev(v_cache, "bfloat16", "v_cache"),
+                                _dev(block_tables, "int32", "block_tables"),
+                                _dev(context_lens, "int32", "context_lens"), n,
+                                int(max_context_len), float(scale), _dev(out, "bfloat16", "out"), ws,
+                                wbytes, ctypes.byref(desc),
+                                ctypes.byref(options) if options is not None else None,
+                                _stream(stream)), "pa_append_decode")
 
 
 def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,

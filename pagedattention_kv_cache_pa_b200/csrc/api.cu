@@ -214,11 +214,12 @@ extern "C" int32_t pa_decode_max_splits(int32_t num_seqs, int32_t max_context_le
     return plan.max_splits;
 }
 
-extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
-                            const int32_t* block_tables, const int32_t* context_lens,
-                            int32_t num_seqs, int32_t max_context_len, float scale, pa_bf16* out,
-                            void* workspace, size_t workspace_bytes, const pa_cache_desc* desc,
-                            const pa_decode_options* options, void* stream) {
+// Shared by pa_decode_ex (k_new == v_new == null) and pa_append_decode.
+static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_new,
+                       const pa_bf16* k_cache, const pa_bf16* v_cache, const int32_t* block_tables,
+                       const int32_t* context_lens, int32_t num_seqs, int32_t max_context_len,
+                       float scale, pa_bf16* out, void* workspace, size_t workspace_bytes,
+                       const pa_cache_desc* desc, const pa_decode_options* options, void* stream) {
     int rc = check_decode_shape(num_seqs, max_context_len, desc);
     if (rc != PA_OK) return rc;
     if (options && (options->max_ctas < 0 || options->kernel < 0 || options->kernel > 3))
@@ -241,6 +242,8 @@ extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_b
     p.v_cache = v_cache;
     p.block_tables = block_tables;
     p.context_lens = context_lens;
+    p.k_new = k_new;
+    p.v_new = v_new;
     p.out = out;
     p.status = reinterpret_cast<int32_t*>(ws);
     p.work_counter = reinterpret_cast<int32_t*>(ws) + 1;
@@ -262,6 +265,11 @@ extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_b
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaError_t e;
     const cudaStream_t st = (cudaStream_t)stream;
+    if (k_new && plan.kernel != DecodeKernel::kStream) {   // only the stream kernel fuses the append
+        e = launch_append_at_end(p, st);
+        if (e != cudaSuccess) return PA_ERR_CUDA;
+        p.k_new = p.v_new = nullptr;
+    }
     switch (plan.kernel) {
         case DecodeKernel::kStream: e = launch_decode_stream(p, plan.grid, st); break;
         case DecodeKernel::kSplit: e = launch_decode_tensor(p, st); break;
@@ -275,6 +283,28 @@ extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_b
     if (options && (options->flags & PA_FLAG_CHECK))
         return pa_decode_status(workspace, workspace_bytes, stream);
     return PA_OK;
+}
+
+extern "C" int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            int32_t num_seqs, int32_t max_context_len, float scale, pa_bf16* out,
+                            void* workspace, size_t workspace_bytes, const pa_cache_desc* desc,
+                            const pa_decode_options* options, void* stream) {
+    return decode_call(q, nullptr, nullptr, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       max_context_len, scale, out, workspace, workspace_bytes, desc, options, stream);
+}
+
+extern "C" int pa_append_decode(const pa_bf16* q, const pa_bf16* k, const pa_bf16* v,
+                                pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* block_tables,
+                                const int32_t* context_lens, int32_t num_seqs,
+                                int32_t max_context_len, float scale, pa_bf16* out,
+                                void* workspace, size_t workspace_bytes, const pa_cache_desc* desc,
+                                const pa_decode_options* options, void* stream) {
+    if (num_seqs > 0 && (!k || !v || ((uintptr_t)k % 16) || ((uintptr_t)v % 16) ||
+                         desc == nullptr || desc->head_dim % 8 != 0))
+        return PA_ERR_INVALID;
+    return decode_call(q, k, v, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       max_context_len, scale, out, workspace, workspace_bytes, desc, options, stream);
 }
 
 extern "C" int pa_decode(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,

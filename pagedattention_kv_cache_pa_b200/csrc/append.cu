@@ -40,7 +40,42 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
     }
 }
 
+// Append of each sequence's newest token at position context_lens[b]-1 of its
+// table row (the fused append + decode call on the kernels that do not fuse it).
+__global__ void __launch_bounds__(256) append_at_end_kernel(const DecodeParams p) {
+    const int32_t chunks_per_row = p.head_dim / 8;
+    const int64_t per_seq = (int64_t)p.num_kv_heads * chunks_per_row;
+    const int64_t total = per_seq * p.num_seqs;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t b = (int32_t)(i / per_seq);
+        const int64_t within = i - (int64_t)b * per_seq;
+        const int32_t L = p.context_lens[b];
+        const int32_t cap = p.max_blocks_per_seq * p.block_size;
+        if (L <= 0 || L > cap || L > p.max_context_len) continue;
+        const int32_t pos = L - 1;
+        const int32_t blk = p.block_tables[(size_t)b * p.max_blocks_per_seq + pos / p.block_size];
+        if (blk < 0 || blk >= p.num_blocks) continue;
+        const int64_t h = within / chunks_per_row, c = within - h * chunks_per_row;
+        const int64_t dst = (((int64_t)blk * p.num_kv_heads + h) * p.block_size + pos % p.block_size) *
+                                chunks_per_row + c;
+        reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.k_cache))[dst] =
+            __ldg(reinterpret_cast<const uint4*>(p.k_new) + i);
+        reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.v_cache))[dst] =
+            __ldg(reinterpret_cast<const uint4*>(p.v_new) + i);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_append_at_end(const DecodeParams& p, cudaStream_t stream) {
+    const int64_t total = (int64_t)p.num_seqs * p.num_kv_heads * (p.head_dim / 8);
+    if (total == 0) return cudaSuccess;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    append_at_end_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_append(const pa_bf16* k, const pa_bf16* v, const int64_t* slots, int32_t T,
                           pa_bf16* k_cache, pa_bf16* v_cache, const pa_cache_desc& d,

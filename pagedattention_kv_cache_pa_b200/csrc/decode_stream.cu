@@ -109,6 +109,10 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
     const uint32_t q_base = smem_base + C::kStages * C::kStageBytes;   // q ring after the stages
     const uint32_t q_slot_bytes = (uint32_t)(kGroup * G * D * 2);
     allow_dependents();
+    if (threadIdx.x == kGroup * 32) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -220,6 +224,28 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                     s_hdr[st] = Hdr{b, gi * kGroup, t0, valid,
                                     (first ? kFirst : 0) | (last ? kLast : 0) | (L == 0 ? kEmpty : 0),
                                     seg_q, seg_nsplit, seg_slot, seg_ifirst, seg_fslot, 0, 0};
+                }
+                if (valid > 0 && p.k_new != nullptr && j == nb - 1) {
+                    // fused append: this slab holds the sequence's newest token (position L-1);
+                    // write its K/V rows for the group's 8 kv heads before the slab is loaded
+                    const int32_t pos = L - 1, lbn = pos / Bs;
+                    const int32_t blk = __ldg(table + lbn);
+                    if (blk >= 0 && blk < p.num_blocks) {
+                        constexpr int kChunks = D / 8;                    // 16-byte chunks per row
+                        for (int i = lane; i < kGroup * kChunks; i += 32) {
+                            const int hh = i / kChunks, cc = i - hh * kChunks;
+                            const size_t dst = (((size_t)blk * Hkv + gi * kGroup + hh) * Bs + (pos - lbn * Bs)) * D + cc * 8;
+                            const size_t src = ((size_t)b * Hkv + gi * kGroup + hh) * D + cc * 8;
+                            // the caches are the caller's writable buffers (pa_append_decode)
+                            reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.k_cache) + dst)[0] =
+                                __ldg(reinterpret_cast<const uint4*>(p.k_new + src));
+                            reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.v_cache) + dst)[0] =
+                                __ldg(reinterpret_cast<const uint4*>(p.v_new + src));
+                        }
+                    }
+                    // order these generic-proxy writes before the TMA reads of the slab
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    __syncwarp();
                 }
                 if (valid > 0) {
                     const int32_t nbox = (valid + tb - 1) / tb;

@@ -4,12 +4,12 @@
 // and query head h, the normalised output o_s[h][:] and the piece's log2-
 // domain log-sum-exp lse_s[h].  The softmax over the whole context is
 //   M = max_s lse_s,  w_s = 2^(lse_s - M),  out = sum_s w_s o_s / sum_s w_s,
-// rounded once to bf16.  One CTA of D threads per (sequence, kv head, query
-// head): the piece weights are computed once into shared memory, then each
-// thread accumulates one head-dim element with its global loads in flight
-// together.  The kernel runs as a programmatic dependent launch: its CTAs may
-// start while the decode kernel drains and wait (griddepcontrol.wait) for the
-// decode grid to complete before reading.
+// rounded once to bf16.  One CTA per (sequence, kv head, query head); the
+// pieces are spread over the CTA's threads and folded with a running max, so a
+// merge costs one round of L2 reads (after the piece descriptor).  The
+// kernel runs as a programmatic dependent launch: its CTAs may start while the
+// decode kernel drains and wait (griddepcontrol.wait) for the decode grid to
+// complete before reading.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,62 +18,85 @@
 namespace pa {
 namespace {
 
-constexpr int kSmemSplits = 2048;   // pieces whose weights fit in shared memory
+constexpr int kPieceGroups = 4;
 
+// One CTA of D threads per (sequence, kv head, query head): 4 groups over the
+// pieces (piece k goes to group k % 4) times D/4 float4 columns of the head
+// dimension.  Each thread folds its pieces into a running (max, weight, sum)
+// state as their lse and output arrive (one round of independent loads), and
+// the 4 groups' states are merged the same way through shared memory.
 template <int D, bool kStream>
 __global__ void __launch_bounds__(D) merge_kernel(const DecodeParams p) {
+    constexpr int kCols = D / 4;
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    __shared__ float s_w[kSmemSplits];
-    __shared__ float s_red[D / 32];
+    __shared__ float4 s_acc[kPieceGroups][kCols];
+    __shared__ float s_m[kPieceGroups], s_w[kPieceGroups];
     const int32_t b = blockIdx.x, kvh = blockIdx.y, h = blockIdx.z;
     const int32_t G = p.group, Hkv = p.num_kv_heads;
     const int tid = threadIdx.x;
     int32_t nsplit;
-    size_t row0, row_step;       // row of piece k: first piece row0, then row0 + k * row_step
-    int64_t first_row;           // stream layout: the first piece lives in its own row
+    size_t first_row, row0, row_step;   // piece 0: first_row; piece k >= 1: row0 + (k-1) * row_step
     if (kStream) {
         const int4 dsc = reinterpret_cast<const int4*>(p.seq_desc)[(size_t)(kvh / 8) * p.num_seqs + b];
         nsplit = dsc.x;
         if (nsplit <= 1) return;
-        // CTA i_first + k, slot 0 (k > 0); the first CTA used slot dsc.z
-        first_row = (((int64_t)dsc.y * 2 + dsc.z) * Hkv + kvh) * G + h;
-        row0 = (((size_t)(dsc.y + 1) * 2) * Hkv + kvh) * G + h;   // piece k >= 1: row0 + (k-1) * step
+        // CTA i_first + k wrote slot 0 for k > 0; the first CTA used slot dsc.z
+        first_row = (((size_t)dsc.y * 2 + dsc.z) * Hkv + kvh) * G + h;
+        row0 = (((size_t)(dsc.y + 1) * 2) * Hkv + kvh) * G + h;
         row_step = (size_t)2 * Hkv * G;
     } else {
         const int32_t L = clipped_length(p, b);
         nsplit = (L + p.split_tokens - 1) / p.split_tokens;
         if (nsplit <= 1) return;
-        first_row = (((int64_t)b * Hkv + kvh) * p.max_splits) * G + h;
-        row0 = (size_t)first_row + G;
+        first_row = (((size_t)b * Hkv + kvh) * p.max_splits) * G + h;
+        row0 = first_row + G;
         row_step = (size_t)G;
     }
-    auto row_of = [&](int32_t k) -> size_t {
-        return k == 0 ? (size_t)first_row : row0 + (size_t)(k - 1) * row_step;
-    };
-    // block-wide max of the pieces' log-sum-exps
-    float M = -INFINITY;
-    for (int32_t k = tid; k < nsplit; k += D) M = fmaxf(M, __ldcg(p.part_lse + row_of(k)));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if ((tid & 31) == 0) s_red[tid >> 5] = M;
+    const int kg = tid / kCols, col = tid - kg * kCols;
+    float m = -INFINITY, W = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int32_t k = kg; k < nsplit; k += kPieceGroups) {
+        const size_t r = k == 0 ? first_row : row0 + (size_t)(k - 1) * row_step;
+        const float lse = __ldcg(p.part_lse + r);
+        const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + r * D) + col);
+        const float mn = fmaxf(m, lse);
+        const float sc = fast_exp2(m - mn), w = fast_exp2(lse - mn);
+        W = W * sc + w;
+        acc.x = acc.x * sc + w * o.x;
+        acc.y = acc.y * sc + w * o.y;
+        acc.z = acc.z * sc + w * o.z;
+        acc.w = acc.w * sc + w * o.w;
+        m = mn;
+    }
+    s_acc[kg][col] = acc;
+    if (col == 0) {
+        s_m[kg] = m;
+        s_w[kg] = W;
+    }
     __syncthreads();
-    M = s_red[0];
+    if (tid < kCols) {
+        float M = s_m[0];
 #pragma unroll
-    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, s_red[w]);
-    const bool cached = nsplit <= kSmemSplits;
-    if (cached) {
-        for (int32_t k = tid; k < nsplit; k += D) s_w[k] = fast_exp2(__ldcg(p.part_lse + row_of(k)) - M);
-        __syncthreads();
+        for (int g = 1; g < kPieceGroups; ++g) M = fmaxf(M, s_m[g]);
+        float Wt = 0.f;
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int g = 0; g < kPieceGroups; ++g) {
+            const float sc = fast_exp2(s_m[g] - M);   // a group with no piece has m = -inf: weight 0
+            const float4 u = s_acc[g][tid];
+            Wt += s_w[g] * sc;
+            t.x += u.x * sc;
+            t.y += u.y * sc;
+            t.z += u.z * sc;
+            t.w += u.w * sc;
+        }
+        const float inv = 1.f / Wt;
+        uint2 packed;
+        packed.x = pack_bf16x2(t.x * inv, t.y * inv);
+        packed.y = pack_bf16x2(t.z * inv, t.w * inv);
+        reinterpret_cast<uint2*>(p.out + ((size_t)b * p.num_q_heads + (size_t)kvh * G + h) * D)[tid] = packed;
     }
-    float W = 0.f, acc = 0.f;
-#pragma unroll 8
-    for (int32_t k = 0; k < nsplit; ++k) {
-        const size_t r = row_of(k);
-        const float w = cached ? s_w[k] : fast_exp2(__ldcg(p.part_lse + r) - M);
-        W += w;
-        acc += w * __ldcg(p.part_o + r * D + tid);
-    }
-    p.out[((size_t)b * p.num_q_heads + (size_t)kvh * G + h) * D + tid] = f32_to_bf16_rn(acc / W);
 }
 
 template <int D, bool kStream>

@@ -23,6 +23,8 @@ struct DecodeParams {
     const uint16_t* v_cache;
     const int32_t* block_tables;   // [B][MB]
     const int32_t* context_lens;   // [B]
+    const uint16_t* k_new;         // fused append: [B][Hkv][D] row of each sequence's newest
+    const uint16_t* v_new;         //   token (position context_lens[b]-1), or null
     uint16_t* out;                 // [B][Hq][D]
     int32_t* status;               // device status word (workspace word 0)
     int32_t* work_counter;         // next work item to hand out (word 1, self-resetting)
@@ -68,6 +70,7 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
 cudaError_t launch_append(const pa_bf16* k, const pa_bf16* v, const int64_t* slots, int32_t T,
                           pa_bf16* k_cache, pa_bf16* v_cache, const pa_cache_desc& d,
                           cudaStream_t stream);
+cudaError_t launch_append_at_end(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_tensor(const DecodeParams& p, cudaStream_t stream);
 bool tensor_kernel_supports(const pa_cache_desc& d);

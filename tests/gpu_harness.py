@@ -55,8 +55,12 @@ def host_step(b: wl.DecodeBatch):
 
 
 def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int = 0,
-             max_ctas: int = 0, check_pool: bool = True, sample=None):
-    """Runs one step on both sides; returns a dict of results and checks."""
+             max_ctas: int = 0, check_pool: bool = True, sample=None, fused: bool = False):
+    """Runs one step on both sides; returns a dict of results and checks.
+
+    fused=False: pa_append_kv through the host slot mapping, then pa_decode.
+    fused=True: pa_append_decode (append at position L-1 through the table, then decode).
+    """
     (slots, tables, lens), (o_slots, o_tables, o_lens) = host_step(b)
     assert np.array_equal(slots, o_slots), "slot mapping differs from the model"
     assert np.array_equal(tables, o_tables), "block tables differ from the model"
@@ -72,10 +76,15 @@ def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int =
                             max_ctas=max_ctas)
     ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, max_len, desc, opts), dtype=torch.uint8,
                      device=DEV)
-    pa.pa_append_kv(to_dev(b.k_new), to_dev(b.v_new), torch.from_numpy(slots).to(DEV), k_cache,
-                    v_cache, desc)
-    pa.pa_decode(q, k_cache, v_cache, torch.from_numpy(tables).to(DEV),
-                 torch.from_numpy(lens).to(DEV), max_len, b.scale, out, ws, desc, opts)
+    if fused:
+        pa.pa_append_decode(q, to_dev(b.k_new), to_dev(b.v_new), k_cache, v_cache,
+                            torch.from_numpy(tables).to(DEV), torch.from_numpy(lens).to(DEV),
+                            max_len, b.scale, out, ws, desc, opts)
+    else:
+        pa.pa_append_kv(to_dev(b.k_new), to_dev(b.v_new), torch.from_numpy(slots).to(DEV), k_cache,
+                        v_cache, desc)
+        pa.pa_decode(q, k_cache, v_cache, torch.from_numpy(tables).to(DEV),
+                     torch.from_numpy(lens).to(DEV), max_len, b.scale, out, ws, desc, opts)
     torch.cuda.synchronize()
 
     ref_k, ref_v = oracle.append_kv(b.k_new, b.v_new, o_slots, b.k_cache, b.v_cache)

@@ -45,6 +45,13 @@ def test_c2_llama_1b_layer(h, kernel, split):
     _assert(res)
 
 
+@pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
+@pytest.mark.parametrize("cfg", ["c1", "c2", "c3", "c4"])
+def test_fused_append_decode(h, kernel, cfg):
+    # pa_append_decode: the append through the table inside the decode call
+    _assert(h.run_step(wl.CONFIGS[cfg](), kernel=kernel, fused=True))
+
+
 @pytest.mark.parametrize("ctas", [1, 2, 5, 64, 1000])
 def test_c2_stream_partitions(h, ctas):
     # the tensor kernel's slices of the token stream: one CTA (no merge), a few (long
@@ -84,8 +91,8 @@ def test_edge_lengths(h, kernel, shape):
     lens = [x for x in lens if x >= 0]
     b = wl.small_batch(1000 + Bs + D + Hq, lens, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
                        block_size=Bs)
-    for split, ctas in ((64, 3), (128, 17), (0, 0), (0, 1)):
-        _assert(h.run_step(b, kernel=kernel, split_tokens=split, max_ctas=ctas))
+    for split, ctas, fused in ((64, 3, False), (128, 17, True), (0, 0, False), (0, 1, True)):
+        _assert(h.run_step(b, kernel=kernel, split_tokens=split, max_ctas=ctas, fused=fused))
 
 
 @pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
@@ -211,3 +218,65 @@ def test_argument_errors(h):
     with pytest.raises(pa.PaError) as e:   # misaligned output pointer
         pa.pa_decode(q, kc, kc, tables, lens, 37, b.scale, out.data_ptr() + 2, ws, desc)
     assert e.value.status == -1
+
+
+@pytest.mark.parametrize("kernel", [pa.PA_KERNEL_TENSOR, pa.PA_KERNEL_SIMT], ids=["tensor", "simt"])
+def test_c5_continuous_batching_trace(h, kernel):
+    """Full-size C5 batch (256 sequences) through 12 trace steps on layers 0 and 15.
+
+    Each step: retire finished sequences, admit newcomers, append one token per
+    sequence (host block manager vs its model, bit-exact), then the fused
+    append + decode per layer; the oracle keeps its own pools, appending at the
+    model's slots.  Outputs compared in full at steps 0, 5 and 11 (step 11 is
+    past the trace's first retirements).
+    """
+    t = wl.Trace5()
+    B, Bs, MB, N = t.batch, t.block_size, t.max_blocks_per_seq, t.num_blocks
+    layers, steps, check = (0, 15), 12, {0, 5, 11}
+    assert t.finish[1:steps].any()
+    bm = pa.BlockManager(N, Bs, B, MB, t.free_order)
+    model = oracle.BlockManagerModel(N, Bs, B, MB, t.free_order)
+    for s in range(B):
+        bm.add_seq(s, int(t.initial_lens[s]))
+        model.add_seq(s, int(t.initial_lens[s]))
+    host = {l: [a.copy() for a in t.pool(l)] for l in layers}
+    devp = {l: [h.to_dev(a) for a in host[l]] for l in layers}
+    desc = pa.CacheDesc.make(num_blocks=N, block_size=Bs, num_kv_heads=t.num_kv_heads,
+                             num_q_heads=t.num_q_heads, head_dim=t.head_dim, max_blocks_per_seq=MB)
+    opts = pa.DecodeOptions(kernel=kernel, flags=pa.PA_FLAG_CHECK)
+    ws = torch.zeros(pa.pa_decode_workspace_size(B, 16384 + 200, desc, opts), dtype=torch.uint8,
+                     device=h.DEV)
+    seqs = np.arange(B, dtype=np.int32)
+    for step, retired, admitted in t.events():
+        if step >= steps:
+            break
+        for s in retired:
+            bm.free_seq(s)
+            model.free_seq(s)
+        for s, n in admitted:
+            bm.add_seq(s, n)
+            model.add_seq(s, n)
+        slots = bm.append_tokens(seqs)
+        m_slots = np.array(model.append_tokens(list(range(B))), dtype=np.int64)
+        assert np.array_equal(slots, m_slots)
+        tables = bm.block_tables().copy()
+        lens = bm.context_lens().copy()
+        m_tables = np.array([model.table_array(s) for s in range(B)], dtype=np.int32)
+        assert np.array_equal(tables, m_tables) and list(lens) == model.lens
+        td, ld = torch.from_numpy(tables).to(h.DEV), torch.from_numpy(lens).to(h.DEV)
+        for l in layers:
+            q, k, v = t.token_inputs(l, step)
+            out = torch.empty_like(h.to_dev(q))
+            pa.pa_append_decode(h.to_dev(q), h.to_dev(k), h.to_dev(v), devp[l][0], devp[l][1], td, ld,
+                                int(lens.max()), t.scale, out, ws, desc, opts)
+            oracle.append_kv(k, v, m_slots, host[l][0], host[l][1], in_place=True)
+            if step in check:
+                torch.cuda.synchronize()
+                ref = oracle.paged_decode(q, host[l][0], host[l][1], m_tables, lens, t.scale)
+                ok, ex = oracle.within_tolerance(out.float().cpu().numpy(), ref)
+                assert ok, "layer %d step %d: excess %g" % (l, step, ex)
+    torch.cuda.synchronize()
+    for l in layers:   # the pools the GPU appended into equal the oracle's, byte for byte
+        assert np.array_equal(h.to_host_bits(devp[l][0]), host[l][0])
+        assert np.array_equal(h.to_host_bits(devp[l][1]), host[l][1])
+    bm.close()

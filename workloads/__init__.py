@@ -279,7 +279,7 @@ class Trace5:
                  num_q_heads: int = 32, num_kv_heads: int = 8, head_dim: int = 64,
                  block_size: int = 16, median: float = 512.0, sigma: float = 1.0,
                  max_len: int = 16384, finish_p: float = 0.01,
-                 seed: int = CONFIG_SEED_BASE + 5, pool_slack: float = 1.25):
+                 seed: int = CONFIG_SEED_BASE + 5, pool_slack: float = 1.10):
         self.layers, self.steps, self.batch = layers, steps, batch
         self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
         self.block_size, self.seed = block_size, seed
@@ -292,11 +292,18 @@ class Trace5:
         n_new = int(self.finish.sum())
         self.new_lens = lognormal_lengths(stream_seed(seed, "new_lens"), max(n_new + (n_new & 1), 2),
                                           median, sigma, 1, max_len)[:n_new]
-        # Pool: blocks for the worst case of all lengths alive at once, plus slack.
+        # Pool: the most blocks the trace ever holds at once (counted per step after the
+        # newcomers arrive and every live sequence has its new token), plus slack.
         Bs = block_size
-        worst = int(np.sum(_ceil_div(self.initial_lens + steps, Bs)))
-        worst_new = int(np.sum(_ceil_div(self.new_lens + steps, Bs))) if n_new else 0
-        self.num_blocks = int(math.ceil(pool_slack * (worst + worst_new)))
+        lens = self.initial_lens.copy()
+        peak, k = 0, 0
+        for s in range(steps):
+            for slot in np.nonzero(self.finish[s])[0]:
+                lens[slot] = self.new_lens[k]
+                k += 1
+            lens = lens + 1
+            peak = max(peak, int(np.sum(_ceil_div(lens, Bs))))
+        self.num_blocks = int(math.ceil(pool_slack * peak))
         self.max_blocks_per_seq = _ceil_div(max_len + steps, Bs)
         self.free_order = permutation(stream_seed(seed, "block_order"), self.num_blocks)
 
