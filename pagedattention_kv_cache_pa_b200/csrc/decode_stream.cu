@@ -133,12 +133,22 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
         const int32_t tb = Bs < kSlab ? Bs : kSlab;             // tokens per TMA box
         const int32_t groups = Hkv / kGroup;
         const int32_t zmax = p.num_blocks * Hkv;                // z extent of the maps
+        const uint64_t kv_policy = l2_evict_first_policy();      // K/V are read once
         // slabs per group of kv heads: S_seq = sum_b nslabs(b)
-        int64_t part = 0;
-        for (int32_t b = lane; b < B; b += 32) part += nslabs(p, b);
+        // slabs per group of kv heads, S_seq = sum_b nslabs(b): lane i sums the contiguous
+        // chunk of sequences [i cs, (i+1) cs) (independent loads), then one warp scan
+        const int32_t cs = (B + 31) / 32;
+        const int32_t c_lo = min(B, lane * cs), c_hi = min(B, c_lo + cs);
+        int64_t lane_sum = 0;
+#pragma unroll 4
+        for (int32_t b = c_lo; b < c_hi; ++b) lane_sum += nslabs(p, b);
+        int64_t incl = lane_sum;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-        const int64_t S_seq = part;
+        for (int off = 1; off < 32; off <<= 1) {
+            const int64_t v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        const int64_t S_seq = __shfl_sync(0xffffffffu, incl, 31);
         const int64_t S = S_seq * groups;
         // slices: CTA i < Gc takes slabs [i S / Gc, (i+1) S / Gc); never more slices than slabs,
         // so that every slice a sequence spans holds at least one of its slabs
@@ -156,31 +166,31 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
             return true;
         };
         if (lo < hi) {
-            // locate slab lo: kv group gi, sequence b, slab j of b; P = stream index of b's slab 0
+            // locate slab lo: kv group gi, sequence b, slab j of b; P = stream index of b's slab 0.
+            // The lane whose chunk holds it walks its chunk (values still in L1).
             int32_t gi = (int32_t)(lo / S_seq);
             const int64_t r = lo - (int64_t)gi * S_seq;
+            const int64_t excl = incl - lane_sum;
+            const unsigned hit = __ballot_sync(0xffffffffu, r >= excl && r < incl);
+            const int k = __ffs(hit) - 1;
             int32_t b = 0, j = 0;
-            int64_t P = 0, cum = 0;
-            for (int32_t base = 0; base < B; base += 32) {
-                const int32_t n = base + lane < B ? nslabs(p, base + lane) : 0;
-                int32_t incl = n;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += v;
+            int64_t P = 0;
+            if (lane == k) {
+                int64_t acc = excl;
+                for (int32_t bb = c_lo; bb < c_hi; ++bb) {
+                    const int32_t n = nslabs(p, bb);
+                    if (r < acc + n) {
+                        b = bb;
+                        j = (int32_t)(r - acc);
+                        P = (int64_t)gi * S_seq + acc;
+                        break;
+                    }
+                    acc += n;
                 }
-                const int32_t total = __shfl_sync(0xffffffffu, incl, 31);
-                if (r < cum + total) {
-                    const unsigned hit = __ballot_sync(0xffffffffu, r < cum + incl);
-                    const int k = __ffs(hit) - 1;
-                    const int32_t excl = __shfl_sync(0xffffffffu, incl - n, k);
-                    b = base + k;
-                    j = (int32_t)(r - (cum + excl));
-                    P = (int64_t)gi * S_seq + cum + excl;
-                    break;
-                }
-                cum += total;
             }
+            b = __shfl_sync(0xffffffffu, b, k);
+            j = __shfl_sync(0xffffffffu, j, k);
+            P = __shfl_sync(0xffffffffu, P, k);
             int32_t L = clipped_length(p, b);
             int32_t nb = L == 0 ? 1 : (L + kSlab - 1) / kSlab;
             // segment state
@@ -274,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                             const uint32_t off = (uint32_t)(x * kGroup * tb * kRowBytes);
 #pragma unroll
                             for (int h = 0; h < C::kHalves; ++h) {
-                                tma_load_3d(k_tile + h * C::kHalfBytes + off, &kmap, h * 64, y, z, fbar);
-                                tma_load_3d(v_tile + h * C::kHalfBytes + off, &vmap, h * 64, y, z, fbar);
+                                tma_load_3d_hint(k_tile + h * C::kHalfBytes + off, &kmap, h * 64, y, z, fbar, kv_policy);
+                                tma_load_3d_hint(v_tile + h * C::kHalfBytes + off, &vmap, h * 64, y, z, fbar, kv_policy);
                             }
                         }
                     }

@@ -163,6 +163,56 @@ def test_workspace_reused_without_clearing(h, kernel):
     np.testing.assert_array_equal(outs[0], outs[2])
 
 
+def _decode_into(h, b, ws, opts):
+    desc = h.desc_of(b)
+    q = h.to_dev(b.q)
+    out = torch.full_like(q, 5.0)
+    max_len = int(b.context_lens.max())
+    assert ws.numel() >= pa.pa_decode_workspace_size(b.batch, max_len, desc, opts)
+    pa.pa_decode(q, h.to_dev(b.k_cache), h.to_dev(b.v_cache), torch.from_numpy(b.block_tables).to(h.DEV),
+                 torch.from_numpy(b.context_lens).to(h.DEV), max_len, b.scale, out, ws, desc, opts)
+    torch.cuda.synchronize()
+    ref = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale)
+    return oracle.within_tolerance(out.float().cpu().numpy(), ref)
+
+
+def test_stream_workspace_shared_across_shapes_and_kernels(h):
+    # one workspace, never cleared, through calls of different shapes, partitions and
+    # kernels: nothing a call leaves behind may leak into the next one
+    rng = np.random.default_rng(31)
+    ws = torch.zeros(64 << 20, dtype=torch.uint8, device=h.DEV)
+    a = wl.small_batch(501, list(rng.integers(1, 3000, 12)), num_q_heads=32, num_kv_heads=8)
+    mixed = wl.small_batch(502, [5000] + list(rng.integers(1, 200, 30)), num_q_heads=16,
+                           num_kv_heads=8, head_dim=128)
+    wide = wl.small_batch(503, list(rng.integers(1, 400, 300)), num_q_heads=8, num_kv_heads=8)
+    steps = [
+        (a, dict(kernel=pa.PA_KERNEL_TENSOR, max_ctas=7)),             # a few pieces per sequence
+        (wide, dict(kernel=pa.PA_KERNEL_TENSOR_SPLIT, split_tokens=64)),  # partials over the region
+        (wide, dict(kernel=pa.PA_KERNEL_TENSOR)),
+        (a, dict(kernel=pa.PA_KERNEL_TENSOR)),                         # > 16 pieces per sequence
+        (mixed, dict(kernel=pa.PA_KERNEL_TENSOR, max_ctas=40)),        # one long + many short
+        (wide, dict(kernel=pa.PA_KERNEL_SIMT, split_tokens=64)),
+        (a, dict(kernel=pa.PA_KERNEL_TENSOR, max_ctas=7)),
+        (mixed, dict(kernel=pa.PA_KERNEL_TENSOR, max_ctas=40)),
+    ]
+    for i, (b, o) in enumerate(steps):
+        ok, ex = _decode_into(h, b, ws, pa.DecodeOptions(flags=pa.PA_FLAG_CHECK, **o))
+        assert ok, "call %d outside tolerance by %g" % (i, ex)
+
+
+def test_stream_many_short_sequences(h):
+    # 8200 short sequences (65600 (sequence, kv head) pairs), cut by a 50-CTA grid and by
+    # the full one
+    rng = np.random.default_rng(32)
+    b = wl.small_batch(504, list(rng.integers(1, 48, 8200)), num_q_heads=8, num_kv_heads=8)
+    for ctas in (50, 0):
+        opts = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR, flags=pa.PA_FLAG_CHECK, max_ctas=ctas)
+        ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, int(b.context_lens.max()), h.desc_of(b),
+                                                     opts), dtype=torch.uint8, device=h.DEV)
+        ok, ex = _decode_into(h, b, ws, opts)
+        assert ok, ex
+
+
 @pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
 def test_bad_block_id_reported_not_faulted(h, kernel):
     b = wl.small_batch(111, [50, 20], num_q_heads=4, num_kv_heads=2)
