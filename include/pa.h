@@ -110,6 +110,7 @@ PA_API int pa_append_kv(const pa_bf16* k, const pa_bf16* v, const int64_t* slot_
 #define PA_KERNEL_TENSOR_SPLIT  3  /* tensor cores, one (sequence, kv head, split) per work item */
 
 #define PA_FLAG_CHECK     1   /* synchronise after the launch and report device-side errors     */
+#define PA_FLAG_PDL       2   /* early start (programmatic dependent launch), see pa_decode     */
 
 typedef struct pa_decode_options {
     int32_t split_tokens;  /* SIMT / TENSOR_SPLIT: 0 automatic, else tokens per KV split, a      */
@@ -154,6 +155,16 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * max_context_len or the table is clipped; both raise a bit in the
  * workspace's status word, which pa_decode_status reports (PA_FLAG_CHECK
  * does so before returning).
+ *
+ * PA_FLAG_PDL (whole-group tensor kernel only; ignored by the others): the
+ * decode kernel is launched as a programmatic dependent of the kernel before
+ * it on `stream`, so it may start while that kernel is still running.  Before
+ * it waits for that kernel to complete it reads ONLY context_lens and
+ * block_tables (to plan its slice of the work); q, the caches, out and the
+ * workspace are touched after the wait.  Set the flag only when context_lens
+ * and block_tables were complete before the previous kernel on `stream`
+ * started (host-written metadata, as in a serving step's layer loop).  The
+ * library's own kernels (append, merge) let such a launch start early.
  */
 PA_API int pa_decode(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
               const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,

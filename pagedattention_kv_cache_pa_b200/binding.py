@@ -31,6 +31,7 @@ STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ER
           -7: "PA_ERR_BAD_BLOCK", -8: "PA_ERR_BAD_LENGTH", -9: "PA_ERR_TIMEOUT"}
 PA_KERNEL_AUTO, PA_KERNEL_SIMT, PA_KERNEL_TENSOR, PA_KERNEL_TENSOR_SPLIT = 0, 1, 2, 3
 PA_FLAG_CHECK = 1
+PA_FLAG_PDL = 2
 
 
 class PaError(RuntimeError):

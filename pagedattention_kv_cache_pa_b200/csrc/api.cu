@@ -222,7 +222,8 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
                        const pa_cache_desc* desc, const pa_decode_options* options, void* stream) {
     int rc = check_decode_shape(num_seqs, max_context_len, desc);
     if (rc != PA_OK) return rc;
-    if (options && (options->max_ctas < 0 || options->kernel < 0 || options->kernel > 3))
+    if (options && (options->max_ctas < 0 || options->kernel < 0 || options->kernel > 3 ||
+                    (options->flags & ~(PA_FLAG_CHECK | PA_FLAG_PDL)) != 0))
         return PA_ERR_INVALID;
     if (num_seqs == 0) return PA_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
@@ -271,7 +272,9 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
         p.k_new = p.v_new = nullptr;
     }
     switch (plan.kernel) {
-        case DecodeKernel::kStream: e = launch_decode_stream(p, plan.grid, st); break;
+        case DecodeKernel::kStream:
+            e = launch_decode_stream(p, plan.grid, options && (options->flags & PA_FLAG_PDL), st);
+            break;
         case DecodeKernel::kSplit: e = launch_decode_tensor(p, st); break;
         default: e = launch_decode_simt(p, st); break;
     }

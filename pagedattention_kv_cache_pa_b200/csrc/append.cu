@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "pa_device.cuh"
 #include "pa_internal.h"
 
 namespace pa {
@@ -21,6 +22,7 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, const int64_t* __restrict__ slots,
     int64_t chunks, int32_t chunks_per_row, int32_t num_kv_heads, int32_t block_size,
     int64_t num_slots, uint4* __restrict__ k_cache, uint4* __restrict__ v_cache) {
+    allow_dependents();   // a decode launched early may plan while the rows are written
     const int64_t per_token = (int64_t)num_kv_heads * chunks_per_row;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks;
          i += (int64_t)gridDim.x * blockDim.x) {

@@ -195,8 +195,12 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
             int32_t nb = L == 0 ? 1 : (L + kSlab - 1) / kSlab;
             // segment state
             int32_t seg_nsplit = 1, seg_slot = 0, seg_ifirst = 0, seg_fslot = 0, seg_q = 0;
-            const int32_t* table = nullptr;
-            int32_t win_base = -1, win_entry = -1;
+            const int32_t* table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+            // the first table window, fetched while a prerequisite grid may still run
+            int32_t win_base = (j * kSlab) / Bs, win_entry = -1;
+            if (win_base + lane < p.max_blocks_per_seq) win_entry = __ldg(table + win_base + lane);
+            // everything below reads or writes what the previous kernel on the stream may touch
+            wait_prerequisite();
             for (int64_t s = lo; s < hi && alive; ++s) {
                 const bool first = (s == lo) || (j == 0);
                 const bool last = (s == hi - 1) || (j == nb - 1);
@@ -209,8 +213,10 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                     if (P >= lo && lane == 0)   // this CTA holds the sequence's first slab
                         reinterpret_cast<int4*>(p.seq_desc)[(size_t)gi * B + b] =
                             make_int4(seg_nsplit, i_first, seg_fslot, 0);
-                    table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
-                    win_base = -1;
+                    if (s != lo) {
+                        table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+                        win_base = -1;
+                    }
                     if (L > 0) {
                         int qs;
                         if (!acquire(qempty_bar, qk, kQSlots, qs)) { alive = false; break; }
@@ -315,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
         }
     } else {
         // ================================ consumers ===============================
+        wait_prerequisite();   // they write out / partials: not before the previous kernel ends
         // warp w owns kv head kvh0 + w of every stage
         const int r = lane >> 2, c = lane & 3;
         const int mi = lane >> 3, rr = lane & 7;
@@ -571,10 +578,19 @@ int occupancy_for(int D, int g) {
 
 template <int D, int NT>
 cudaError_t launch_s(const DecodeParams& p, int grid, const CUtensorMap& km, const CUtensorMap& vm,
-                     cudaStream_t stream) {
+                     bool pdl, cudaStream_t stream) {
     if (!ensure_smem_attr<D, NT>() || occupancy<D, NT>(p.group) <= 0) return cudaErrorInvalidConfiguration;
-    decode_stream_kernel<D, NT><<<grid, kThreads, SCfg<D, NT>::smem_bytes(p.group), stream>>>(p, km, vm);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SCfg<D, NT>::smem_bytes(p.group);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<D, NT>, p, km, vm);
 }
 
 }  // namespace
@@ -595,14 +611,16 @@ int stream_kernel_grid(const pa_cache_desc& d, int max_ctas) {
     return grid;
 }
 
-cudaError_t launch_decode_stream(const DecodeParams& p, int grid, cudaStream_t stream) {
+cudaError_t launch_decode_stream(const DecodeParams& p, int grid, bool pdl, cudaStream_t stream) {
     CUtensorMap km, vm;
     if (!make_map(&km, p.k_cache, p) || !make_map(&vm, p.v_cache, p)) return cudaErrorInvalidValue;
     const bool two = p.group > 8;
     if (p.head_dim == 64)
-        return two ? launch_s<64, 2>(p, grid, km, vm, stream) : launch_s<64, 1>(p, grid, km, vm, stream);
+        return two ? launch_s<64, 2>(p, grid, km, vm, pdl, stream)
+                   : launch_s<64, 1>(p, grid, km, vm, pdl, stream);
     if (p.head_dim == 128)
-        return two ? launch_s<128, 2>(p, grid, km, vm, stream) : launch_s<128, 1>(p, grid, km, vm, stream);
+        return two ? launch_s<128, 2>(p, grid, km, vm, pdl, stream)
+                   : launch_s<128, 1>(p, grid, km, vm, pdl, stream);
     return cudaErrorInvalidValue;
 }
 

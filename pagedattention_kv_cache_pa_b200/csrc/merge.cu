@@ -28,7 +28,8 @@ constexpr int kPieceGroups = 4;
 template <int D, bool kStream>
 __global__ void __launch_bounds__(D) merge_kernel(const DecodeParams p) {
     constexpr int kCols = D / 4;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    allow_dependents();   // a next decode call launched early may plan while this runs
+    wait_prerequisite();
     __shared__ float4 s_acc[kPieceGroups][kCols];
     __shared__ float s_m[kPieceGroups], s_w[kPieceGroups];
     const int32_t b = blockIdx.x, kvh = blockIdx.y, h = blockIdx.z;

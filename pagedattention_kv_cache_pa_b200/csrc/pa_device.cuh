@@ -30,10 +30,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
-// Lets a programmatic dependent launch (the merge kernel) be scheduled; it still
-// waits for this grid to complete before it reads anything.
+// Lets a programmatic dependent launch (the merge kernel, or a decode kernel
+// launched early) be scheduled; it still waits for this grid to complete
+// before it reads anything this grid writes.
 __device__ __forceinline__ void allow_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the grid this one was launched as a programmatic dependent of has
+// completed and its writes are visible; returns at once for a plain launch.
+__device__ __forceinline__ void wait_prerequisite() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 __device__ __forceinline__ void raise_status(int32_t* status, int32_t bit) {

@@ -74,7 +74,8 @@ cudaError_t launch_append_at_end(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_tensor(const DecodeParams& p, cudaStream_t stream);
 bool tensor_kernel_supports(const pa_cache_desc& d);
-cudaError_t launch_decode_stream(const DecodeParams& p, int grid, cudaStream_t stream);
+// pdl: launch as a programmatic dependent of the previous kernel on the stream.
+cudaError_t launch_decode_stream(const DecodeParams& p, int grid, bool pdl, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeParams& p, bool stream_layout, bool pdl, cudaStream_t stream);
 bool stream_kernel_supports(const pa_cache_desc& d);
 int stream_kernel_grid(const pa_cache_desc& d, int max_ctas);

@@ -55,11 +55,13 @@ def host_step(b: wl.DecodeBatch):
 
 
 def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int = 0,
-             max_ctas: int = 0, check_pool: bool = True, sample=None, fused: bool = False):
+             max_ctas: int = 0, check_pool: bool = True, sample=None, fused: bool = False,
+             pdl: bool = False):
     """Runs one step on both sides; returns a dict of results and checks.
 
     fused=False: pa_append_kv through the host slot mapping, then pa_decode.
     fused=True: pa_append_decode (append at position L-1 through the table, then decode).
+    pdl=True: PA_FLAG_PDL (the decode kernel may start while the append kernel runs).
     """
     (slots, tables, lens), (o_slots, o_tables, o_lens) = host_step(b)
     assert np.array_equal(slots, o_slots), "slot mapping differs from the model"
@@ -72,8 +74,8 @@ def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int =
     q = to_dev(b.q)
     out = torch.empty_like(q)
     max_len = int(lens.max()) if lens.size else 0
-    opts = pa.DecodeOptions(split_tokens=split_tokens, kernel=kernel, flags=pa.PA_FLAG_CHECK,
-                            max_ctas=max_ctas)
+    opts = pa.DecodeOptions(split_tokens=split_tokens, kernel=kernel, max_ctas=max_ctas,
+                            flags=pa.PA_FLAG_CHECK | (pa.PA_FLAG_PDL if pdl else 0))
     ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, max_len, desc, opts), dtype=torch.uint8,
                      device=DEV)
     if fused:

@@ -72,6 +72,10 @@ def test_decode_rejects_unsupported_shapes_without_a_gpu():
     opts = pa.DecodeOptions(split_tokens=128, kernel=pa.PA_KERNEL_SIMT)  # no device query needed
     assert lib.pa_decode_max_splits(1, 1000, ctypes.byref(d), ctypes.byref(opts)) == 8
     assert pa.pa_decode_workspace_size(2, 1000, d, opts) > 0
+    for bad in (4, 1 << 30, -1):                       # flag bits outside CHECK | PDL
+        o = pa.DecodeOptions(flags=bad)
+        assert lib.pa_decode_ex(fake, fake, fake, fake, fake, 1, 16, ctypes.c_float(0.1), fake, fake,
+                                1 << 20, ctypes.byref(d), ctypes.byref(o), None) == -1, bad
 
 
 def test_slot_mapping_entry_matches_oracle():

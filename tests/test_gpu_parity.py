@@ -213,6 +213,48 @@ def test_stream_many_short_sequences(h):
         assert ok, ex
 
 
+@pytest.mark.parametrize("cfg", ["c1", "c2", "c3", "c4"])
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_pdl_early_start(h, cfg, fused):
+    # PA_FLAG_PDL: the decode kernel may start while the append kernel before it runs;
+    # the new token's K/V (written by that kernel) must still be seen
+    _assert(h.run_step(wl.CONFIGS[cfg](), kernel=pa.PA_KERNEL_TENSOR, fused=fused, pdl=True))
+
+
+def test_pdl_chain_matches_plain_launches(h):
+    # calls chained through their outputs (each call's q is the previous call's out, written
+    # by the previous merge kernel): with PA_FLAG_PDL every call starts early and must
+    # still read the finished q; the chain is bitwise the chain of plain launches
+    b = wl.config2()
+    desc = h.desc_of(b)
+    kc, vc = h.to_dev(b.k_cache), h.to_dev(b.v_cache)
+    tables = torch.from_numpy(b.block_tables).to(h.DEV)
+    lens = torch.from_numpy(b.context_lens).to(h.DEV)
+    max_len = int(b.context_lens.max())
+
+    def chain(flags, ctas):
+        opts = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR, flags=flags, max_ctas=ctas)
+        ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, max_len, desc, opts), dtype=torch.uint8,
+                         device=h.DEV)
+        bufs = [h.to_dev(b.q)] + [torch.empty_like(h.to_dev(b.q)) for _ in range(6)]
+        for i in range(6):
+            pa.pa_decode(bufs[i], kc, vc, tables, lens, max_len, b.scale, bufs[i + 1], ws, desc, opts)
+        torch.cuda.synchronize()
+        assert pa.pa_decode_status(ws) == 0
+        return [h.to_host_bits(x) for x in bufs[1:]]
+
+    ref = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale)
+    for ctas in (0, 37):
+        plain = chain(0, ctas)
+        early = chain(pa.PA_FLAG_PDL, ctas)
+        first = plain[0].view(np.int16)
+        got = torch.from_numpy(first.copy()).view(torch.bfloat16).float().numpy()
+        ok, ex = oracle.within_tolerance(got, ref)
+        assert ok, ex
+        for i, (x, y) in enumerate(zip(plain, early)):
+            np.testing.assert_array_equal(x, y, err_msg="call %d of the chain" % i)
+
+
 @pytest.mark.parametrize("kernel", KERNELS, ids=KNAMES.get)
 def test_bad_block_id_reported_not_faulted(h, kernel):
     b = wl.small_batch(111, [50, 20], num_q_heads=4, num_kv_heads=2)
