@@ -264,6 +264,7 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     p.split_tokens = plan.split_tokens;
     p.max_splits = plan.max_splits;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.early = plan.kernel == DecodeKernel::kStream && options && (options->flags & PA_FLAG_PDL) ? 1 : 0;
     cudaError_t e;
     const cudaStream_t st = (cudaStream_t)stream;
     if (k_new && plan.kernel != DecodeKernel::kStream) {   // only the stream kernel fuses the append
@@ -273,7 +274,7 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     }
     switch (plan.kernel) {
         case DecodeKernel::kStream:
-            e = launch_decode_stream(p, plan.grid, options && (options->flags & PA_FLAG_PDL), st);
+            e = launch_decode_stream(p, plan.grid, p.early != 0, st);
             break;
         case DecodeKernel::kSplit: e = launch_decode_tensor(p, st); break;
         default: e = launch_decode_simt(p, st); break;

@@ -62,6 +62,9 @@ struct SCfg {
 
 enum : int32_t { kFirst = 1, kLast = 2, kEmpty = 4, kEnd = 8 };
 
+// Slabs an early-launched CTA prefetches into L2 before it waits for the previous kernel.
+constexpr int32_t kPrefetchSlabs = 2;
+
 struct Hdr {
     int32_t b, kvh0, t0, valid;   // sequence, first kv head of the group, stage tokens [t0, t0+valid)
     int32_t flags, qslot;         // kFirst / kLast / kEmpty / kEnd; q ring slot of the segment
@@ -199,6 +202,26 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
             // the first table window, fetched while a prerequisite grid may still run
             int32_t win_base = (j * kSlab) / Bs, win_entry = -1;
             if (win_base + lane < p.max_blocks_per_seq) win_entry = __ldg(table + win_base + lane);
+            if (p.early) {
+                // launched early: pull the first slabs of the slice (inside the first sequence
+                // and the fetched table window) into L2 while the previous kernel finishes
+                const int32_t pf_end = min(min((int64_t)nb, (int64_t)j + (hi - lo)), (int64_t)j + kPrefetchSlabs);
+                for (int32_t jj = j; jj < pf_end && L > 0; ++jj) {
+                    const int32_t t0 = jj * kSlab, valid = min(kSlab, L - t0);
+                    for (int32_t x = 0; x * tb < valid; ++x) {
+                        const int32_t tok = t0 + x * tb, lbk = tok / Bs;
+                        if (lbk - win_base >= 32) break;
+                        const int32_t blk = __shfl_sync(0xffffffffu, win_entry, lbk - win_base);
+                        if (lane == 0 && blk >= 0 && blk < p.num_blocks) {
+#pragma unroll
+                            for (int h = 0; h < C::kHalves; ++h) {
+                                tma_prefetch_3d(&kmap, h * 64, tok - lbk * Bs, blk * Hkv + gi * kGroup);
+                                tma_prefetch_3d(&vmap, h * 64, tok - lbk * Bs, blk * Hkv + gi * kGroup);
+                            }
+                        }
+                    }
+                }
+            }
             // everything below reads or writes what the previous kernel on the stream may touch
             wait_prerequisite();
             for (int64_t s = lo; s < hi && alive; ++s) {

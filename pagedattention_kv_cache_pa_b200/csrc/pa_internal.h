@@ -44,6 +44,7 @@ struct DecodeParams {
     int32_t split_tokens;          // C: tokens per split (multiple of 64)
     int32_t max_splits;            // S = ceil(max_context_len / C)
     float scale_log2;              // scale * log2(e): scores are kept in the log2 domain
+    int32_t early;                 // launched early (PA_FLAG_PDL): prefetch before the wait
 };
 
 // Which decode kernel a plan runs.
