@@ -62,6 +62,10 @@ def _lib():
         lib.oracle_paged_decode_partial.restype = ctypes.c_int
         lib.oracle_merge_partials.argtypes = [vp, vp, i64, i64, vp]
         lib.oracle_merge_partials.restype = None
+        lib.oracle_rope.argtypes = [vp, i64, i64, i64, vp, dbl, vp]
+        lib.oracle_rope.restype = None
+        lib.oracle_round_bf16.argtypes = [vp, i64, vp]
+        lib.oracle_round_bf16.restype = None
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_num_threads.restype = None
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -187,3 +191,42 @@ def within_tolerance(gpu: np.ndarray, ref: np.ndarray, atol: float = 1e-2, rtol:
     bound = atol + rtol * np.abs(ref)
     excess = float(np.max(err - bound)) if err.size else 0.0
     return bool(np.all(err <= bound)), excess
+
+
+def rope(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """fp64 rotary embedding of bf16 rows x [T, H, D] at positions [T] (unrounded).
+
+    Pair (x[i], x[i + D/2]) turns by positions[t] * theta^(-2i/D) (rotate-half pairing)."""
+    x = _c(x, np.uint16)
+    pos = _c(positions, np.int32)
+    T, H, D = x.shape
+    assert pos.shape == (T,) and D % 2 == 0
+    out = np.empty((T, H, D), dtype=np.float64)
+    _lib().oracle_rope(x.ctypes.data, T, H, D, pos.ctypes.data, float(theta), out.ctypes.data)
+    return out
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Nearest bf16 (ties to even) of each double, as uint16 bit patterns."""
+    x = _c(x, np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _lib().oracle_round_bf16(x.ctypes.data, x.size, out.ctypes.data)
+    return out
+
+
+def rope_bf16(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """Rotary embedding rounded to bf16, as the rotated rows are stored."""
+    return round_bf16(rope(x, positions, theta))
+
+
+def rope_append_decode(q, k_new, v_new, slots, k_cache, v_cache, block_tables, context_lens,
+                       scale: float, theta: float):
+    """One decode step with RoPE at each sequence's newest position (context_lens[b] - 1):
+    q and the new K rows are rotated and rounded to bf16, K (rotated) and V go into their
+    slots, and the rotated q attends over the cache.  Returns (out fp64, k_cache, v_cache, q_rot)."""
+    lens = _c(context_lens, np.int32)
+    pos = np.maximum(lens - 1, 0).astype(np.int32)
+    q_rot = rope_bf16(q, pos, theta)
+    k_rot = rope_bf16(k_new, pos, theta)
+    kc, vc = append_kv(k_rot, v_new, slots, k_cache, v_cache)
+    return paged_decode(q_rot, kc, vc, block_tables, lens, scale), kc, vc, q_rot

@@ -298,3 +298,64 @@ void oracle_merge_partials(const double* o, const double* lse, int64_t num_split
     }
     for (int64_t d = 0; d < head_dim; ++d) out[d] /= W;
 }
+
+/*
+ * ---- RoPE (rotary position embedding) ----
+ * "[Hacker News 요약] ... Tiny-vLLM ..." (aisleshub), section "핵심 LLM 연산의 CUDA
+ * 커널 구현", names RoPE among the per-layer operations of the Llama 3.2 1B model
+ * it targets, and gives no formula.  Reading (stated, not derived): RoFormer's
+ * rotation in the rotate-half pairing, with the caller's frequency base theta.
+ * For i < D/2, the pair (x[i], x[i + D/2]) of each head of a token at
+ * position p turns by the angle a_i = p * theta^(-2i/D):
+ *   y[i]       = x[i] cos a_i - x[i + D/2] sin a_i
+ *   y[i + D/2] = x[i] sin a_i + x[i + D/2] cos a_i
+ * x: [T][H][D] bf16, pos: [T]; out: [T][H][D] double, unrounded.
+ */
+void oracle_rope(const uint16_t* x, int64_t T, int64_t H, int64_t D, const int32_t* pos,
+                 double theta, double* out) {
+    const int64_t half = D / 2;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            const uint16_t* xr = x + (t * H + h) * D;
+            double* yr = out + (t * H + h) * D;
+            for (int64_t i = 0; i < half; ++i) {
+                const double a = (double)pos[t] * pow(theta, -2.0 * (double)i / (double)D);
+                const double c = cos(a), s = sin(a);
+                const double x1 = oracle_bf16_to_double(xr[i]);
+                const double x2 = oracle_bf16_to_double(xr[i + half]);
+                yr[i] = x1 * c - x2 * s;
+                yr[i + half] = x1 * s + x2 * c;
+            }
+        }
+}
+
+/*
+ * Round to the nearest bf16, ties to even (the format q and the caches are
+ * stored in).  With |x| in [2^(e-1), 2^e), a normal bf16 there is a multiple
+ * of 2^(e-8); below 2^-126 the subnormals are multiples of 2^-133.  Scaling by
+ * a power of two is exact, and rint() rounds half to even, so
+ * y = rint(x / q) * q is the correctly rounded value; past the largest finite
+ * bf16 it becomes infinity.  y is then exact in float, whose upper 16 bits are
+ * the bf16.
+ */
+void oracle_round_bf16(const double* x, int64_t n, uint16_t* out) {
+    const double max_bf16 = (2.0 - ldexp(1.0, -7)) * ldexp(1.0, 127);
+    for (int64_t k = 0; k < n; ++k) {
+        double v = x[k];
+        uint32_t u;
+        if (isnan(v)) {
+            out[k] = 0x7FC0;
+            continue;
+        }
+        if (v != 0.0 && isfinite(v)) {
+            int e;
+            frexp(v, &e);                          /* |v| in [2^(e-1), 2^e) */
+            const int qexp = e - 8 > -133 ? e - 8 : -133;
+            v = ldexp(rint(ldexp(v, -qexp)), qexp);
+            if (fabs(v) > max_bf16) v = v > 0 ? INFINITY : -INFINITY;
+        }
+        const float f = (float)v;                 /* exact: v is a bf16 value */
+        memcpy(&u, &f, sizeof u);
+        out[k] = (uint16_t)(u >> 16);
+    }
+}

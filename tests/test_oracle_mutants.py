@@ -1,5 +1,6 @@
 """The oracle pins have teeth: each plausible mistake, planted in a copy of the
-oracle's C source and compiled on the CPU, must make at least one pin fail.
+oracle's C source and compiled on the CPU, must make at least one pin fail
+(pins of tests/test_oracle.py and tests/test_oracle_rope.py).
 
 The mutant library replaces the oracle's loaded library only for the duration
 of one test; the real oracle source is never modified.
@@ -13,6 +14,7 @@ import pytest
 
 import oracle
 from tests import test_oracle as pins
+from tests import test_oracle_rope as rope_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.c")
 
@@ -46,13 +48,27 @@ MUTANTS = {
                                     "const int64_t slot = slot_mapping[t] < 0 ? 0 : slot_mapping[t];"),
     # K and V swapped in the gather
     "k_v_swapped": ("gather_sequence(k_cache, table_row, L, kvh", "gather_sequence(v_cache, table_row, L, kvh"),
+    # RoPE: rotation sense flipped
+    "rope_sign": ("yr[i] = x1 * c - x2 * s;", "yr[i] = x1 * c + x2 * s;"),
+    # RoPE: frequency exponent i/D instead of 2i/D
+    "rope_exponent": ("pow(theta, -2.0 * (double)i / (double)D)", "pow(theta, -1.0 * (double)i / (double)D)"),
+    # RoPE: wrong partner (neighbour instead of the other half)
+    "rope_pairing": ("const double x2 = oracle_bf16_to_double(xr[i + half]);",
+                     "const double x2 = oracle_bf16_to_double(xr[(i + 1) % D]);"),
+    # RoPE: position off by one
+    "rope_position": ("const double a = (double)pos[t] *", "const double a = (double)(pos[t] + 1) *"),
+    # bf16 rounding truncates instead of rounding to nearest
+    "round_truncates": ("v = ldexp(rint(ldexp(v, -qexp)), qexp);", "v = ldexp(trunc(ldexp(v, -qexp)), qexp);"),
+    # bf16 rounding breaks ties away from zero instead of to even
+    "round_ties_away": ("v = ldexp(rint(ldexp(v, -qexp)), qexp);", "v = ldexp(round(ldexp(v, -qexp)), qexp);"),
 }
 
 
 def _pin_calls():
     """Every pin in test_oracle as a zero-argument callable (parametrised ones expanded)."""
     calls = []
-    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+    members = inspect.getmembers(pins, inspect.isfunction) + inspect.getmembers(rope_pins, inspect.isfunction)
+    for name, fn in members:
         if not name.startswith("test_"):
             continue
         marks = getattr(fn, "pytestmark", [])
@@ -91,7 +107,8 @@ def test_pins_catch_planted_mistake(mutant, monkeypatch):
         # reuse the real library's prototypes on the mutant's symbols
         for sym in ("oracle_bf16_to_double", "oracle_kv_bytes", "oracle_slot", "oracle_slot_mapping",
                     "oracle_append_kv", "oracle_paged_decode", "oracle_paged_decode_partial",
-                    "oracle_merge_partials", "oracle_set_num_threads", "oracle_num_threads"):
+                    "oracle_merge_partials", "oracle_set_num_threads", "oracle_num_threads",
+                    "oracle_rope", "oracle_round_bf16"):
             f_real, f_mut = getattr(real, sym), getattr(mut, sym)
             f_mut.argtypes = f_real.argtypes
             f_mut.restype = f_real.restype
