@@ -77,6 +77,9 @@ def parse_args(argv=None):
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--rope", type=float, default=0.0,
+                    help="RoPE frequency base for the fused call (q and the new K turned at position "
+                         "L-1); 0 = no rotation")
     ap.add_argument("--pdl", choices=["on", "off"], default="on",
                     help="PA_FLAG_PDL: the tensor kernel plans its work while the previous kernel "
                          "runs; tables and lengths are written once before the timed region, as "
@@ -309,12 +312,31 @@ def run_ours(args, rank, world, dist):
               "tensor": pa.PA_KERNEL_TENSOR, "split": pa.PA_KERNEL_TENSOR_SPLIT}[args.kernel]
     pdl = args.pdl == "on"
     opts = pa.DecodeOptions(split_tokens=args.split_tokens, kernel=kernel, max_ctas=args.max_ctas,
-                            flags=pa.PA_FLAG_PDL if pdl else 0)
+                            flags=pa.PA_FLAG_PDL if pdl else 0, rope_theta=args.rope)
     wsb = pa.pa_decode_workspace_size(B, max_len, desc, opts)
     ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
     splits = pa.pa_decode_max_splits(B, max_len, desc, opts)
 
     fused = args.path == "fused"
+    # separate path: pa_append_kv (or pa_rope_append_kv) through the slot mapping, then pa_decode
+    opts_dec = pa.DecodeOptions(split_tokens=args.split_tokens, kernel=kernel, max_ctas=args.max_ctas,
+                                flags=pa.PA_FLAG_PDL if pdl else 0)
+    pos_d = torch.from_numpy(np.maximum(lens - 1, 0).astype(np.int32)).to(dev)
+    q_rot = torch.empty_like(q)
+
+    def separate(qq, kk, vv, sl, tb, ln, L, ev=None):
+        if args.rope > 0:
+            pa.pa_rope_append_kv(qq, q_rot, kk, vv, pos_d, sl, args.rope, kcs[L], vcs[L], desc,
+                                 stream=stream)
+            qq = q_rot
+        else:
+            pa.pa_append_kv(kk, vv, sl, kcs[L], vcs[L], desc, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_decode(qq, kcs[L], vcs[L], tb, ln, max_len, b.scale, out, ws, desc, opts_dec,
+                     stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
 
     def step(i):
         L = i % layers
@@ -322,9 +344,7 @@ def run_ours(args, rank, world, dist):
             pa.pa_append_decode(q, k_new, v_new, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale,
                                 out, ws, desc, opts, stream=stream)
         else:
-            pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
-            pa.pa_decode(q, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts,
-                         stream=stream)
+            separate(q, k_new, v_new, slots_d, tables_d, lens_d, L)
 
     # correctness guard before timing: the kernel must not report device errors
     step(0)
@@ -355,13 +375,7 @@ def run_ours(args, rank, world, dist):
             if not pdl:
                 ev_dec[i][1].record(stream)
         else:
-            pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
-            if not pdl:
-                ev_dec[i][0].record(stream)
-            pa.pa_decode(q, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts,
-                         stream=stream)
-            if not pdl:
-                ev_dec[i][1].record(stream)
+            separate(q, k_new, v_new, slots_d, tables_d, lens_d, L, None if pdl else ev_dec[i])
     t_end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -408,9 +422,7 @@ def run_ours(args, rank, world, dist):
             pa.pa_append_decode(d_q, d_k, d_v, kcs[L], vcs[L], d_tables, d_lens, max_len, b.scale,
                                 out, ws, desc, opts, stream=stream)
         else:
-            pa.pa_append_kv(d_k, d_v, d_slots, kcs[L], vcs[L], desc, stream=stream)
-            pa.pa_decode(d_q, kcs[L], vcs[L], d_tables, d_lens, max_len, b.scale, out, ws, desc, opts,
-                         stream=stream)
+            separate(d_q, d_k, d_v, d_slots, d_tables, d_lens, L)
         h_out.copy_(out, non_blocking=True)
 
     for i in range(min(args.warmup, 20)):
@@ -450,8 +462,9 @@ def run_ours(args, rank, world, dist):
                    "block_size": Bs, "num_blocks": b.num_blocks, "mean_context": float(lens.mean()),
                    "max_context": max_len, "decode_kernel": kernel_name,
                    "split_tokens": args.split_tokens or "auto", "max_splits": splits,
-                   "call": "pa_append_decode" if fused else "pa_append_kv + pa_decode",
-                   "pdl": pdl,
+                   "call": "pa_append_decode" if fused else
+                           ("pa_rope_append_kv + pa_decode" if args.rope > 0 else "pa_append_kv + pa_decode"),
+                   "pdl": pdl, "rope_theta": args.rope,
                    "l2": "inputs larger than L2: %d rotating layer pools of %.0f MB" % (layers, pool_bytes / 1e6),
                    "parallelism": "replicas x%d" % world},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -533,7 +546,7 @@ def run_c5(args, rank, world, dist):
               "tensor": pa.PA_KERNEL_TENSOR, "split": pa.PA_KERNEL_TENSOR_SPLIT}[args.kernel]
     pdl = args.pdl == "on"
     opts = pa.DecodeOptions(split_tokens=args.split_tokens, kernel=kernel, max_ctas=args.max_ctas,
-                            flags=pa.PA_FLAG_PDL if pdl else 0)
+                            flags=pa.PA_FLAG_PDL if pdl else 0, rope_theta=args.rope)
     ws = torch.zeros(pa.pa_decode_workspace_size(B, int(lens.max()), desc, opts), dtype=torch.uint8,
                      device=dev)
 
@@ -637,6 +650,7 @@ def run_c5(args, rank, world, dist):
         "config": {"workload": WORKLOAD_TEXT["c5"], "config": "c5", "batch": B, "layers": NL,
                    "trace_steps": S, "num_blocks": N, "mean_context": float(lens.mean()),
                    "decode_kernel": kernel_name, "call": "pa_append_decode per layer", "pdl": pdl,
+                   "rope_theta": args.rope,
                    "l2": "inputs larger than L2: 16 layer pools of %.0f MB" % (2 * kcs[0].numel() * 2 / 1e6),
                    "parallelism": "replicas x%d" % world},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",

@@ -102,6 +102,32 @@ PA_API int pa_append_kv(const pa_bf16* k, const pa_bf16* v, const int64_t* slot_
                  int32_t num_tokens, pa_bf16* k_cache, pa_bf16* v_cache,
                  const pa_cache_desc* desc, void* stream);
 
+/*
+ * RoPE (rotary position embedding) fused with the KV append.  The Tiny-vLLM
+ * summary page ("[Hacker News 요약] ... Tiny-vLLM ...", section "핵심 LLM 연산의
+ * CUDA 커널 구현") names RoPE among the per-layer kernels of the model it
+ * targets, without a formula; this library applies RoFormer's rotation in the
+ * rotate-half pairing: for i < D/2 the pair (x[i], x[i + D/2]) of every head of
+ * token t turns by the angle positions[t] * rope_theta^(-2i/D):
+ *   y[i] = x[i] cos a - x[i + D/2] sin a,   y[i + D/2] = x[i] sin a + x[i + D/2] cos a.
+ * Angles are formed in double, cos/sin and the rotation in float, and every
+ * rotated row is rounded to nearest-even bf16.
+ *
+ * q: [num_tokens][Hq][D] bf16, rotated into q_out (q_out == q rotates in
+ * place).  k: [num_tokens][Hkv][D] bf16, rotated and written into slot
+ * slot_mapping[t] of k_cache; v: the same shape, copied unchanged into the
+ * same slot of v_cache.  Slots follow pa_append_kv (negative or past the pool:
+ * nothing written for that token's K/V; its q is still rotated).  positions:
+ * [num_tokens] int32 device array.  rope_theta > 0.
+ * Requirements: head_dim 64 or 128; q, q_out, k, v, k_cache, v_cache 16-byte
+ * aligned.  num_tokens == 0 is a no-op.
+ * Errors: PA_ERR_INVALID (arguments), PA_ERR_UNSUPPORTED (head_dim), PA_ERR_CUDA.
+ */
+PA_API int pa_rope_append_kv(const pa_bf16* q, pa_bf16* q_out, const pa_bf16* k, const pa_bf16* v,
+                             const int32_t* positions, const int64_t* slot_mapping,
+                             int32_t num_tokens, float rope_theta, pa_bf16* k_cache,
+                             pa_bf16* v_cache, const pa_cache_desc* desc, void* stream);
+
 /* ---- paged decode attention ------------------------------------------------------------ */
 #define PA_KERNEL_AUTO          0  /* the fastest built kernel for the shape                    */
 #define PA_KERNEL_SIMT          1  /* CUDA cores: plain loads, fp32 FMA                         */
@@ -118,6 +144,9 @@ typedef struct pa_decode_options {
     int32_t kernel;        /* PA_KERNEL_*                                                        */
     int32_t flags;         /* PA_FLAG_*                                                          */
     int32_t max_ctas;      /* TENSOR: 0 = one CTA per resident slot, else at most this many      */
+    float rope_theta;      /* pa_append_decode only: > 0 turns q and the new K rows by RoPE at   */
+                           /* position L-1 with this frequency base (see pa_rope_append_kv);    */
+                           /* 0 = no rotation.  pa_decode(_ex) rejects a nonzero value.         */
 } pa_decode_options;
 
 /*
@@ -185,6 +214,14 @@ PA_API int pa_decode_ex(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16*
  * just before it loads the block that holds them, which saves a launch and a
  * pass.  Same arguments and errors as pa_decode_ex plus k and v (16-byte
  * aligned); k_cache and v_cache are written.
+ *
+ * With options->rope_theta > 0, q[b] and k[b] are first turned by RoPE at
+ * position L-1 (as pa_rope_append_kv does) and the rotated rows are rounded to
+ * bf16: the cache receives the rotated K, and the rotated q attends.  q itself
+ * is not modified.  The whole-group tensor kernel rotates in place of the
+ * append; the other kernels run one rotation kernel first, which writes the
+ * rotated q into the workspace (pa_decode_workspace_size_ex counts it when
+ * given the same options).
  */
 PA_API int pa_append_decode(const pa_bf16* q, const pa_bf16* k, const pa_bf16* v,
                             pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* block_tables,

@@ -53,7 +53,8 @@ class CacheDesc(ctypes.Structure):
 
 class DecodeOptions(ctypes.Structure):
     _fields_ = [("split_tokens", ctypes.c_int32), ("kernel", ctypes.c_int32),
-                ("flags", ctypes.c_int32), ("max_ctas", ctypes.c_int32)]
+                ("flags", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
+                ("rope_theta", ctypes.c_float)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -64,6 +65,9 @@ lib.pa_status_string.argtypes = [ctypes.c_int]
 lib.pa_status_string.restype = ctypes.c_char_p
 lib.pa_append_kv.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _DESC, _vp]
 lib.pa_append_kv.restype = ctypes.c_int
+lib.pa_rope_append_kv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, ctypes.c_float, _vp, _vp, _DESC,
+                                  _vp]
+lib.pa_rope_append_kv.restype = ctypes.c_int
 lib.pa_decode_workspace_size.argtypes = [_i32, _i32, _DESC]
 lib.pa_decode_workspace_size.restype = _sz
 lib.pa_decode_workspace_size_ex.argtypes = [_i32, _i32, _DESC, _OPTS]
@@ -169,6 +173,17 @@ def pa_append_kv(k, v, slot_mapping, k_cache, v_cache, desc: CacheDesc, stream=N
                             _dev(slot_mapping, "int64", "slot_mapping"), n,
                             _dev(k_cache, "bfloat16", "k_cache"), _dev(v_cache, "bfloat16", "v_cache"),
                             ctypes.byref(desc), _stream(stream)), "pa_append_kv")
+
+
+def pa_rope_append_kv(q, q_out, k, v, positions, slot_mapping, rope_theta: float, k_cache, v_cache,
+                      desc: CacheDesc, stream=None, num_tokens: int | None = None) -> None:
+    n = int(slot_mapping.shape[0]) if num_tokens is None else int(num_tokens)
+    _check(lib.pa_rope_append_kv(_dev(q, "bfloat16", "q"), _dev(q_out, "bfloat16", "q_out"),
+                                 _dev(k, "bfloat16", "k"), _dev(v, "bfloat16", "v"),
+                                 _dev(positions, "int32", "positions"),
+                                 _dev(slot_mapping, "int64", "slot_mapping"), n, float(rope_theta),
+                                 _dev(k_cache, "bfloat16", "k_cache"), _dev(v_cache, "bfloat16", "v_cache"),
+                                 ctypes.byref(desc), _stream(stream)), "pa_rope_append_kv")
 
 
 def pa_decode_workspace_size(num_seqs: int, max_context_len: int, desc: CacheDesc,

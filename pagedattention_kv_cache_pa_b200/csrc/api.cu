@@ -1,6 +1,7 @@
 // C-ABI entry points of libpa: argument checks, the split plan, dispatch.
 // The kernels themselves live in append.cu, decode_simt.cu and decode_tensor.cu.
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -96,6 +97,7 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
     auto up = [](size_t x) { return (x + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign; };
     plan->off_desc = kWorkspaceAlign;
     plan->off_lse = plan->off_desc;
+    plan->off_qrot = 0;
     plan->grid = 0;
     plan->split_tokens = 0;
     plan->max_splits = 1;
@@ -140,6 +142,10 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
         plan->off_o = plan->off_lse;
         plan->bytes = plan->off_lse;
     }
+    if (opt && opt->rope_theta > 0.f) {   // the rotated q of the fused call, from the rotation kernel
+        plan->off_qrot = plan->bytes;
+        plan->bytes += up((size_t)num_seqs * d.num_q_heads * d.head_dim * sizeof(uint16_t));
+    }
     return PA_OK;
 }
 
@@ -177,6 +183,26 @@ extern "C" int pa_append_kv(const pa_bf16* k, const pa_bf16* v, const int64_t* s
         return PA_ERR_INVALID;
     const cudaError_t e = launch_append(k, v, slot_mapping, num_tokens, k_cache, v_cache, *desc,
                                         (cudaStream_t)stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" int pa_rope_append_kv(const pa_bf16* q, pa_bf16* q_out, const pa_bf16* k, const pa_bf16* v,
+                                 const int32_t* positions, const int64_t* slot_mapping,
+                                 int32_t num_tokens, float rope_theta, pa_bf16* k_cache,
+                                 pa_bf16* v_cache, const pa_cache_desc* desc, void* stream) {
+    int rc = check_desc(desc);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0 || !(rope_theta > 0.f) || !(rope_theta < INFINITY)) return PA_ERR_INVALID;
+    if (desc->head_dim != 64 && desc->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!q || !q_out || !k || !v || !positions || !slot_mapping || !k_cache || !v_cache)
+        return PA_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(q_out, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(slot_mapping, 8) ||
+        !aligned(positions, 4))
+        return PA_ERR_INVALID;
+    const cudaError_t e = launch_rope_append(q, q_out, k, v, positions, slot_mapping, num_tokens,
+                                             rope_theta, k_cache, v_cache, *desc, (cudaStream_t)stream);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -223,8 +249,11 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     int rc = check_decode_shape(num_seqs, max_context_len, desc);
     if (rc != PA_OK) return rc;
     if (options && (options->max_ctas < 0 || options->kernel < 0 || options->kernel > 3 ||
-                    (options->flags & ~(PA_FLAG_CHECK | PA_FLAG_PDL)) != 0))
+                    (options->flags & ~(PA_FLAG_CHECK | PA_FLAG_PDL)) != 0 ||
+                    !(options->rope_theta >= 0.f) || !(options->rope_theta < INFINITY)))
         return PA_ERR_INVALID;
+    const float rope_theta = options ? options->rope_theta : 0.f;
+    if (rope_theta > 0.f && !k_new) return PA_ERR_INVALID;   // RoPE needs the new token (pa_append_decode)
     if (num_seqs == 0) return PA_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
         return PA_ERR_INVALID;
@@ -265,10 +294,19 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     p.max_splits = plan.max_splits;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.early = plan.kernel == DecodeKernel::kStream && options && (options->flags & PA_FLAG_PDL) ? 1 : 0;
+    p.rope_theta = plan.kernel == DecodeKernel::kStream ? rope_theta : 0.f;
     cudaError_t e;
     const cudaStream_t st = (cudaStream_t)stream;
     if (k_new && plan.kernel != DecodeKernel::kStream) {   // only the stream kernel fuses the append
-        e = launch_append_at_end(p, st);
+        if (rope_theta > 0.f) {
+            uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws + plan.off_qrot);
+            p.rope_theta = rope_theta;
+            e = launch_rope_append_at_end(p, q_rot, st);
+            p.rope_theta = 0.f;
+            p.q = q_rot;
+        } else {
+            e = launch_append_at_end(p, st);
+        }
         if (e != cudaSuccess) return PA_ERR_CUDA;
         p.k_new = p.v_new = nullptr;
     }

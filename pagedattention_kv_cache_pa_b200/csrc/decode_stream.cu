@@ -70,7 +70,7 @@ struct Hdr {
     int32_t flags, qslot;         // kFirst / kLast / kEmpty / kEnd; q ring slot of the segment
     int32_t nsplit, slot;         // CTAs sharing the sequence; this CTA's partial slot (0/1)
     int32_t i_first, first_slot;  // first CTA of the sequence and the slot it used
-    int32_t pad0, pad1;
+    int32_t rope_pos, pad1;       // RoPE: position of the sequence's newest token (L-1)
 };
 
 // Row of (kv head hl, token t) inside a stage half-tile filled by boxes of tb tokens x 8 heads.
@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
     __shared__ __align__(8) uint64_t empty_bar[C::kStages];
     __shared__ __align__(8) uint64_t qfull_bar[kQSlots];
     __shared__ __align__(8) uint64_t qempty_bar[kQSlots];
+    __shared__ double s_rope_inv[64];   // RoPE inverse frequencies of the D/2 pairs
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t G = p.group;
@@ -128,6 +129,8 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (p.rope_theta > 0.f)
+        for (int i = threadIdx.x; i < D / 2; i += blockDim.x) s_rope_inv[i] = rope_inv_freq(i, D, p.rope_theta);
     __syncthreads();
 
     if (warp == kGroup) {
@@ -262,24 +265,44 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                 if (lane == 0) {
                     s_hdr[st] = Hdr{b, gi * kGroup, t0, valid,
                                     (first ? kFirst : 0) | (last ? kLast : 0) | (L == 0 ? kEmpty : 0),
-                                    seg_q, seg_nsplit, seg_slot, seg_ifirst, seg_fslot, 0, 0};
+                                    seg_q, seg_nsplit, seg_slot, seg_ifirst, seg_fslot, L - 1, 0};
                 }
                 if (valid > 0 && p.k_new != nullptr && j == nb - 1) {
                     // fused append: this slab holds the sequence's newest token (position L-1);
                     // write its K/V rows for the group's 8 kv heads before the slab is loaded
+                    // (K turned by RoPE at that position when the call asks for it)
                     const int32_t pos = L - 1, lbn = pos / Bs;
                     const int32_t blk = __ldg(table + lbn);
                     if (blk >= 0 && blk < p.num_blocks) {
                         constexpr int kChunks = D / 8;                    // 16-byte chunks per row
+                        // the caches are the caller's writable buffers (pa_append_decode)
+                        uint16_t* kc = const_cast<uint16_t*>(p.k_cache);
+                        uint16_t* vc = const_cast<uint16_t*>(p.v_cache);
+                        const size_t row0 = ((size_t)blk * Hkv + gi * kGroup) * Bs + (pos - lbn * Bs);
+                        const size_t src0 = ((size_t)b * Hkv + gi * kGroup) * D;
+                        if (p.rope_theta > 0.f) {
+                            constexpr int kHalfChunks = D / 16;
+                            for (int i = lane; i < kGroup * kHalfChunks; i += 32) {
+                                const int hh = i / kHalfChunks, cc = i - hh * kHalfChunks;
+                                float cs[8], sn[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) rope_cos_sin(pos, s_rope_inv[cc * 8 + e], &cs[e], &sn[e]);
+                                const uint16_t* src = p.k_new + src0 + (size_t)hh * D + cc * 8;
+                                uint4 x1 = __ldg(reinterpret_cast<const uint4*>(src));
+                                uint4 x2 = __ldg(reinterpret_cast<const uint4*>(src + D / 2));
+                                rope_rotate8(x1, x2, cs, sn);
+                                uint16_t* dst = kc + (row0 + (size_t)hh * Bs) * D + cc * 8;
+                                *reinterpret_cast<uint4*>(dst) = x1;
+                                *reinterpret_cast<uint4*>(dst + D / 2) = x2;
+                            }
+                        }
                         for (int i = lane; i < kGroup * kChunks; i += 32) {
                             const int hh = i / kChunks, cc = i - hh * kChunks;
-                            const size_t dst = (((size_t)blk * Hkv + gi * kGroup + hh) * Bs + (pos - lbn * Bs)) * D + cc * 8;
-                            const size_t src = ((size_t)b * Hkv + gi * kGroup + hh) * D + cc * 8;
-                            // the caches are the caller's writable buffers (pa_append_decode)
-                            reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.k_cache) + dst)[0] =
-                                __ldg(reinterpret_cast<const uint4*>(p.k_new + src));
-                            reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.v_cache) + dst)[0] =
-                                __ldg(reinterpret_cast<const uint4*>(p.v_new + src));
+                            const size_t dst = (row0 + (size_t)hh * Bs) * D + cc * 8;
+                            const size_t src = src0 + (size_t)hh * D + cc * 8;
+                            if (p.rope_theta <= 0.f)
+                                reinterpret_cast<uint4*>(kc + dst)[0] = __ldg(reinterpret_cast<const uint4*>(p.k_new + src));
+                            reinterpret_cast<uint4*>(vc + dst)[0] = __ldg(reinterpret_cast<const uint4*>(p.v_new + src));
                         }
                     }
                     // order these generic-proxy writes before the TMA reads of the slab
@@ -372,8 +395,24 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
             if (hd.flags & kFirst) {
                 const int qs = qk % kQSlots;
                 if (!warp_wait(smem_u32(&qfull_bar[qs]), (qk / kQSlots) & 1, p.status)) break;
-                const uint16_t* qsm = reinterpret_cast<const uint16_t*>(
+                uint16_t* qsm = reinterpret_cast<uint16_t*>(
                     smem_gen + (q_base - smem_base) + qs * (size_t)(kGroup * G * D * 2)) + (size_t)warp * G * D;
+                if (p.rope_theta > 0.f) {
+                    // RoPE: turn this warp's G query rows at the newest token's position, in place
+                    for (int i = lane; i < D / 2; i += 32) {
+                        float cs, sn;
+                        rope_cos_sin(hd.rope_pos, s_rope_inv[i], &cs, &sn);
+                        for (int h = 0; h < G; ++h) {
+                            const float x1 = __uint_as_float((uint32_t)qsm[h * D + i] << 16);
+                            const float x2 = __uint_as_float((uint32_t)qsm[h * D + i + D / 2] << 16);
+                            qsm[h * D + i] = f32_to_bf16_rn(x1 * cs - x2 * sn);
+                            qsm[h * D + i + D / 2] = f32_to_bf16_rn(x1 * sn + x2 * cs);
+                        }
+                    }
+                    // generic writes to a slot the bulk copy refills later: order them first
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int h = nt * 8 + r;

@@ -59,6 +59,34 @@ __device__ __forceinline__ int32_t clipped_length(const DecodeParams& p, int32_t
     return L;
 }
 
+// RoPE: pair i (of D/2) at position pos turns by a = pos * theta^(-2i/D).  The
+// inverse frequency theta^(-2i/D) is formed once per CTA in double; the angle
+// is formed and reduced to [-pi, pi] in double (positions reach 2^17, where a
+// float product would already be off by ~1e-2 rad), then cos/sin in float
+// (errors ~5e-7, far below the bf16 rounding of the rotated values).
+// The rotation of (x[i], x[i + D/2]) by a is (x[i] c - x[i + D/2] s, x[i] s + x[i + D/2] c).
+__device__ __forceinline__ double rope_inv_freq(int32_t i, int32_t D, float theta) {
+    return exp2(-2.0 * (double)i / (double)D * log2((double)theta));
+}
+__device__ __forceinline__ void rope_cos_sin(int32_t pos, double inv_freq, float* c, float* s) {
+    const double a = (double)pos * inv_freq;
+    const double two_pi = 6.283185307179586476925286766559;
+    const double r = a - two_pi * rint(a * (1.0 / two_pi));
+    __sincosf((float)r, s, c);   // on [-pi, pi] the hardware form is within ~5e-7 of cos/sin
+}
+// Rotates 8 pairs: x1 = elements [i0, i0 + 8), x2 = the same of the second half.
+__device__ __forceinline__ void rope_rotate8(uint4& x1, uint4& x2, const float* c, const float* s) {
+    uint32_t* a = reinterpret_cast<uint32_t*>(&x1);
+    uint32_t* b = reinterpret_cast<uint32_t*>(&x2);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const float a0 = bf16_lo(a[w]), a1 = bf16_hi(a[w]), b0 = bf16_lo(b[w]), b1 = bf16_hi(b[w]);
+        const int e = 2 * w;
+        a[w] = pack_bf16x2(a0 * c[e] - b0 * s[e], a1 * c[e + 1] - b1 * s[e + 1]);
+        b[w] = pack_bf16x2(a0 * s[e] + b0 * c[e], a1 * s[e + 1] + b1 * c[e + 1]);
+    }
+}
+
 // Writes zeros for the query heads of (b, kv head): the output of an empty context.
 __device__ __forceinline__ void store_zero_group(const DecodeParams& p, int32_t b, int32_t kvh,
                                                  int tid, int nthreads) {

@@ -45,6 +45,7 @@ struct DecodeParams {
     int32_t max_splits;            // S = ceil(max_context_len / C)
     float scale_log2;              // scale * log2(e): scores are kept in the log2 domain
     int32_t early;                 // launched early (PA_FLAG_PDL): prefetch before the wait
+    float rope_theta;              // > 0: rotate q and the new K rows at position L-1 (fused append)
 };
 
 // Which decode kernel a plan runs.
@@ -59,7 +60,7 @@ struct DecodePlan {
     int32_t split_tokens;          // kSimt / kSplit: tokens per split
     int32_t max_splits;            // kSimt / kSplit: splits per (sequence, kv head) at most
     int32_t grid;                  // kStream: persistent CTAs (partial slots: 2 per CTA)
-    size_t off_desc, off_lse, off_o, bytes;
+    size_t off_desc, off_lse, off_o, off_qrot, bytes;
 };
 
 constexpr size_t kWorkspaceAlign = 256;
@@ -72,6 +73,14 @@ cudaError_t launch_append(const pa_bf16* k, const pa_bf16* v, const int64_t* slo
                           pa_bf16* k_cache, pa_bf16* v_cache, const pa_cache_desc& d,
                           cudaStream_t stream);
 cudaError_t launch_append_at_end(const DecodeParams& p, cudaStream_t stream);
+// RoPE + append through the slot mapping (pa_rope_append_kv).
+cudaError_t launch_rope_append(const pa_bf16* q, pa_bf16* q_out, const pa_bf16* k, const pa_bf16* v,
+                               const int32_t* positions, const int64_t* slots, int32_t T, float theta,
+                               pa_bf16* k_cache, pa_bf16* v_cache, const pa_cache_desc& d,
+                               cudaStream_t stream);
+// RoPE + append of each sequence's newest token at position L-1 through the table, with the
+// rotated q written to q_out (the fused call on the kernels that do not fuse it).
+cudaError_t launch_rope_append_at_end(const DecodeParams& p, uint16_t* q_out, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_tensor(const DecodeParams& p, cudaStream_t stream);
 bool tensor_kernel_supports(const pa_cache_desc& d);

@@ -54,15 +54,72 @@ def host_step(b: wl.DecodeBatch):
     return (slots, tables, lens), (o_slots, o_tables, o_lens)
 
 
+def bf16_ulps(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in units in the last place between bf16 bit patterns (adjacent values: 1)."""
+    def ordered(x):
+        x = np.asarray(x, dtype=np.uint16).astype(np.int32)
+        return np.where(x & 0x8000, -(x & 0x7FFF), x & 0x7FFF)
+    return np.abs(ordered(a) - ordered(b))
+
+
+def widen(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def rope_close(gpu_bits: np.ndarray, x_bits: np.ndarray, positions: np.ndarray, theta: float):
+    """RoPE outputs [T, H, D] against the oracle's unrounded rotation of x_bits: each value
+    within 2^-8 |exact| (its bf16 rounding) + 2^-20 (|x[i]| + |x[i + D/2]|) (float cos/sin and
+    products on the pair's inputs; where the rotation cancels, the second term dominates).
+    Returns (ok, worst error / bound)."""
+    exact = oracle.rope(x_bits, positions, theta)
+    x = widen(x_bits)
+    half = x.shape[-1] // 2
+    mag = np.abs(x[..., :half]) + np.abs(x[..., half:])
+    mag = np.concatenate([mag, mag], axis=-1)
+    bound = 2.0 ** -8 * np.abs(exact) + 2.0 ** -20 * mag + 1e-30
+    ratio = np.abs(widen(gpu_bits) - exact) / bound
+    return bool(np.all(ratio <= 1.0)), float(ratio.max())
+
+
+def pool_rows(shape, slots) -> np.ndarray:
+    """Mask of the pool rows ([N, Hkv, Bs, D] broadcast) that the given slots address."""
+    N, Hkv, Bs, D = shape
+    rows = np.zeros((N, Bs), dtype=bool)
+    for sl in np.asarray(slots):
+        if 0 <= sl < N * Bs:
+            rows[sl // Bs, sl % Bs] = True
+    return np.broadcast_to(rows[:, None, :, None], shape)
+
+
+def rope_pool_matches(gpu: np.ndarray, initial: np.ndarray, k_new: np.ndarray, slots, positions,
+                      theta: float) -> bool:
+    """K pool after a RoPE append: bytes outside the slots' rows unchanged from `initial`, and
+    each slot's rows the rotation of its token's K within rope_close's bound."""
+    mask = pool_rows(initial.shape, slots)
+    if not np.array_equal(gpu[~mask], initial[~mask]):
+        return False
+    Bs = initial.shape[2]
+    for t, sl in enumerate(np.asarray(slots)):
+        if 0 <= sl < initial.shape[0] * Bs:
+            got = gpu[sl // Bs, :, sl % Bs, :][None]
+            ok, _ = rope_close(got, k_new[t:t + 1], positions[t:t + 1], theta)
+            if not ok:
+                return False
+    return True
+
+
 def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int = 0,
              max_ctas: int = 0, check_pool: bool = True, sample=None, fused: bool = False,
-             pdl: bool = False):
+             pdl: bool = False, rope_theta: float = 0.0):
     """Runs one step on both sides; returns a dict of results and checks.
 
     fused=False: pa_append_kv through the host slot mapping, then pa_decode.
     fused=True: pa_append_decode (append at position L-1 through the table, then decode).
     pdl=True: PA_FLAG_PDL (the decode kernel may start while the append kernel runs).
+    rope_theta > 0 (fused only): q and the new K rows turned by RoPE at position L-1; the
+    rotated K rows are held to rope_close's bound, every other byte must be identical.
     """
+    assert rope_theta == 0.0 or fused
     (slots, tables, lens), (o_slots, o_tables, o_lens) = host_step(b)
     assert np.array_equal(slots, o_slots), "slot mapping differs from the model"
     assert np.array_equal(tables, o_tables), "block tables differ from the model"
@@ -75,7 +132,8 @@ def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int =
     out = torch.empty_like(q)
     max_len = int(lens.max()) if lens.size else 0
     opts = pa.DecodeOptions(split_tokens=split_tokens, kernel=kernel, max_ctas=max_ctas,
-                            flags=pa.PA_FLAG_CHECK | (pa.PA_FLAG_PDL if pdl else 0))
+                            flags=pa.PA_FLAG_CHECK | (pa.PA_FLAG_PDL if pdl else 0),
+                            rope_theta=rope_theta)
     ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, max_len, desc, opts), dtype=torch.uint8,
                      device=DEV)
     if fused:
@@ -89,18 +147,30 @@ def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int =
                      torch.from_numpy(lens).to(DEV), max_len, b.scale, out, ws, desc, opts)
     torch.cuda.synchronize()
 
-    ref_k, ref_v = oracle.append_kv(b.k_new, b.v_new, o_slots, b.k_cache, b.v_cache)
+    if rope_theta > 0:
+        _, ref_k, ref_v, q_ref = oracle.rope_append_decode(b.q, b.k_new, b.v_new, o_slots, b.k_cache,
+                                                           b.v_cache, o_tables, o_lens, b.scale,
+                                                           rope_theta)
+    else:
+        ref_k, ref_v = oracle.append_kv(b.k_new, b.v_new, o_slots, b.k_cache, b.v_cache)
+        q_ref = b.q
     res = {"splits": pa.pa_decode_max_splits(b.batch, max_len, desc, opts)}
     if check_pool:
-        res["pool_equal"] = (np.array_equal(to_host_bits(k_cache), ref_k) and
-                             np.array_equal(to_host_bits(v_cache), ref_v))
+        if rope_theta > 0:
+            pos = np.maximum(o_lens - 1, 0).astype(np.int32)
+            res["pool_equal"] = (rope_pool_matches(to_host_bits(k_cache), b.k_cache, b.k_new, o_slots,
+                                                   pos, rope_theta) and
+                                 np.array_equal(to_host_bits(v_cache), ref_v))
+        else:
+            res["pool_equal"] = (np.array_equal(to_host_bits(k_cache), ref_k) and
+                                 np.array_equal(to_host_bits(v_cache), ref_v))
     got = out.float().cpu().numpy().astype(np.float64)
     if sample is None:
-        ref = oracle.paged_decode(b.q, ref_k, ref_v, o_tables, o_lens, b.scale)
+        ref = oracle.paged_decode(q_ref, ref_k, ref_v, o_tables, o_lens, b.scale)
         res["ok"], res["excess"] = oracle.within_tolerance(got, ref)
     else:
         idx = np.asarray(sample)
-        ref = oracle.paged_decode(b.q[idx], ref_k, ref_v, o_tables[idx], o_lens[idx], b.scale)
+        ref = oracle.paged_decode(q_ref[idx], ref_k, ref_v, o_tables[idx], o_lens[idx], b.scale)
         res["ok"], res["excess"] = oracle.within_tolerance(got[idx], ref)
     res["out"] = got
     res["finite"] = bool(np.isfinite(got).all())

@@ -78,6 +78,28 @@ def test_decode_rejects_unsupported_shapes_without_a_gpu():
                                 1 << 20, ctypes.byref(d), ctypes.byref(o), None) == -1, bad
 
 
+def test_rope_append_rejects_bad_arguments_without_a_gpu():
+    lib = binding.lib
+    fake = ctypes.c_void_p(0x10000)
+    d = _desc()
+    args = lambda n, theta, dd: (fake, fake, fake, fake, fake, fake, n, ctypes.c_float(theta), fake, fake,
+                                 ctypes.byref(dd), None)
+    assert lib.pa_rope_append_kv(*args(1, 0.0, d)) == -1            # theta must be > 0
+    assert lib.pa_rope_append_kv(*args(1, -5.0, d)) == -1
+    assert lib.pa_rope_append_kv(*args(1, float("nan"), d)) == -1
+    assert lib.pa_rope_append_kv(*args(1, float("inf"), d)) == -1
+    assert lib.pa_rope_append_kv(*args(-1, 10000.0, d)) == -1
+    assert lib.pa_rope_append_kv(*args(1, 10000.0, _desc(head_dim=96))) == -2
+    assert lib.pa_rope_append_kv(*args(0, 10000.0, d)) == 0          # nothing to do
+    mis = ctypes.c_void_p(0x10002)                                  # q not 16-byte aligned
+    assert lib.pa_rope_append_kv(mis, fake, fake, fake, fake, fake, 1, ctypes.c_float(1e4), fake, fake,
+                                 ctypes.byref(d), None) == -1
+    for bad in (-1.0, float("nan")):                                 # decode options too
+        o = pa.DecodeOptions(rope_theta=bad)
+        assert lib.pa_decode_ex(fake, fake, fake, fake, fake, 1, 16, ctypes.c_float(0.1), fake, fake,
+                                1 << 20, ctypes.byref(d), ctypes.byref(o), None) == -1, bad
+
+
 def test_slot_mapping_entry_matches_oracle():
     import oracle
     rng = np.random.default_rng(0)
