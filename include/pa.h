@@ -318,6 +318,57 @@ PA_API const int32_t* pa_bm_context_lens(const pa_block_manager* bm);
 /* Rows whose table changed since the last call (up to cap, ascending); returns the count. */
 PA_API int32_t pa_bm_take_dirty_rows(pa_block_manager* bm, int32_t* rows, int32_t cap);
 
+/*
+ * ---- prefix caching and copy-on-write ----
+ * The Nano-vLLM page ("Nano-vLLM로 배우는 vLLM 추론 엔진 작동 원리 한눈에 정리",
+ * section "KV 캐시와 Block Manager") reuses the blocks of a shared prompt
+ * prefix, identified by a hash, without recomputing them.  Here a FULL block
+ * is identified by the 64-bit FNV-1a hash of its parent block's hash (8 bytes,
+ * little-endian; 0 for the first block) followed by its Bs token ids (4 bytes
+ * each, little-endian); a lookup hits only when the stored ids are equal too.
+ * Copy-on-write follows the OS paging the vLLM overview page likens the pool
+ * to (section "PagedAttention — OS 가상 메모리에서 영감"): an append into a
+ * block that several tables hold first moves the writer to a fresh block.
+ * Free-list policy: a block freed without a hash returns to the top (the
+ * stack above, unchanged); a freed hashed block stays cached at the bottom
+ * (a sequence's blocks tail first, so a prefix outlives its extensions) until
+ * allocation reaches it, which evicts its hash.  A sequence's blocks are
+ * hashed while every token it holds has an id (admitted by
+ * pa_bm_add_seq_tokens, grown by pa_bm_append_token_ids, or forked whole from
+ * such a sequence); a block is registered when it fills, unless its hash is
+ * already registered.  The caller fills the KV of the blocks that were not
+ * found cached (prefill) and runs the reported copies (pa_copy_blocks) before
+ * the appends that follow them.
+ */
+/* Admit a sequence by its num_tokens token ids; the blocks of its longest cached prefix of
+ * full blocks are shared, the rest are fresh.  *num_cached_tokens (may be NULL) receives the
+ * number of tokens found cached (a multiple of Bs).  All-or-nothing: PA_ERR_OOM_BLOCKS when the
+ * free list cannot cover the fresh blocks (cached free blocks that hit do not count as fresh). */
+PA_API int pa_bm_add_seq_tokens(pa_block_manager* bm, int32_t seq, const int32_t* token_ids,
+                                int32_t num_tokens, int32_t* num_cached_tokens);
+/* Admit seq as a copy of src sharing every block, its partial last block included (for
+ * parallel sampling); the first append of either into the shared partial block copies it. */
+PA_API int pa_bm_fork_all(pa_block_manager* bm, int32_t seq, int32_t src);
+/* pa_bm_append_tokens with token ids and copy-on-write: token token_ids[i] is appended to
+ * seqs[i] (n distinct sequences) and slots[i] receives its slot.  When the token lands in a
+ * block other tables also hold, the sequence gets a fresh block first and the pair (old,
+ * fresh) is written to copies[2 k], copies[2 k + 1] (capacity 2 n), k < *num_copies.
+ * All-or-nothing on PA_ERR_OOM_BLOCKS. */
+PA_API int pa_bm_append_token_ids(pa_block_manager* bm, const int32_t* seqs, const int32_t* token_ids,
+                                  int32_t n, int64_t* slots, int32_t* copies, int32_t* num_copies);
+/* Number of registered (hash-identified) blocks, in use or cached free. */
+PA_API int32_t pa_bm_num_cached_blocks(const pa_block_manager* bm);
+
+/*
+ * Device side of copy-on-write: for k < n, block copies[2 k + 1] of k_cache and of v_cache
+ * receives a bit-exact copy of block copies[2 k] (all kv heads, all Bs slots).  copies is a
+ * device int32 array [n][2]; ids outside [0, num_blocks) skip that pair; destinations must
+ * be distinct and no destination may be a source of another pair.  Caches 16-byte aligned,
+ * head_dim a multiple of 8.  n == 0 is a no-op.  Errors: PA_ERR_INVALID, PA_ERR_CUDA.
+ */
+PA_API int pa_copy_blocks(pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* copies, int32_t n,
+                          const pa_cache_desc* desc, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

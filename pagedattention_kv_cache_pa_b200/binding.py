@@ -114,6 +114,16 @@ lib.pa_bm_context_lens.argtypes = [_vp]
 lib.pa_bm_context_lens.restype = ctypes.POINTER(ctypes.c_int32)
 lib.pa_bm_take_dirty_rows.argtypes = [_vp, _vp, _i32]
 lib.pa_bm_take_dirty_rows.restype = _i32
+lib.pa_bm_add_seq_tokens.argtypes = [_vp, _i32, _vp, _i32, _vp]
+lib.pa_bm_add_seq_tokens.restype = ctypes.c_int
+lib.pa_bm_fork_all.argtypes = [_vp, _i32, _i32]
+lib.pa_bm_fork_all.restype = ctypes.c_int
+lib.pa_bm_append_token_ids.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _vp]
+lib.pa_bm_append_token_ids.restype = ctypes.c_int
+lib.pa_bm_num_cached_blocks.argtypes = [_vp]
+lib.pa_bm_num_cached_blocks.restype = _i32
+lib.pa_copy_blocks.argtypes = [_vp, _vp, _vp, _i32, _DESC, _vp]
+lib.pa_copy_blocks.restype = ctypes.c_int
 
 
 def pa_status_string(status: int) -> str:
@@ -184,6 +194,14 @@ def pa_rope_append_kv(q, q_out, k, v, positions, slot_mapping, rope_theta: float
                                  _dev(slot_mapping, "int64", "slot_mapping"), n, float(rope_theta),
                                  _dev(k_cache, "bfloat16", "k_cache"), _dev(v_cache, "bfloat16", "v_cache"),
                                  ctypes.byref(desc), _stream(stream)), "pa_rope_append_kv")
+
+
+def pa_copy_blocks(k_cache, v_cache, copies, desc: CacheDesc, stream=None) -> None:
+    """Device copy-on-write: copies is a device int32 [n, 2] tensor of (src, dst) block pairs."""
+    n = int(copies.shape[0])
+    _check(lib.pa_copy_blocks(_dev(k_cache, "bfloat16", "k_cache"), _dev(v_cache, "bfloat16", "v_cache"),
+                              _dev(copies, "int32", "copies") if n else None, n, ctypes.byref(desc),
+                              _stream(stream)), "pa_copy_blocks")
 
 
 def pa_decode_workspace_size(num_seqs: int, max_context_len: int, desc: CacheDesc,
@@ -309,6 +327,34 @@ class BlockManager:
         _check(lib.pa_bm_append_tokens(self._h, s.ctypes.data, int(s.size), slots.ctypes.data),
                "pa_bm_append_tokens")
         return slots
+
+    def add_seq_tokens(self, seq: int, token_ids) -> int:
+        """Admit by token ids (prefix caching); returns the number of tokens found cached."""
+        t = _host(np.asarray(token_ids, dtype=np.int32), np.int32, "token_ids")
+        cached = ctypes.c_int32(0)
+        _check(lib.pa_bm_add_seq_tokens(self._h, int(seq), t.ctypes.data if t.size else None,
+                                        int(t.size), ctypes.byref(cached)), "pa_bm_add_seq_tokens")
+        return int(cached.value)
+
+    def fork_all(self, seq: int, src: int) -> None:
+        _check(lib.pa_bm_fork_all(self._h, int(seq), int(src)), "pa_bm_fork_all")
+
+    def append_token_ids(self, seqs, token_ids):
+        """Appends with ids and copy-on-write; returns (slots int64 [n], copies int32 [k, 2])."""
+        s = _host(np.asarray(seqs, dtype=np.int32), np.int32, "seqs")
+        t = _host(np.asarray(token_ids, dtype=np.int32), np.int32, "token_ids")
+        if s.size != t.size:
+            raise ValueError("seqs and token_ids differ in length")
+        slots = np.empty(s.size, dtype=np.int64)
+        copies = np.empty((max(s.size, 1), 2), dtype=np.int32)
+        nc = ctypes.c_int32(0)
+        _check(lib.pa_bm_append_token_ids(self._h, s.ctypes.data, t.ctypes.data, int(s.size),
+                                          slots.ctypes.data, copies.ctypes.data, ctypes.byref(nc)),
+               "pa_bm_append_token_ids")
+        return slots, copies[:nc.value].copy()
+
+    def num_cached_blocks(self) -> int:
+        return int(lib.pa_bm_num_cached_blocks(self._h))
 
     def num_free(self) -> int:
         return int(lib.pa_bm_num_free(self._h))

@@ -206,6 +206,19 @@ extern "C" int pa_rope_append_kv(const pa_bf16* q, pa_bf16* q_out, const pa_bf16
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+extern "C" int pa_copy_blocks(pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* copies, int32_t n,
+                              const pa_cache_desc* desc, void* stream) {
+    int rc = check_desc(desc);
+    if (rc != PA_OK) return rc;
+    if (n < 0 || desc->head_dim % 8 != 0) return PA_ERR_INVALID;
+    if (n == 0) return PA_OK;
+    if (!k_cache || !v_cache || !copies || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(copies, 4))
+        return PA_ERR_INVALID;
+    const cudaError_t e = launch_copy_blocks(k_cache, v_cache, copies, n, *desc, (cudaStream_t)stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 static int check_decode_shape(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc* d) {
     int rc = check_desc(d);
     if (rc != PA_OK) return rc;

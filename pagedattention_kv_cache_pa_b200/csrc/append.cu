@@ -68,7 +68,39 @@ __global__ void __launch_bounds__(256) append_at_end_kernel(const DecodeParams p
     }
 }
 
+// Copy-on-write on the device: pair k copies block copies[2k] onto block copies[2k+1] in
+// both caches (a block is Hkv x Bs x D contiguous elements), 16 bytes per thread.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_cache,
+                                                          uint4* __restrict__ v_cache,
+                                                          const int32_t* __restrict__ copies,
+                                                          int32_t n, int64_t chunks_per_block,
+                                                          int32_t num_blocks) {
+    allow_dependents();
+    const int64_t total = (int64_t)n * chunks_per_block;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t pair = i / chunks_per_block, c = i - pair * chunks_per_block;
+        const int32_t src = copies[2 * pair], dst = copies[2 * pair + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) continue;
+        k_cache[dst * chunks_per_block + c] = k_cache[src * chunks_per_block + c];
+        v_cache[dst * chunks_per_block + c] = v_cache[src * chunks_per_block + c];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_copy_blocks(pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* copies, int32_t n,
+                               const pa_cache_desc& d, cudaStream_t stream) {
+    const int64_t cpb = (int64_t)d.num_kv_heads * d.block_size * d.head_dim / 8;
+    const int64_t total = (int64_t)n * cpb;
+    if (total == 0) return cudaSuccess;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    copy_blocks_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        reinterpret_cast<uint4*>(k_cache), reinterpret_cast<uint4*>(v_cache), copies, n, cpb,
+        d.num_blocks);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_append_at_end(const DecodeParams& p, cudaStream_t stream) {
     const int64_t total = (int64_t)p.num_seqs * p.num_kv_heads * (p.head_dim / 8);

@@ -73,6 +73,8 @@ cudaError_t launch_append(const pa_bf16* k, const pa_bf16* v, const int64_t* slo
                           pa_bf16* k_cache, pa_bf16* v_cache, const pa_cache_desc& d,
                           cudaStream_t stream);
 cudaError_t launch_append_at_end(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_copy_blocks(pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* copies, int32_t n,
+                               const pa_cache_desc& d, cudaStream_t stream);
 // RoPE + append through the slot mapping (pa_rope_append_kv).
 cudaError_t launch_rope_append(const pa_bf16* q, pa_bf16* q_out, const pa_bf16* k, const pa_bf16* v,
                                const int32_t* positions, const int64_t* slots, int32_t T, float theta,
