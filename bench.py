@@ -55,6 +55,9 @@ WORKLOAD_TEXT = {
     "c5": "continuous-batching trace: 16 layers (own pools), 256 live sequences, lognormal L (median 512, "
           "sigma 1, <=16384), 100 decode steps, finish p=0.01 per step with replacement, Hq=32, Hkv=8, "
           "D=64, Bs=16",
+    "pc": "prefix caching + copy-on-write: host admission by token ids of 32 C3-shaped requests "
+          "(1024-token shared prefix + suffix~U[256,7168], Bs=256); device copy of 8192 random "
+          "blocks of the C2 geometry (Hkv=8, Bs=16, D=64) per step",
 }
 
 
@@ -64,7 +67,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4", "c5"], default="c2")
+    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4", "c5", "pc"], default="c2",
+                    help="pc: prefix caching + copy-on-write (host admission by token ids on the "
+                         "C3 request mix, device block copies)")
     ap.add_argument("--trace-steps", type=int, default=200,
                     help="c5: decode steps timed (the 100-step trace replayed as needed)")
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "split"], default="auto")
@@ -210,6 +215,31 @@ def run_reference(args, rank):
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "seq-steps/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
+    if args.config == "pc":
+        # the model of the prefix-caching manager admitting the C3 request mix by token ids
+        rng = np.random.default_rng(wl.CONFIG_SEED_BASE + 31)
+        prefix = [int(t) for t in rng.integers(0, 128256, 1024)]
+        reqs = [prefix + [int(t) for t in rng.integers(0, 128256, int(rng.integers(256, 7169)))]
+                for _ in range(32)]
+        nb = sum(-(-len(r) // 256) for r in reqs) + 64
+        m = oracle.BlockManagerModel(nb, 256, 32, 40, list(range(nb)))
+        n, t0 = 0, time.perf_counter()
+        while n < max(1, args.steps) * 32 and time.perf_counter() - t0 < 30.0:
+            for s, r in enumerate(reqs):
+                m.add_seq_tokens(s, r)
+            for s in range(32):
+                m.free_seq(s)
+            n += 32
+        dt = time.perf_counter() - t0
+        v = n / dt
+        return {"metric": "prefix-cached admissions/s (host model)", "value": v, "unit": "admissions/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(n, 1),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": WORKLOAD_TEXT["pc"], "config": "pc"},
+                "cpu_baseline": {"value": v, "unit": "admissions/s", "cores": 1, "kind": "oracle",
+                                 "sample": "%d admissions of the C3 mix by the Python model, %.1f s" % (n, dt)},
+                "e2e": {"value": v, "unit": "admissions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     b = wl.CONFIGS[args.config]()
     B, Bs = b.batch, b.block_size
     model = oracle.BlockManagerModel(b.num_blocks, Bs, B, b.max_blocks_per_seq, b.free_order)
@@ -693,6 +723,86 @@ def cpu_baseline_c5(t, tables, lens, budget_s):
                       "value scaled to all %d layers" % (n, dt, t.layers)}
 
 
+def run_pc(args, rank, world, dist):
+    """Prefix caching + copy-on-write: a step is one pa_copy_blocks of 8192 block pairs (K and
+    V) on the device; the host side times admission by token ids of the C3 request mix."""
+    import torch
+    import pagedattention_kv_cache_pa_b200 as pa
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    # host: C3 mix, admitted by token ids, released, admitted again (steady state)
+    rng = np.random.default_rng(wl.CONFIG_SEED_BASE + 31)
+    Bs3, reqs = 256, []
+    prefix = [int(t) for t in rng.integers(0, 128256, 1024)]
+    for _ in range(32):
+        reqs.append(np.asarray(prefix + [int(t) for t in rng.integers(0, 128256, int(rng.integers(256, 7169)))],
+                               dtype=np.int32))
+    blocks_needed = sum(-(-len(r) // Bs3) for r in reqs)
+    bm = pa.BlockManager(blocks_needed + 64, Bs3, 32, 40, np.arange(blocks_needed + 64, dtype=np.int32))
+    rounds, cached, total = 0, 0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < 1.0 or rounds < 3:
+        for s, r in enumerate(reqs):
+            c = bm.add_seq_tokens(s, r)
+            if rounds >= 1:
+                cached += c
+                total += len(r)
+        for s in range(32):
+            bm.free_seq(s)
+        rounds += 1
+    host_s = time.perf_counter() - t0
+    bm.close()
+    # device: block copies of the C2 geometry
+    Hkv, Bs, D, P = 8, 16, 64, 8192
+    N = 2 * P + 1024
+    desc = pa.CacheDesc.make(num_blocks=N, block_size=Bs, num_kv_heads=Hkv, num_q_heads=32,
+                             head_dim=D, max_blocks_per_seq=1)
+    kc = torch.empty((N, Hkv, Bs, D), dtype=torch.bfloat16, device=dev).normal_()
+    vc = torch.empty_like(kc).normal_()
+    perm = np.random.default_rng(3).permutation(N)
+    pairs = torch.from_numpy(np.stack([perm[:P], perm[P:2 * P]], 1).astype(np.int32)).to(dev)
+    for _ in range(args.warmup):
+        pa.pa_copy_blocks(kc, vc, pairs, desc, stream=stream)
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
+    e0.record(stream)
+    for _ in range(K):
+        pa.pa_copy_blocks(kc, vc, pairs, desc, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+    if rank != 0:
+        return None
+    bytes_step = 2 * 2 * P * Hkv * Bs * D * 2            # K and V, read + write
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_step / (ms / K / 1e3) / 1e9
+    return {
+        "metric": "copy-on-write block copies/s (device) and prefix-cached admissions/s (host)",
+        "value": world * P * K / (ms / 1e3), "unit": "blocks/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT["pc"], "config": "pc", "pairs": P,
+                   "l2": "inputs larger than L2: %d MB read per step" % (bytes_step // 2 // 1000000)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                     "kernel": "pa_copy_blocks", "algorithmic_bytes_per_launch": bytes_step,
+                     "avg_launch_ms": ms / K},
+        "host": {"admissions_per_s": rounds * 32 / host_s, "rounds": rounds,
+                 "cached_token_fraction": cached / max(total, 1),
+                 "prefix_token_fraction": 1024 * 32 / max(sum(len(r) for r in reqs), 1)},
+        "e2e": None, "gpu_launches": K, "clocks": clk,
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -712,7 +822,8 @@ def main(argv=None):
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = dist_mod
     try:
-        res = (run_c5 if args.config == "c5" else run_ours)(args, rank, world, dist)
+        runner = {"c5": run_c5, "pc": run_pc}.get(args.config, run_ours)
+        res = runner(args, rank, world, dist)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

@@ -159,6 +159,15 @@ def _dev(t, dtype_name: str, what: str):
     return t.data_ptr()
 
 
+def _cache(t, desc: "CacheDesc", what: str):
+    """Device pointer of a KV cache tensor that holds at least the pool desc describes."""
+    if t is not None and not isinstance(t, int):
+        need = int(desc.num_blocks) * desc.num_kv_heads * desc.block_size * desc.head_dim
+        if t.numel() < need:
+            raise ValueError("%s holds %d elements, the pool described needs %d" % (what, t.numel(), need))
+    return _dev(t, "bfloat16", what)
+
+
 def _stream(stream):
     if stream is None:
         import torch
@@ -181,7 +190,7 @@ def pa_append_kv(k, v, slot_mapping, k_cache, v_cache, desc: CacheDesc, stream=N
     n = int(slot_mapping.shape[0]) if num_tokens is None else int(num_tokens)
     _check(lib.pa_append_kv(_dev(k, "bfloat16", "k"), _dev(v, "bfloat16", "v"),
                             _dev(slot_mapping, "int64", "slot_mapping"), n,
-                            _dev(k_cache, "bfloat16", "k_cache"), _dev(v_cache, "bfloat16", "v_cache"),
+                            _cache(k_cache, desc, "k_cache"), _cache(v_cache, desc, "v_cache"),
                             ctypes.byref(desc), _stream(stream)), "pa_append_kv")
 
 
@@ -192,14 +201,14 @@ def pa_rope_append_kv(q, q_out, k, v, positions, slot_mapping, rope_theta: float
                                  _dev(k, "bfloat16", "k"), _dev(v, "bfloat16", "v"),
                                  _dev(positions, "int32", "positions"),
                                  _dev(slot_mapping, "int64", "slot_mapping"), n, float(rope_theta),
-                                 _dev(k_cache, "bfloat16", "k_cache"), _dev(v_cache, "bfloat16", "v_cache"),
+                                 _cache(k_cache, desc, "k_cache"), _cache(v_cache, desc, "v_cache"),
                                  ctypes.byref(desc), _stream(stream)), "pa_rope_append_kv")
 
 
 def pa_copy_blocks(k_cache, v_cache, copies, desc: CacheDesc, stream=None) -> None:
     """Device copy-on-write: copies is a device int32 [n, 2] tensor of (src, dst) block pairs."""
     n = int(copies.shape[0])
-    _check(lib.pa_copy_blocks(_dev(k_cache, "bfloat16", "k_cache"), _dev(v_cache, "bfloat16", "v_cache"),
+    _check(lib.pa_copy_blocks(_cache(k_cache, desc, "k_cache"), _cache(v_cache, desc, "v_cache"),
                               _dev(copies, "int32", "copies") if n else None, n, ctypes.byref(desc),
                               _stream(stream)), "pa_copy_blocks")
 
@@ -225,8 +234,8 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: 
     n = int(context_lens.shape[0]) if num_seqs is None else int(num_seqs)
     wbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else int(workspace_bytes)
     ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
-    _check(lib.pa_decode_ex(_dev(q, "bfloat16", "q"), _dev(k_cache, "bfloat16", "k_cache"),
-                            _dev(v_cache, "bfloat16", "v_cache"),
+    _check(lib.pa_decode_ex(_dev(q, "bfloat16", "q"), _cache(k_cache, desc, "k_cache"),
+                            _cache(v_cache, desc, "v_cache"),
                             _dev(block_tables, "int32", "block_tables"),
                             _dev(context_lens, "int32", "context_lens"), n, int(max_context_len),
                             float(scale), _dev(out, "bfloat16", "out"), ws, wbytes,
@@ -244,8 +253,8 @@ def pa_append_decode(q, k, v, k_cache, v_cache, block_tables, context_lens, max_
     wbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else int(workspace_bytes)
     ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
     _check(lib.pa_append_decode(_dev(q, "bfloat16", "q"), _dev(k, "bfloat16", "k"),
-                                _dev(v, "bfloat16", "v"), _dev(k_cache, "bfloat16", "k_cache"),
-                                _dev(v_cache, "bfloat16", "v_cache"),
+                                _dev(v, "bfloat16", "v"), _cache(k_cache, desc, "k_cache"),
+                                _cache(v_cache, desc, "v_cache"),
                                 _dev(block_tables, "int32", "block_tables"),
                                 _dev(context_lens, "int32", "context_lens"), n,
                                 int(max_context_len), float(scale), _dev(out, "bfloat16", "out"), ws,
@@ -259,8 +268,8 @@ def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, max_conte
                       stream=None, num_seqs: int | None = None) -> None:
     """pa_decode with the library's fixed scratch array instead of a caller workspace."""
     n = int(context_lens.shape[0]) if num_seqs is None else int(num_seqs)
-    _check(lib.pa_decode_noalloc(_dev(q, "bfloat16", "q"), _dev(k_cache, "bfloat16", "k_cache"),
-                                 _dev(v_cache, "bfloat16", "v_cache"),
+    _check(lib.pa_decode_noalloc(_dev(q, "bfloat16", "q"), _cache(k_cache, desc, "k_cache"),
+                                 _cache(v_cache, desc, "v_cache"),
                                  _dev(block_tables, "int32", "block_tables"),
                                  _dev(context_lens, "int32", "context_lens"), n,
                                  int(max_context_len), float(scale), _dev(out, "bfloat16", "out"),

@@ -100,6 +100,17 @@ def test_rope_append_rejects_bad_arguments_without_a_gpu():
                                 1 << 20, ctypes.byref(d), ctypes.byref(o), None) == -1, bad
 
 
+def test_binding_refuses_caches_smaller_than_the_pool():
+    import torch
+    d = _desc()                                         # 8 blocks x 1 head x 16 x 64
+    small = torch.zeros(8 * 16 * 64 - 1, dtype=torch.bfloat16)
+    pairs = torch.zeros((1, 2), dtype=torch.int32)
+    with pytest.raises(ValueError):
+        pa.pa_copy_blocks(small, small, pairs, d)
+    with pytest.raises(ValueError):
+        pa.pa_append_kv(small, small, torch.zeros(1, dtype=torch.int64), small, small, d)
+
+
 def test_slot_mapping_entry_matches_oracle():
     import oracle
     rng = np.random.default_rng(0)
