@@ -66,6 +66,17 @@ def _lib():
         lib.oracle_rope.restype = None
         lib.oracle_round_bf16.argtypes = [vp, i64, vp]
         lib.oracle_round_bf16.restype = None
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = dbl
+        lib.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_from_float.restype = ctypes.c_uint8
+        lib.oracle_quantize_e4m3.argtypes = [vp, i64, ctypes.c_float, vp]
+        lib.oracle_quantize_e4m3.restype = None
+        lib.oracle_append_kv_e4m3.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, vp, vp]
+        lib.oracle_append_kv_e4m3.restype = None
+        lib.oracle_paged_decode_e4m3.argtypes = [vp, vp, vp, dbl, dbl, vp, vp, i64, i64, i64, i64, i64,
+                                                 i64, dbl, vp]
+        lib.oracle_paged_decode_e4m3.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_num_threads.restype = None
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -230,3 +241,61 @@ def rope_append_decode(q, k_new, v_new, slots, k_cache, v_cache, block_tables, c
     k_rot = rope_bf16(k_new, pos, theta)
     kc, vc = append_kv(k_rot, v_new, slots, k_cache, v_cache)
     return paged_decode(q_rot, kc, vc, block_tables, lens, scale), kc, vc, q_rot
+
+
+def e4m3_to_double(codes) -> np.ndarray:
+    """Value of each E4M3 code (NaN for the NaN codes)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    lib = _lib()
+    return np.array([lib.oracle_e4m3_to_double(int(x)) for x in c.ravel()], dtype=np.float64).reshape(c.shape)
+
+
+def e4m3_from_float(y) -> np.ndarray:
+    """E4M3 code of each float32 value: nearest, ties to even, saturating at +-448."""
+    y = np.asarray(y, dtype=np.float32)
+    lib = _lib()
+    return np.array([lib.oracle_e4m3_from_float(float(v)) for v in y.ravel()], dtype=np.uint8).reshape(y.shape)
+
+
+def inv_scale(scale: float) -> np.float32:
+    """float(1 / scale), the multiplier that quantization applies (both sides form it in float)."""
+    return np.float32(1.0) / np.float32(scale)
+
+
+def quantize_e4m3(x: np.ndarray, scale: float) -> np.ndarray:
+    """E4M3 codes of bf16 values x: e4m3(float(x) * float(1/scale))."""
+    x = _c(x, np.uint16)
+    out = np.empty(x.shape, dtype=np.uint8)
+    _lib().oracle_quantize_e4m3(x.ctypes.data, x.size, float(inv_scale(scale)), out.ctypes.data)
+    return out
+
+
+def append_kv_e4m3(k_codes, v_codes, slot_mapping_, k_cache, v_cache):
+    """Write each token's (already quantized) K/V codes into its slot of u8 pools (copies)."""
+    k = _c(k_codes, np.uint8)
+    v = _c(v_codes, np.uint8)
+    sm = _c(slot_mapping_, np.int64)
+    kc, vc = k_cache.copy(), v_cache.copy()
+    N, Hkv, Bs, D = kc.shape
+    _lib().oracle_append_kv_e4m3(k.ctypes.data, v.ctypes.data, sm.ctypes.data, sm.shape[0], Hkv, D, Bs, N,
+                                 kc.ctypes.data, vc.ctypes.data)
+    return kc, vc
+
+
+def paged_decode_e4m3(q, k_cache, v_cache, k_scale: float, v_scale: float, block_tables, context_lens,
+                      scale: float):
+    """fp64 [B, Hq, D] attention over E4M3 pools (values = code value x scale)."""
+    q = _c(q, np.uint16)
+    kc = _c(k_cache, np.uint8)
+    vc = _c(v_cache, np.uint8)
+    bt = _c(block_tables, np.int32)
+    lens = _c(context_lens, np.int32)
+    B, Hq, D = q.shape
+    N, Hkv, Bs, _ = kc.shape
+    out = np.empty((B, Hq, D), dtype=np.float64)
+    rc = _lib().oracle_paged_decode_e4m3(q.ctypes.data, kc.ctypes.data, vc.ctypes.data, float(k_scale),
+                                         float(v_scale), bt.ctypes.data, lens.ctypes.data, B, Hq, Hkv, D,
+                                         Bs, bt.shape[1], float(scale), out.ctypes.data)
+    if rc != 0:
+        raise RuntimeError("oracle_paged_decode_e4m3 failed (%d)" % rc)
+    return out

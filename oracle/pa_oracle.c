@@ -359,3 +359,136 @@ void oracle_round_bf16(const double* x, int64_t n, uint16_t* out) {
         out[k] = (uint16_t)(u >> 16);
     }
 }
+
+/*
+ * ---- FP8 KV cache (e4m3) ----
+ * "[Hacker News 요약] ... Tiny-vLLM ..." (aisleshub), section "향후 전망", names
+ * FP8 among the data types to support next, with no format or scale scheme.
+ * Reading (stated, not derived): the OCP 8-bit floating-point E4M3 format --
+ * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
+ * exponent and mantissa all ones = NaN, largest finite 448, subnormals
+ * m * 2^-9 -- with one scale per cache tensor.  A bf16 value x is stored as
+ * code = e4m3(y), y = float(x) * float(1/scale) formed in float (that
+ * product decides the code, so both sides take it in float), rounded to
+ * nearest even with values past +-448 saturating to +-448; it reads back as
+ * value(code) * scale.
+ */
+double oracle_e4m3_to_double(uint8_t code) {
+    const int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);                          /* subnormal: m/8 * 2^(1-7) */
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+uint8_t oracle_e4m3_from_float(float y) {
+    if (isnan(y)) return 0x7F;
+    const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    double a = fabs((double)y);
+    if (a >= 448.0) return sign | 0x7E;                     /* saturate: S.1111.110 = 448 */
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);                                           /* a in [2^(e-1), 2^e) */
+    const int qexp = e - 4 > -9 ? e - 4 : -9;               /* 3 mantissa bits; subnormal quantum 2^-9 */
+    a = ldexp(rint(ldexp(a, -qexp)), qexp);                 /* nearest, ties to even */
+    if (a == 0.0) return sign;
+    int e2;
+    frexp(a, &e2);                                          /* a in [2^(e2-1), 2^e2) */
+    const int E = e2 - 1 + 7;
+    if (E >= 1) {
+        const int m = (int)(ldexp(a, -(e2 - 1)) * 8.0 - 8.0);
+        return sign | (uint8_t)(E << 3) | (uint8_t)m;
+    }
+    return sign | (uint8_t)(int)ldexp(a, 9);
+}
+
+/* codes of n bf16 values: e4m3(float(x) * inv_scale) */
+void oracle_quantize_e4m3(const uint16_t* x, int64_t n, float inv_scale, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t u = ((uint32_t)x[i]) << 16;
+        float f;
+        memcpy(&f, &u, sizeof f);
+        volatile float y = f * inv_scale;                   /* one float multiply, rounded */
+        out[i] = oracle_e4m3_from_float(y);
+    }
+}
+
+/* Append of e4m3 codes (already quantized rows) into u8 pools: same slots as oracle_append_kv. */
+void oracle_append_kv_e4m3(const uint8_t* k, const uint8_t* v, const int64_t* slot_mapping,
+                           int64_t num_tokens, int64_t num_kv_heads, int64_t head_dim,
+                           int64_t block_size, int64_t num_blocks, uint8_t* k_cache,
+                           uint8_t* v_cache) {
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0 || slot >= num_blocks * block_size) continue;
+        const int64_t block = slot / block_size, offset = slot % block_size;
+        for (int64_t h = 0; h < num_kv_heads; ++h)
+            for (int64_t d = 0; d < head_dim; ++d) {
+                const int64_t dst = pool_index(block, h, offset, d, num_kv_heads, block_size, head_dim);
+                const int64_t src = (t * num_kv_heads + h) * head_dim + d;
+                k_cache[dst] = k[src];
+                v_cache[dst] = v[src];
+            }
+    }
+}
+
+static void gather_sequence_e4m3(const uint8_t* cache, double cache_scale, const int32_t* table_row,
+                                 int64_t L, int64_t kv_head, int64_t num_kv_heads,
+                                 int64_t block_size, int64_t head_dim, double* rows) {
+    for (int64_t j = 0; j < L; ++j) {
+        const int64_t slot = oracle_slot(table_row, j, block_size);
+        const int64_t block = slot / block_size;
+        const int64_t offset = slot % block_size;
+        for (int64_t d = 0; d < head_dim; ++d)
+            rows[j * head_dim + d] = cache_scale * oracle_e4m3_to_double(
+                cache[pool_index(block, kv_head, offset, d, num_kv_heads, block_size, head_dim)]);
+    }
+}
+
+/* oracle_paged_decode over e4m3 pools: K and V values are code values times their scale. */
+int oracle_paged_decode_e4m3(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                             double k_scale, double v_scale, const int32_t* block_tables,
+                             const int32_t* context_lens, int64_t num_seqs, int64_t num_q_heads,
+                             int64_t num_kv_heads, int64_t head_dim, int64_t block_size,
+                             int64_t max_blocks_per_seq, double scale, double* out) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return -1;
+    const int64_t pairs = num_seqs * num_kv_heads;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_num_threads())
+    for (int64_t pair = 0; pair < pairs; ++pair) {
+        const int64_t b = pair / num_kv_heads, kvh = pair % num_kv_heads;
+        const int64_t L = context_lens[b];
+        const int32_t* table_row = block_tables + b * max_blocks_per_seq;
+        for (int64_t h = 0; h < num_q_heads; ++h) {
+            if (kv_head_of(h, num_q_heads, num_kv_heads) != kvh) continue;
+            double* o = out + (b * num_q_heads + h) * head_dim;
+            for (int64_t d = 0; d < head_dim; ++d) o[d] = 0.0;
+        }
+        if (L <= 0) continue;
+        double* K = (double*)malloc(sizeof(double) * (size_t)(L * head_dim));
+        double* V = (double*)malloc(sizeof(double) * (size_t)(L * head_dim));
+        double* s = (double*)malloc(sizeof(double) * (size_t)L);
+        double* qd = (double*)malloc(sizeof(double) * (size_t)head_dim);
+        if (!K || !V || !s || !qd) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            gather_sequence_e4m3(k_cache, k_scale, table_row, L, kvh, num_kv_heads, block_size, head_dim, K);
+            gather_sequence_e4m3(v_cache, v_scale, table_row, L, kvh, num_kv_heads, block_size, head_dim, V);
+            for (int64_t h = 0; h < num_q_heads; ++h) {
+                if (kv_head_of(h, num_q_heads, num_kv_heads) != kvh) continue;
+                for (int64_t d = 0; d < head_dim; ++d)
+                    qd[d] = oracle_bf16_to_double(q[(b * num_q_heads + h) * head_dim + d]);
+                attend(qd, K, V, 0, L, head_dim, scale, s, out + (b * num_q_heads + h) * head_dim, NULL);
+            }
+        }
+        free(K);
+        free(V);
+        free(s);
+        free(qd);
+    }
+    return failed ? -2 : 0;
+}

@@ -1,6 +1,6 @@
 """The oracle pins have teeth: each plausible mistake, planted in a copy of the
 oracle's C source and compiled on the CPU, must make at least one pin fail
-(pins of tests/test_oracle.py and tests/test_oracle_rope.py).
+(pins of tests/test_oracle.py, tests/test_oracle_rope.py and tests/test_oracle_fp8.py).
 
 The mutant library replaces the oracle's loaded library only for the duration
 of one test; the real oracle source is never modified.
@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 from tests import test_oracle as pins
+from tests import test_oracle_fp8 as fp8_pins
 from tests import test_oracle_rope as rope_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.c")
@@ -59,6 +60,19 @@ MUTANTS = {
     "rope_position": ("const double a = (double)pos[t] *", "const double a = (double)(pos[t] + 1) *"),
     # bf16 rounding truncates instead of rounding to nearest
     "round_truncates": ("v = ldexp(rint(ldexp(v, -qexp)), qexp);", "v = ldexp(trunc(ldexp(v, -qexp)), qexp);"),
+    # E4M3: exponent bias off by one
+    "e4m3_bias": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 6);"),
+    # E4M3: subnormal step 2^-10 instead of 2^-9
+    "e4m3_subnormal": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    # E4M3: no saturation below the next binade
+    "e4m3_saturation": ("if (a >= 448.0) return sign | 0x7E;", "if (a >= 480.0) return sign | 0x7E;"),
+    # E4M3: ties away from zero
+    "e4m3_ties_away": ("a = ldexp(rint(ldexp(a, -qexp)), qexp);", "a = ldexp(round(ldexp(a, -qexp)), qexp);"),
+    # E4M3 quantization divides by the inverse scale
+    "e4m3_quantize_scale": ("volatile float y = f * inv_scale;", "volatile float y = f / inv_scale;"),
+    # FP8 decode: V scale dropped; K and V scales swapped
+    "e4m3_decode_v_scale": ("gather_sequence_e4m3(v_cache, v_scale,", "gather_sequence_e4m3(v_cache, 1.0,"),
+    "e4m3_decode_scales_swapped": ("gather_sequence_e4m3(k_cache, k_scale,", "gather_sequence_e4m3(k_cache, v_scale,"),
     # bf16 rounding breaks ties away from zero instead of to even
     "round_ties_away": ("v = ldexp(rint(ldexp(v, -qexp)), qexp);", "v = ldexp(round(ldexp(v, -qexp)), qexp);"),
 }
@@ -67,7 +81,8 @@ MUTANTS = {
 def _pin_calls():
     """Every pin in test_oracle as a zero-argument callable (parametrised ones expanded)."""
     calls = []
-    members = inspect.getmembers(pins, inspect.isfunction) + inspect.getmembers(rope_pins, inspect.isfunction)
+    members = (inspect.getmembers(pins, inspect.isfunction) + inspect.getmembers(rope_pins, inspect.isfunction)
+               + inspect.getmembers(fp8_pins, inspect.isfunction))
     for name, fn in members:
         if not name.startswith("test_"):
             continue
@@ -108,7 +123,8 @@ def test_pins_catch_planted_mistake(mutant, monkeypatch):
         for sym in ("oracle_bf16_to_double", "oracle_kv_bytes", "oracle_slot", "oracle_slot_mapping",
                     "oracle_append_kv", "oracle_paged_decode", "oracle_paged_decode_partial",
                     "oracle_merge_partials", "oracle_set_num_threads", "oracle_num_threads",
-                    "oracle_rope", "oracle_round_bf16"):
+                    "oracle_rope", "oracle_round_bf16", "oracle_e4m3_to_double", "oracle_e4m3_from_float",
+                    "oracle_quantize_e4m3", "oracle_append_kv_e4m3", "oracle_paged_decode_e4m3"):
             f_real, f_mut = getattr(real, sym), getattr(mut, sym)
             f_mut.argtypes = f_real.argtypes
             f_mut.restype = f_real.restype
