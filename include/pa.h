@@ -103,6 +103,22 @@ PA_API int pa_append_kv(const pa_bf16* k, const pa_bf16* v, const int64_t* slot_
                  const pa_cache_desc* desc, void* stream);
 
 /*
+ * FP8 KV append.  The Tiny-vLLM summary page ("[Hacker News 요약] ... Tiny-vLLM
+ * ...", section "향후 전망") names FP8 among the data types to add, with no format
+ * or scale scheme.  This library uses the OCP E4M3 format (1 sign, 4 exponent
+ * bits of bias 7, 3 mantissa bits, no infinities, S.1111.111 = NaN, largest
+ * finite 448) with one scale per cache tensor: a bf16 value x is stored as the
+ * code of float(x) * float(1/scale) (one float multiply) rounded to nearest
+ * even, saturating at +-448, and reads back as code value * scale.  Halves the
+ * bytes every decode reads.
+ * Same slots and requirements as pa_append_kv; k_cache / v_cache are uint8
+ * pools [N][Hkv][Bs][D] (8-byte aligned); k_scale, v_scale > 0 and finite.
+ */
+PA_API int pa_append_kv_e4m3(const pa_bf16* k, const pa_bf16* v, const int64_t* slot_mapping,
+                             int32_t num_tokens, float k_scale, float v_scale, uint8_t* k_cache,
+                             uint8_t* v_cache, const pa_cache_desc* desc, void* stream);
+
+/*
  * RoPE (rotary position embedding) fused with the KV append.  The Tiny-vLLM
  * summary page ("[Hacker News 요약] ... Tiny-vLLM ...", section "핵심 LLM 연산의
  * CUDA 커널 구현") names RoPE among the per-layer kernels of the model it
@@ -138,6 +154,9 @@ PA_API int pa_rope_append_kv(const pa_bf16* q, pa_bf16* q_out, const pa_bf16* k,
 #define PA_FLAG_CHECK     1   /* synchronise after the launch and report device-side errors     */
 #define PA_FLAG_PDL       2   /* early start (programmatic dependent launch), see pa_decode     */
 
+#define PA_KV_BF16        0   /* caches hold bf16 values                                         */
+#define PA_KV_E4M3        1   /* caches hold E4M3 codes (uint8), see pa_append_kv_e4m3           */
+
 typedef struct pa_decode_options {
     int32_t split_tokens;  /* SIMT / TENSOR_SPLIT: 0 automatic, else tokens per KV split, a      */
                            /* positive multiple of 64                                           */
@@ -147,6 +166,11 @@ typedef struct pa_decode_options {
     float rope_theta;      /* pa_append_decode only: > 0 turns q and the new K rows by RoPE at   */
                            /* position L-1 with this frequency base (see pa_rope_append_kv);    */
                            /* 0 = no rotation.  pa_decode(_ex) rejects a nonzero value.         */
+    int32_t kv_dtype;      /* PA_KV_BF16 (default) or PA_KV_E4M3: the caches are uint8 E4M3     */
+                           /* pools of the same [N][Hkv][Bs][D] shape (the pointers are read as */
+                           /* bytes); the whole-group tensor kernel only, no RoPE               */
+    float k_scale;         /* PA_KV_E4M3: K value = code value * k_scale (> 0)                  */
+    float v_scale;         /* PA_KV_E4M3: V value = code value * v_scale (> 0)                  */
 } pa_decode_options;
 
 /*
@@ -184,6 +208,12 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * max_context_len or the table is clipped; both raise a bit in the
  * workspace's status word, which pa_decode_status reports (PA_FLAG_CHECK
  * does so before returning).
+ *
+ * options->kv_dtype == PA_KV_E4M3: the caches are E4M3 pools (see
+ * pa_append_kv_e4m3) and the attention reads K = code value * k_scale,
+ * V = code value * v_scale; only the whole-group tensor kernel serves it
+ * (PA_ERR_UNSUPPORTED otherwise, and with rope_theta).  pa_append_decode then
+ * quantizes the new rows with the same scales as it writes them.
  *
  * PA_FLAG_PDL (whole-group tensor kernel only; ignored by the others): the
  * decode kernel is launched as a programmatic dependent of the kernel before

@@ -32,6 +32,8 @@ STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ER
 PA_KERNEL_AUTO, PA_KERNEL_SIMT, PA_KERNEL_TENSOR, PA_KERNEL_TENSOR_SPLIT = 0, 1, 2, 3
 PA_FLAG_CHECK = 1
 PA_FLAG_PDL = 2
+PA_KV_BF16 = 0
+PA_KV_E4M3 = 1
 
 
 class PaError(RuntimeError):
@@ -54,7 +56,8 @@ class CacheDesc(ctypes.Structure):
 class DecodeOptions(ctypes.Structure):
     _fields_ = [("split_tokens", ctypes.c_int32), ("kernel", ctypes.c_int32),
                 ("flags", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
-                ("rope_theta", ctypes.c_float)]
+                ("rope_theta", ctypes.c_float), ("kv_dtype", ctypes.c_int32),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -123,6 +126,8 @@ lib.pa_bm_append_token_ids.restype = ctypes.c_int
 lib.pa_bm_num_cached_blocks.argtypes = [_vp]
 lib.pa_bm_num_cached_blocks.restype = _i32
 lib.pa_copy_blocks.argtypes = [_vp, _vp, _vp, _i32, _DESC, _vp]
+lib.pa_append_kv_e4m3.argtypes = [_vp, _vp, _vp, _i32, ctypes.c_float, ctypes.c_float, _vp, _vp, _DESC, _vp]
+lib.pa_append_kv_e4m3.restype = ctypes.c_int
 lib.pa_copy_blocks.restype = ctypes.c_int
 
 
@@ -159,13 +164,15 @@ def _dev(t, dtype_name: str, what: str):
     return t.data_ptr()
 
 
-def _cache(t, desc: "CacheDesc", what: str):
-    """Device pointer of a KV cache tensor that holds at least the pool desc describes."""
+def _cache(t, desc: "CacheDesc", what: str, options=None):
+    """Device pointer of a KV cache tensor (bf16, or uint8 E4M3 codes when the options say so)
+    that holds at least the pool desc describes."""
     if t is not None and not isinstance(t, int):
         need = int(desc.num_blocks) * desc.num_kv_heads * desc.block_size * desc.head_dim
         if t.numel() < need:
             raise ValueError("%s holds %d elements, the pool described needs %d" % (what, t.numel(), need))
-    return _dev(t, "bfloat16", what)
+    e4m3 = options is not None and options.kv_dtype == PA_KV_E4M3
+    return _dev(t, "uint8" if e4m3 else "bfloat16", what)
 
 
 def _stream(stream):
@@ -192,6 +199,18 @@ def pa_append_kv(k, v, slot_mapping, k_cache, v_cache, desc: CacheDesc, stream=N
                             _dev(slot_mapping, "int64", "slot_mapping"), n,
                             _cache(k_cache, desc, "k_cache"), _cache(v_cache, desc, "v_cache"),
                             ctypes.byref(desc), _stream(stream)), "pa_append_kv")
+
+
+def pa_append_kv_e4m3(k, v, slot_mapping, k_scale: float, v_scale: float, k_cache, v_cache,
+                      desc: CacheDesc, stream=None, num_tokens: int | None = None) -> None:
+    """Quantizing append into uint8 E4M3 pools."""
+    n = int(slot_mapping.shape[0]) if num_tokens is None else int(num_tokens)
+    e4m3 = DecodeOptions(kv_dtype=PA_KV_E4M3)
+    _check(lib.pa_append_kv_e4m3(_dev(k, "bfloat16", "k"), _dev(v, "bfloat16", "v"),
+                                 _dev(slot_mapping, "int64", "slot_mapping"), n, float(k_scale),
+                                 float(v_scale), _cache(k_cache, desc, "k_cache", e4m3),
+                                 _cache(v_cache, desc, "v_cache", e4m3), ctypes.byref(desc),
+                                 _stream(stream)), "pa_append_kv_e4m3")
 
 
 def pa_rope_append_kv(q, q_out, k, v, positions, slot_mapping, rope_theta: float, k_cache, v_cache,
@@ -234,8 +253,8 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: 
     n = int(context_lens.shape[0]) if num_seqs is None else int(num_seqs)
     wbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else int(workspace_bytes)
     ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
-    _check(lib.pa_decode_ex(_dev(q, "bfloat16", "q"), _cache(k_cache, desc, "k_cache"),
-                            _cache(v_cache, desc, "v_cache"),
+    _check(lib.pa_decode_ex(_dev(q, "bfloat16", "q"), _cache(k_cache, desc, "k_cache", options),
+                            _cache(v_cache, desc, "v_cache", options),
                             _dev(block_tables, "int32", "block_tables"),
                             _dev(context_lens, "int32", "context_lens"), n, int(max_context_len),
                             float(scale), _dev(out, "bfloat16", "out"), ws, wbytes,
@@ -253,8 +272,8 @@ def pa_append_decode(q, k, v, k_cache, v_cache, block_tables, context_lens, max_
     wbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else int(workspace_bytes)
     ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
     _check(lib.pa_append_decode(_dev(q, "bfloat16", "q"), _dev(k, "bfloat16", "k"),
-                                _dev(v, "bfloat16", "v"), _cache(k_cache, desc, "k_cache"),
-                                _cache(v_cache, desc, "v_cache"),
+                                _dev(v, "bfloat16", "v"), _cache(k_cache, desc, "k_cache", options),
+                                _cache(v_cache, desc, "v_cache", options),
                                 _dev(block_tables, "int32", "block_tables"),
                                 _dev(context_lens, "int32", "context_lens"), n,
                                 int(max_context_len), float(scale), _dev(out, "bfloat16", "out"), ws,
@@ -268,8 +287,8 @@ def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, max_conte
                       stream=None, num_seqs: int | None = None) -> None:
     """pa_decode with the library's fixed scratch array instead of a caller workspace."""
     n = int(context_lens.shape[0]) if num_seqs is None else int(num_seqs)
-    _check(lib.pa_decode_noalloc(_dev(q, "bfloat16", "q"), _cache(k_cache, desc, "k_cache"),
-                                 _cache(v_cache, desc, "v_cache"),
+    _check(lib.pa_decode_noalloc(_dev(q, "bfloat16", "q"), _cache(k_cache, desc, "k_cache", options),
+                                 _cache(v_cache, desc, "v_cache", options),
                                  _dev(block_tables, "int32", "block_tables"),
                                  _dev(context_lens, "int32", "context_lens"), n,
                                  int(max_context_len), float(scale), _dev(out, "bfloat16", "out"),

@@ -102,9 +102,12 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
     plan->split_tokens = 0;
     plan->max_splits = 1;
 
+    const bool fp8 = opt && opt->kv_dtype == PA_KV_E4M3;
+    if (fp8 && !(kernel == PA_KERNEL_TENSOR && stream_kernel_supports(d)))
+        return PA_ERR_UNSUPPORTED;   // E4M3 pools: the whole-group tensor kernel only
     if (kernel == PA_KERNEL_TENSOR && stream_kernel_supports(d)) {
         plan->kernel = DecodeKernel::kStream;
-        plan->grid = stream_kernel_grid(d, opt ? opt->max_ctas : 0);
+        plan->grid = stream_kernel_grid(d, opt ? opt->max_ctas : 0, fp8);
         if (plan->grid <= 0) return PA_ERR_CUDA;
         plan->off_lse = plan->off_desc + up((size_t)(d.num_kv_heads / 8) * num_seqs * 16);
         const size_t rows = (size_t)plan->grid * 2 * d.num_kv_heads * G;
@@ -206,6 +209,23 @@ extern "C" int pa_rope_append_kv(const pa_bf16* q, pa_bf16* q_out, const pa_bf16
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+extern "C" int pa_append_kv_e4m3(const pa_bf16* k, const pa_bf16* v, const int64_t* slot_mapping,
+                                 int32_t num_tokens, float k_scale, float v_scale, uint8_t* k_cache,
+                                 uint8_t* v_cache, const pa_cache_desc* desc, void* stream) {
+    int rc = check_desc(desc);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0 || desc->head_dim % 8 != 0 || !(k_scale > 0.f) || !(k_scale < INFINITY) ||
+        !(v_scale > 0.f) || !(v_scale < INFINITY))
+        return PA_ERR_INVALID;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(k_cache, 8) || !aligned(v_cache, 8) || !aligned(slot_mapping, 8))
+        return PA_ERR_INVALID;
+    const cudaError_t e = launch_append_e4m3(k, v, slot_mapping, num_tokens, 1.f / k_scale, 1.f / v_scale,
+                                             k_cache, v_cache, *desc, (cudaStream_t)stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 extern "C" int pa_copy_blocks(pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* copies, int32_t n,
                               const pa_cache_desc* desc, void* stream) {
     int rc = check_desc(desc);
@@ -263,9 +283,15 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     if (rc != PA_OK) return rc;
     if (options && (options->max_ctas < 0 || options->kernel < 0 || options->kernel > 3 ||
                     (options->flags & ~(PA_FLAG_CHECK | PA_FLAG_PDL)) != 0 ||
-                    !(options->rope_theta >= 0.f) || !(options->rope_theta < INFINITY)))
+                    !(options->rope_theta >= 0.f) || !(options->rope_theta < INFINITY) ||
+                    (options->kv_dtype != PA_KV_BF16 && options->kv_dtype != PA_KV_E4M3)))
         return PA_ERR_INVALID;
     const float rope_theta = options ? options->rope_theta : 0.f;
+    const bool fp8 = options && options->kv_dtype == PA_KV_E4M3;
+    if (fp8 && (!(options->k_scale > 0.f) || !(options->k_scale < INFINITY) ||
+                !(options->v_scale > 0.f) || !(options->v_scale < INFINITY)))
+        return PA_ERR_INVALID;
+    if (fp8 && rope_theta > 0.f) return PA_ERR_UNSUPPORTED;   // RoPE on E4M3 pools: not built
     if (rope_theta > 0.f && !k_new) return PA_ERR_INVALID;   // RoPE needs the new token (pa_append_decode)
     if (num_seqs == 0) return PA_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
@@ -305,7 +331,11 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     p.max_context_len = max_context_len;
     p.split_tokens = plan.split_tokens;
     p.max_splits = plan.max_splits;
-    p.scale_log2 = scale * 1.4426950408889634f;
+    p.scale_log2 = scale * (fp8 ? options->k_scale : 1.f) * 1.4426950408889634f;
+    p.kv_fp8 = fp8 ? 1 : 0;
+    p.k_inv_scale = fp8 ? 1.f / options->k_scale : 1.f;
+    p.v_inv_scale = fp8 ? 1.f / options->v_scale : 1.f;
+    p.out_scale = fp8 ? options->v_scale : 1.f;
     p.early = plan.kernel == DecodeKernel::kStream && options && (options->flags & PA_FLAG_PDL) ? 1 : 0;
     p.rope_theta = plan.kernel == DecodeKernel::kStream ? rope_theta : 0.f;
     cudaError_t e;

@@ -68,6 +68,42 @@ __global__ void __launch_bounds__(256) append_at_end_kernel(const DecodeParams p
     }
 }
 
+// E4M3 append: like append_kv_kernel, each 16-byte chunk of 8 bf16 becomes 8 codes
+// of value * inv_scale (a float product, then nearest even with saturation at +-448).
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint2 quantize8(uint4 x, float inv) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        c[i] = f32x2_to_e4m3x2(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv));
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__global__ void __launch_bounds__(256) append_e4m3_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, const int64_t* __restrict__ slots,
+    int64_t chunks, int32_t chunks_per_row, int32_t num_kv_heads, int32_t block_size,
+    int64_t num_slots, float k_inv, float v_inv, uint2* __restrict__ k_cache, uint2* __restrict__ v_cache) {
+    allow_dependents();
+    const int64_t per_token = (int64_t)num_kv_heads * chunks_per_row;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / per_token;
+        const int64_t within = i - t * per_token;
+        const int64_t slot = slots[t];
+        if (slot < 0 || slot >= num_slots) continue;
+        const int64_t blk = slot / block_size, off = slot - blk * block_size;
+        const int64_t h = within / chunks_per_row, c = within - h * chunks_per_row;
+        const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * chunks_per_row + c;
+        k_cache[dst] = quantize8(__ldg(k + i), k_inv);
+        v_cache[dst] = quantize8(__ldg(v + i), v_inv);
+    }
+}
+
 // Copy-on-write on the device: pair k copies block copies[2k] onto block copies[2k+1] in
 // both caches (a block is Hkv x Bs x D contiguous elements), 16 bytes per thread.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_cache,
@@ -88,6 +124,21 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_
 }
 
 }  // namespace
+
+cudaError_t launch_append_e4m3(const pa_bf16* k, const pa_bf16* v, const int64_t* slots, int32_t T,
+                               float k_inv_scale, float v_inv_scale, uint8_t* k_cache,
+                               uint8_t* v_cache, const pa_cache_desc& d, cudaStream_t stream) {
+    const int32_t chunks_per_row = d.head_dim / 8;
+    const int64_t chunks = (int64_t)T * d.num_kv_heads * chunks_per_row;
+    if (chunks == 0) return cudaSuccess;
+    int64_t blocks = (chunks + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    append_e4m3_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), slots, chunks,
+        chunks_per_row, d.num_kv_heads, d.block_size, (int64_t)d.num_blocks * d.block_size,
+        k_inv_scale, v_inv_scale, reinterpret_cast<uint2*>(k_cache), reinterpret_cast<uint2*>(v_cache));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_copy_blocks(pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* copies, int32_t n,
                                const pa_cache_desc& d, cudaStream_t stream) {

@@ -44,19 +44,25 @@ constexpr int kSlab = 16;                    // tokens per stage
 constexpr int kRowBytes = 128;               // 64 bf16 of head dim, one swizzled row
 constexpr int kQSlots = 2;
 
-template <int D, int NT>
+template <int D, int NT, bool F8 = false>
 struct SCfg {
     static constexpr int kHalves = D / 64;
     static constexpr int kHalfBytes = kGroup * kSlab * kRowBytes;   // 16 KB
-    static constexpr int kTileBytes = kHalves * kHalfBytes;         // K (or V) of a stage
-    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kTileBytes = kHalves * kHalfBytes;         // bf16 K (or V) of a stage
+    // as loaded: bf16 in 128-byte swizzled rows (one box per 64 dims), or E4M3 in plain D-byte rows
+    static constexpr int kLoadBoxes = F8 ? 1 : kHalves;
+    static constexpr int kLoadRowBytes = F8 ? D : kRowBytes;
+    static constexpr int kTileBytesIn = F8 ? kGroup * kSlab * D : kTileBytes;
+    static constexpr int kStageBytes = 2 * kTileBytesIn;
+    // E4M3: each warp widens its rows of a stage into a bf16 copy laid out as a bf16 stage
+    static constexpr int kStagingBytes = F8 ? 2 * kTileBytes : 0;
     static constexpr int kStages = (D == 128 && NT == 2) ? 2 : 3;
     static constexpr int kKSteps = D / 16;
     static constexpr int kMTiles = D / 16;
     static constexpr int kMinBlocks = (D == 64 && NT == 1) ? 2 : 1;
     // dynamic shared memory for query group size g
     static constexpr size_t smem_bytes(int g) {
-        return (size_t)kStages * kStageBytes + (size_t)kQSlots * kGroup * g * D * 2 + 1024;
+        return (size_t)kStages * kStageBytes + kStagingBytes + (size_t)kQSlots * kGroup * g * D * 2 + 1024;
     }
 };
 
@@ -92,11 +98,39 @@ __device__ __forceinline__ int32_t cta_of(int64_t s, int64_t S, int64_t G) {
     return (int32_t)(((s + 1) * G - 1) / S);
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
+// Eight E4M3 codes (bytes 0..7) -> eight bf16 (exact: every E4M3 value is a bf16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes) {
+    uint32_t h2;
+    asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e4m3x2 %0, c; }" : "=r"(h2) : "r"(codes & 0xFFFFu));
+    float lo, hi;
+    asm("{ .reg .f16 l, h; mov.b32 {l, h}, %2; cvt.f32.f16 %0, l; cvt.f32.f16 %1, h; }"
+        : "=f"(lo), "=f"(hi) : "r"(h2));
+    return pack_bf16x2(lo, hi);
+}
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 q) {
+    return make_uint4(e4m3x2_to_bf16x2(q.x), e4m3x2_to_bf16x2(q.x >> 16), e4m3x2_to_bf16x2(q.y),
+                      e4m3x2_to_bf16x2(q.y >> 16));
+}
+// Eight bf16 -> eight E4M3 codes of value * inv_scale (float product, nearest even, saturating).
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 x, float inv_scale) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        c[i] = f32x2_to_e4m3x2(__fmul_rn(bf16_lo(w[i]), inv_scale), __fmul_rn(bf16_hi(w[i]), inv_scale));
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+template <int D, int NT, bool F8>
+__global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     decode_stream_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap) {
-    using C = SCfg<D, NT>;
+    using C = SCfg<D, NT, F8>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Hdr s_hdr[C::kStages];
     __shared__ __align__(8) uint64_t full_bar[C::kStages];
@@ -110,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
     const int32_t Hkv = p.num_kv_heads;
     const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
-    const uint32_t q_base = smem_base + C::kStages * C::kStageBytes;   // q ring after the stages
+    const uint32_t staging = smem_base + C::kStages * C::kStageBytes;  // E4M3: widened stage
+    const uint32_t q_base = staging + C::kStagingBytes;                 // q ring after them
     const uint32_t q_slot_bytes = (uint32_t)(kGroup * G * D * 2);
     allow_dependents();
     if (threadIdx.x == kGroup * 32) {
@@ -217,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                         const int32_t blk = __shfl_sync(0xffffffffu, win_entry, lbk - win_base);
                         if (lane == 0 && blk >= 0 && blk < p.num_blocks) {
 #pragma unroll
-                            for (int h = 0; h < C::kHalves; ++h) {
+                            for (int h = 0; h < C::kLoadBoxes; ++h) {
                                 tma_prefetch_3d(&kmap, h * 64, tok - lbk * Bs, blk * Hkv + gi * kGroup);
                                 tma_prefetch_3d(&vmap, h * 64, tok - lbk * Bs, blk * Hkv + gi * kGroup);
                             }
@@ -280,7 +315,20 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                         uint16_t* vc = const_cast<uint16_t*>(p.v_cache);
                         const size_t row0 = ((size_t)blk * Hkv + gi * kGroup) * Bs + (pos - lbn * Bs);
                         const size_t src0 = ((size_t)b * Hkv + gi * kGroup) * D;
-                        if (p.rope_theta > 0.f) {
+                        if constexpr (F8) {
+                            // E4M3 pools: the new rows quantized with the caches' scales
+                            uint8_t* kq = reinterpret_cast<uint8_t*>(kc);
+                            uint8_t* vq = reinterpret_cast<uint8_t*>(vc);
+                            for (int i = lane; i < kGroup * kChunks; i += 32) {
+                                const int hh = i / kChunks, cc = i - hh * kChunks;
+                                const size_t dst = (row0 + (size_t)hh * Bs) * D + cc * 8;
+                                const size_t src = src0 + (size_t)hh * D + cc * 8;
+                                *reinterpret_cast<uint2*>(kq + dst) = bf16x8_to_e4m3x8(
+                                    __ldg(reinterpret_cast<const uint4*>(p.k_new + src)), p.k_inv_scale);
+                                *reinterpret_cast<uint2*>(vq + dst) = bf16x8_to_e4m3x8(
+                                    __ldg(reinterpret_cast<const uint4*>(p.v_new + src)), p.v_inv_scale);
+                            }
+                        } else if (p.rope_theta > 0.f) {
                             constexpr int kHalfChunks = D / 16;
                             for (int i = lane; i < kGroup * kHalfChunks; i += 32) {
                                 const int hh = i / kHalfChunks, cc = i - hh * kHalfChunks;
@@ -296,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                                 *reinterpret_cast<uint4*>(dst + D / 2) = x2;
                             }
                         }
-                        for (int i = lane; i < kGroup * kChunks; i += 32) {
+                        for (int i = lane; i < kGroup * kChunks && !F8; i += 32) {
                             const int hh = i / kChunks, cc = i - hh * kChunks;
                             const size_t dst = (row0 + (size_t)hh * Bs) * D + cc * 8;
                             const size_t src = src0 + (size_t)hh * D + cc * 8;
@@ -312,9 +360,9 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                 if (valid > 0) {
                     const int32_t nbox = (valid + tb - 1) / tb;
                     if (lane == 0)
-                        mbar_arrive_expect_tx(fbar, (uint32_t)(nbox * kGroup * tb * kRowBytes * C::kHalves * 2));
+                        mbar_arrive_expect_tx(fbar, (uint32_t)(nbox * kGroup * tb * C::kLoadRowBytes * C::kLoadBoxes * 2));
                     const uint32_t k_tile = smem_base + st * C::kStageBytes;
-                    const uint32_t v_tile = k_tile + C::kTileBytes;
+                    const uint32_t v_tile = k_tile + C::kTileBytesIn;
                     for (int32_t x = 0; x < nbox; ++x) {
                         const int32_t tok = t0 + x * tb;
                         const int32_t lbk = tok / Bs;
@@ -333,9 +381,9 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                                 z = blk * Hkv + gi * kGroup;
                             }
                             const int32_t y = tok - lbk * Bs;
-                            const uint32_t off = (uint32_t)(x * kGroup * tb * kRowBytes);
+                            const uint32_t off = (uint32_t)(x * kGroup * tb * C::kLoadRowBytes);
 #pragma unroll
-                            for (int h = 0; h < C::kHalves; ++h) {
+                            for (int h = 0; h < C::kLoadBoxes; ++h) {
                                 tma_load_3d_hint(k_tile + h * C::kHalfBytes + off, &kmap, h * 64, y, z, fbar, kv_policy);
                                 tma_load_3d_hint(v_tile + h * C::kHalfBytes + off, &vmap, h * 64, y, z, fbar, kv_policy);
                             }
@@ -434,9 +482,29 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                 ++qk;
             }
             const int valid = hd.valid;
-            const uint32_t k_tile = smem_base + st * C::kStageBytes;
-            const uint32_t v_tile = k_tile + C::kTileBytes;
-            if (valid < kSlab) {
+            uint32_t k_tile = smem_base + st * C::kStageBytes;
+            uint32_t v_tile = k_tile + C::kTileBytes;
+            if constexpr (F8) {
+                // widen this warp's 16 token rows of the E4M3 stage into the bf16 staging tile
+                // (rows past the sequence become zeros), then hand the stage back at once
+                const uint32_t f8k = k_tile, f8v = k_tile + C::kTileBytesIn;
+                k_tile = staging;
+                v_tile = staging + C::kTileBytes;
+                constexpr int kCh = D / 8;
+                for (int i = lane; i < kSlab * kCh; i += 32) {
+                    const int t = i / kCh, c = i - t * kCh;
+                    const int row = stage_row(warp, t, tb);
+                    uint4 kb = make_uint4(0, 0, 0, 0), vb = kb;
+                    if (t < valid) {
+                        kb = e4m3x8_to_bf16x8(*reinterpret_cast<const uint2*>(smem_gen + (f8k - smem_base) + row * D + c * 8));
+                        vb = e4m3x8_to_bf16x8(*reinterpret_cast<const uint2*>(smem_gen + (f8v - smem_base) + row * D + c * 8));
+                    }
+                    *reinterpret_cast<uint4*>(smem_gen + (swz(k_tile + (c >> 3) * C::kHalfBytes, row, c & 7) - smem_base)) = kb;
+                    *reinterpret_cast<uint4*>(smem_gen + (swz(v_tile + (c >> 3) * C::kHalfBytes, row, c & 7) - smem_base)) = vb;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+            } else if (valid < kSlab) {
                 // tokens past the sequence: zero V so that 0-probability rows add nothing
                 for (int i = lane; i < (kSlab - valid) * 8 * C::kHalves; i += 32) {
                     const int t = valid + i / (8 * C::kHalves);
@@ -506,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                 for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o_acc[nt][mt], a, pb[nt][0], pb[nt][1]);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+            if (!F8 && lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
             if (!(hd.flags & kLast)) continue;
 
             // ======== end of this warp's segment: store, or publish a partial ========
@@ -526,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                     for (int jj = 0; jj < 2; ++jj) {
                         const int h = nt * 8 + 2 * c + jj;
                         if (h >= G) continue;
-                        const float inv = 1.f / l_run[nt][jj];
+                        const float inv = p.out_scale / l_run[nt][jj];
 #pragma unroll
                         for (int mt = 0; mt < C::kMTiles; ++mt) {
                             out[(size_t)h * D + mt * 16 + r] = f32_to_bf16_rn(o_acc[nt][mt][jj] * inv);
@@ -542,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT>::kMinBlocks)
                 for (int jj = 0; jj < 2; ++jj) {
                     const int h = nt * 8 + 2 * c + jj;
                     if (h >= G) continue;
-                    const float inv = 1.f / l_run[nt][jj];
+                    const float inv = p.out_scale / l_run[nt][jj];
                     float* po = p.part_o + (prow + h) * D;
 #pragma unroll
                     for (int mt = 0; mt < C::kMTiles; ++mt) {
@@ -578,81 +646,100 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D view [blocks * Hkv][block_size][head_dim]; box = 64 dims x tb tokens x 8 kv heads.
+// bf16 pools: boxes of 64 dims in 128-byte swizzled rows; E4M3 pools: whole D-byte rows, no swizzle.
 bool make_map(CUtensorMap* map, const void* base, const DecodeParams& p) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const cuuint64_t esize = p.kv_fp8 ? 1 : 2;
     const cuuint64_t dims[3] = {(cuuint64_t)p.head_dim, (cuuint64_t)p.block_size,
                                 (cuuint64_t)p.num_blocks * p.num_kv_heads};
-    const cuuint64_t strides[2] = {(cuuint64_t)p.head_dim * 2,
-                                   (cuuint64_t)p.block_size * p.head_dim * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)(p.block_size < kSlab ? p.block_size : kSlab),
+    const cuuint64_t strides[2] = {(cuuint64_t)p.head_dim * esize,
+                                   (cuuint64_t)p.block_size * p.head_dim * esize};
+    const cuuint32_t box[3] = {p.kv_fp8 ? (cuuint32_t)p.head_dim : 64u,
+                               (cuuint32_t)(p.block_size < kSlab ? p.block_size : kSlab),
                                (cuuint32_t)kGroup};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    return fn(map, p.kv_fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              p.kv_fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 auto kernel_ptr() {
-    return decode_stream_kernel<D, NT>;
+    return decode_stream_kernel<D, NT, F8>;
 }
 
 // The dynamic shared-memory opt-in is a per-kernel attribute: set it once per
 // device to the instantiation's largest need (its largest query group), then
 // size every launch by its own group.
-template <int D, int NT>
+template <int D, int NT, bool F8>
 bool ensure_smem_attr() {
     static std::atomic<uint64_t> done{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     const uint64_t bit = 1ull << dev;
     if (done.load(std::memory_order_acquire) & bit) return true;
-    if (cudaFuncSetAttribute(kernel_ptr<D, NT>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SCfg<D, NT>::smem_bytes(NT * 8)) != cudaSuccess)
+    if (cudaFuncSetAttribute(kernel_ptr<D, NT, F8>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SCfg<D, NT, F8>::smem_bytes(NT * 8)) != cudaSuccess)
         return false;
     done.fetch_or(bit, std::memory_order_acq_rel);
     return true;
 }
 
 // Resident CTAs per SM for this instantiation and query group size (cached per device).
-template <int D, int NT>
+template <int D, int NT, bool F8>
 int occupancy(int g) {
     static std::atomic<int> cache[64][17];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || g < 1 || g > NT * 8) return 0;
     int occ = cache[dev][g].load(std::memory_order_acquire);
     if (occ > 0) return occ;
-    if (!ensure_smem_attr<D, NT>()) return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel_ptr<D, NT>(), kThreads,
-                                                      SCfg<D, NT>::smem_bytes(g)) != cudaSuccess)
+    if (!ensure_smem_attr<D, NT, F8>()) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel_ptr<D, NT, F8>(), kThreads,
+                                                      SCfg<D, NT, F8>::smem_bytes(g)) != cudaSuccess)
         return 0;
     cache[dev][g].store(occ, std::memory_order_release);
     return occ;
 }
 
+template <bool F8>
 int occupancy_for(int D, int g) {
     const bool two = g > 8;
-    if (D == 64) return two ? occupancy<64, 2>(g) : occupancy<64, 1>(g);
-    if (D == 128) return two ? occupancy<128, 2>(g) : occupancy<128, 1>(g);
+    if (D == 64) return two ? occupancy<64, 2, F8>(g) : occupancy<64, 1, F8>(g);
+    if (D == 128) return two ? occupancy<128, 2, F8>(g) : occupancy<128, 1, F8>(g);
     return 0;
 }
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 cudaError_t launch_s(const DecodeParams& p, int grid, const CUtensorMap& km, const CUtensorMap& vm,
                      bool pdl, cudaStream_t stream) {
-    if (!ensure_smem_attr<D, NT>() || occupancy<D, NT>(p.group) <= 0) return cudaErrorInvalidConfiguration;
+    if (!ensure_smem_attr<D, NT, F8>() || occupancy<D, NT, F8>(p.group) <= 0)
+        return cudaErrorInvalidConfiguration;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = SCfg<D, NT>::smem_bytes(p.group);
+    cfg.dynamicSmemBytes = SCfg<D, NT, F8>::smem_bytes(p.group);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<D, NT>, p, km, vm);
+    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<D, NT, F8>, p, km, vm);
+}
+
+template <bool F8>
+cudaError_t launch_by_shape(const DecodeParams& p, int grid, const CUtensorMap& km, const CUtensorMap& vm,
+                            bool pdl, cudaStream_t stream) {
+    const bool two = p.group > 8;
+    if (p.head_dim == 64)
+        return two ? launch_s<64, 2, F8>(p, grid, km, vm, pdl, stream)
+                   : launch_s<64, 1, F8>(p, grid, km, vm, pdl, stream);
+    if (p.head_dim == 128)
+        return two ? launch_s<128, 2, F8>(p, grid, km, vm, pdl, stream)
+                   : launch_s<128, 1, F8>(p, grid, km, vm, pdl, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -663,10 +750,11 @@ bool stream_kernel_supports(const pa_cache_desc& d) {
            g <= 16 && encode_fn() != nullptr;
 }
 
-int stream_kernel_grid(const pa_cache_desc& d, int max_ctas) {
+int stream_kernel_grid(const pa_cache_desc& d, int max_ctas, bool fp8) {
     int sms = 0;
     if (num_sms_current_device(&sms) != PA_OK) return 0;
-    const int occ = occupancy_for(d.head_dim, d.num_q_heads / d.num_kv_heads);
+    const int g = d.num_q_heads / d.num_kv_heads;
+    const int occ = fp8 ? occupancy_for<true>(d.head_dim, g) : occupancy_for<false>(d.head_dim, g);
     if (occ <= 0) return 0;
     int grid = sms * occ;
     if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
@@ -676,14 +764,8 @@ int stream_kernel_grid(const pa_cache_desc& d, int max_ctas) {
 cudaError_t launch_decode_stream(const DecodeParams& p, int grid, bool pdl, cudaStream_t stream) {
     CUtensorMap km, vm;
     if (!make_map(&km, p.k_cache, p) || !make_map(&vm, p.v_cache, p)) return cudaErrorInvalidValue;
-    const bool two = p.group > 8;
-    if (p.head_dim == 64)
-        return two ? launch_s<64, 2>(p, grid, km, vm, pdl, stream)
-                   : launch_s<64, 1>(p, grid, km, vm, pdl, stream);
-    if (p.head_dim == 128)
-        return two ? launch_s<128, 2>(p, grid, km, vm, pdl, stream)
-                   : launch_s<128, 1>(p, grid, km, vm, pdl, stream);
-    return cudaErrorInvalidValue;
+    return p.kv_fp8 ? launch_by_shape<true>(p, grid, km, vm, pdl, stream)
+                    : launch_by_shape<false>(p, grid, km, vm, pdl, stream);
 }
 
 }  // namespace pa

@@ -46,6 +46,9 @@ struct DecodeParams {
     float scale_log2;              // scale * log2(e): scores are kept in the log2 domain
     int32_t early;                 // launched early (PA_FLAG_PDL): prefetch before the wait
     float rope_theta;              // > 0: rotate q and the new K rows at position L-1 (fused append)
+    int32_t kv_fp8;                // caches hold E4M3 codes (uint8), values = code * scale
+    float k_inv_scale, v_inv_scale;  // E4M3: float(1/scale) applied when quantizing new rows
+    float out_scale;               // multiplies the normalised output (E4M3: the V scale; else 1)
 };
 
 // Which decode kernel a plan runs.
@@ -73,6 +76,10 @@ cudaError_t launch_append(const pa_bf16* k, const pa_bf16* v, const int64_t* slo
                           pa_bf16* k_cache, pa_bf16* v_cache, const pa_cache_desc& d,
                           cudaStream_t stream);
 cudaError_t launch_append_at_end(const DecodeParams& p, cudaStream_t stream);
+// E4M3 append: codes of value * inv_scale (float product, nearest even, saturating).
+cudaError_t launch_append_e4m3(const pa_bf16* k, const pa_bf16* v, const int64_t* slots, int32_t T,
+                               float k_inv_scale, float v_inv_scale, uint8_t* k_cache,
+                               uint8_t* v_cache, const pa_cache_desc& d, cudaStream_t stream);
 cudaError_t launch_copy_blocks(pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* copies, int32_t n,
                                const pa_cache_desc& d, cudaStream_t stream);
 // RoPE + append through the slot mapping (pa_rope_append_kv).
@@ -90,6 +97,6 @@ bool tensor_kernel_supports(const pa_cache_desc& d);
 cudaError_t launch_decode_stream(const DecodeParams& p, int grid, bool pdl, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeParams& p, bool stream_layout, bool pdl, cudaStream_t stream);
 bool stream_kernel_supports(const pa_cache_desc& d);
-int stream_kernel_grid(const pa_cache_desc& d, int max_ctas);
+int stream_kernel_grid(const pa_cache_desc& d, int max_ctas, bool fp8);
 
 }  // namespace pa

@@ -111,6 +111,24 @@ def test_binding_refuses_caches_smaller_than_the_pool():
         pa.pa_append_kv(small, small, torch.zeros(1, dtype=torch.int64), small, small, d)
 
 
+def test_e4m3_arguments_rejected_without_a_gpu():
+    lib = binding.lib
+    fake = ctypes.c_void_p(0x10000)
+    d = _desc()
+    for ks, vs in ((0.0, 1.0), (1.0, -1.0), (float("nan"), 1.0), (1.0, float("inf"))):
+        assert lib.pa_append_kv_e4m3(fake, fake, fake, 1, ctypes.c_float(ks), ctypes.c_float(vs), fake, fake,
+                                     ctypes.byref(d), None) == -1, (ks, vs)
+    assert lib.pa_append_kv_e4m3(fake, fake, fake, 0, ctypes.c_float(1.0), ctypes.c_float(1.0), fake, fake,
+                                 ctypes.byref(d), None) == 0
+    call = lambda o: lib.pa_decode_ex(fake, fake, fake, fake, fake, 1, 16, ctypes.c_float(0.1), fake, fake,
+                                      1 << 20, ctypes.byref(d), ctypes.byref(o), None)
+    assert call(pa.DecodeOptions(kv_dtype=2)) == -1                            # unknown dtype
+    assert call(pa.DecodeOptions(kv_dtype=pa.PA_KV_E4M3, k_scale=0.0, v_scale=1.0)) == -1
+    # E4M3 pools are served by the whole-group tensor kernel only
+    assert call(pa.DecodeOptions(kv_dtype=pa.PA_KV_E4M3, k_scale=1.0, v_scale=1.0,
+                                 kernel=pa.PA_KERNEL_SIMT)) == -2
+
+
 def test_slot_mapping_entry_matches_oracle():
     import oracle
     rng = np.random.default_rng(0)

@@ -1,0 +1,151 @@
+"""FP8 (E4M3) KV cache through the C ABI against the fp64 oracle (needs a B200).
+
+Quantized appends must produce the oracle's codes bit for bit (the code is an
+integer decided by one float product and a nearest-even rounding, which both
+sides take in float), and touch no other byte.  Decodes over E4M3 pools are
+compared with the oracle's fp64 attention over the same codes (values = code
+value * scale) within 1e-2 + 1e-2 * |oracle|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+import pagedattention_kv_cache_pa_b200 as pa
+
+pytestmark = pytest.mark.gpu
+
+SCALES = [(5.0 / 448, 5.0 / 448), (1.0 / 64, 0.37), (0.37, 1.0 / 64)]
+
+
+@pytest.fixture(scope="module")
+def h():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tests import gpu_harness
+    return gpu_harness
+
+
+def _u8(a, h):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(h.DEV)
+
+
+def _pools(b, ks, vs):
+    return oracle.quantize_e4m3(b.k_cache, ks), oracle.quantize_e4m3(b.v_cache, vs)
+
+
+@pytest.mark.parametrize("ks,vs", SCALES)
+@pytest.mark.parametrize("cfg", ["c2", "c4"])
+def test_append_e4m3_codes_bit_exact(h, cfg, ks, vs):
+    b = wl.CONFIGS[cfg]()
+    (slots, _, _), (o_slots, _, _) = h.host_step(b)
+    kq, vq = _pools(b, ks, vs)
+    kc, vc = _u8(kq, h), _u8(vq, h)
+    pa.pa_append_kv_e4m3(h.to_dev(b.k_new), h.to_dev(b.v_new), torch.from_numpy(slots).to(h.DEV), ks, vs,
+                         kc, vc, h.desc_of(b))
+    torch.cuda.synchronize()
+    want_k, want_v = oracle.append_kv_e4m3(oracle.quantize_e4m3(b.k_new, ks), oracle.quantize_e4m3(b.v_new, vs),
+                                           o_slots, kq, vq)
+    np.testing.assert_array_equal(kc.cpu().numpy(), want_k)
+    np.testing.assert_array_equal(vc.cpu().numpy(), want_v)
+
+
+def test_append_e4m3_extremes(h):
+    # saturation, subnormals, signed zero, ties: rows built from chosen bf16 values
+    b = wl.small_batch(81, [5], num_q_heads=8, num_kv_heads=8, head_dim=64, block_size=16)
+    vals = np.array([0.0, -0.0, 1.0, -1.0, 448.0, 449.0, 1e6, -1e6, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -10,
+                     1.0625, 1.1875, 0.3, -7.5, 300.0], dtype=np.float32)
+    bits = (np.resize(vals, b.k_new.size).view(np.uint32) >> 16).astype(np.uint16).reshape(b.k_new.shape)
+    kq, vq = np.zeros_like(b.k_cache, dtype=np.uint8), np.zeros_like(b.v_cache, dtype=np.uint8)
+    kc, vc = _u8(kq, h), _u8(vq, h)
+    slots = np.array([7], dtype=np.int64)
+    pa.pa_append_kv_e4m3(h.to_dev(bits), h.to_dev(bits), torch.from_numpy(slots).to(h.DEV), 1.0, 0.5,
+                         kc, vc, h.desc_of(b))
+    torch.cuda.synchronize()
+    want_k, want_v = oracle.append_kv_e4m3(oracle.quantize_e4m3(bits, 1.0), oracle.quantize_e4m3(bits, 0.5),
+                                           slots, kq, vq)
+    np.testing.assert_array_equal(kc.cpu().numpy(), want_k)
+    np.testing.assert_array_equal(vc.cpu().numpy(), want_v)
+
+
+def _decode_case(h, b, ks, vs, *, max_ctas=0, pdl=False, fused=False):
+    (slots, tables, lens), (o_slots, o_tables, o_lens) = h.host_step(b)
+    kq, vq = _pools(b, ks, vs)
+    desc = h.desc_of(b)
+    kc, vc = _u8(kq, h), _u8(vq, h)
+    q = h.to_dev(b.q)
+    out = torch.empty_like(q)
+    max_len = int(lens.max())
+    opts = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR, kv_dtype=pa.PA_KV_E4M3, k_scale=ks, v_scale=vs,
+                            max_ctas=max_ctas, flags=pa.PA_FLAG_CHECK | (pa.PA_FLAG_PDL if pdl else 0))
+    ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, max_len, desc, opts), dtype=torch.uint8,
+                     device=h.DEV)
+    tb, lb = torch.from_numpy(tables).to(h.DEV), torch.from_numpy(lens).to(h.DEV)
+    if fused:
+        pa.pa_append_decode(q, h.to_dev(b.k_new), h.to_dev(b.v_new), kc, vc, tb, lb, max_len, b.scale, out,
+                            ws, desc, opts)
+    else:
+        pa.pa_append_kv_e4m3(h.to_dev(b.k_new), h.to_dev(b.v_new), torch.from_numpy(slots).to(h.DEV), ks, vs,
+                             kc, vc, desc)
+        pa.pa_decode(q, kc, vc, tb, lb, max_len, b.scale, out, ws, desc, opts)
+    torch.cuda.synchronize()
+    rk, rv = oracle.append_kv_e4m3(oracle.quantize_e4m3(b.k_new, ks), oracle.quantize_e4m3(b.v_new, vs),
+                                   o_slots, kq, vq)
+    np.testing.assert_array_equal(kc.cpu().numpy(), rk)
+    np.testing.assert_array_equal(vc.cpu().numpy(), rv)
+    ref = oracle.paged_decode_e4m3(b.q, rk, rv, ks, vs, o_tables, o_lens, b.scale)
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    ok, ex = oracle.within_tolerance(got, ref)
+    assert ok, "decode outside tolerance by %g" % ex
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+@pytest.mark.parametrize("cfg", ["c2", "c3", "c4"])
+def test_decode_e4m3(h, cfg, fused):
+    ks, vs = SCALES[0]
+    _decode_case(h, wl.CONFIGS[cfg](), ks, vs, fused=fused)
+
+
+@pytest.mark.parametrize("ks,vs", SCALES[1:])
+@pytest.mark.parametrize("ctas,pdl", [(1, False), (5, True), (64, False)])
+def test_decode_e4m3_partitions_and_scales(h, ks, vs, ctas, pdl):
+    _decode_case(h, wl.config2(), ks, vs, max_ctas=ctas, pdl=pdl, fused=True)
+
+
+FP8_SHAPES = [(8, 8, 64, 8), (16, 8, 128, 16), (64, 8, 128, 16), (128, 8, 64, 16), (32, 16, 64, 32),
+              (24, 8, 64, 256), (96, 8, 128, 32)]
+
+
+@pytest.mark.parametrize("shape", FP8_SHAPES, ids=lambda s: "Hq%d-Hkv%d-D%d-Bs%d" % s)
+def test_decode_e4m3_shapes(h, shape):
+    Hq, Hkv, D, Bs = shape
+    lens = sorted({0, 1, Bs - 1, Bs, 62, 63, 64, 65, 127, 128, 129, 300, 777})
+    b = wl.small_batch(5000 + Bs + D + Hq, lens, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, block_size=Bs)
+    for ctas, fused in ((0, False), (3, True), (17, False)):
+        _decode_case(h, b, 5.0 / 448, 0.02, max_ctas=ctas, fused=fused)
+
+
+def test_e4m3_unsupported_combinations(h):
+    b = wl.config1()                                     # Hkv = 1: no whole-group kernel
+    desc = h.desc_of(b)
+    q = h.to_dev(b.q)
+    kc = torch.zeros(b.k_cache.size, dtype=torch.uint8, device=h.DEV)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device=h.DEV)
+    opts = pa.DecodeOptions(kv_dtype=pa.PA_KV_E4M3, k_scale=1.0, v_scale=1.0)
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode(q, kc, kc, torch.from_numpy(b.block_tables).to(h.DEV),
+                     torch.from_numpy(b.context_lens).to(h.DEV), 40, b.scale, torch.empty_like(q), ws, desc,
+                     opts)
+    assert e.value.status == -2
+    b2 = wl.config2()
+    desc2 = h.desc_of(b2)
+    kc2 = torch.zeros(b2.k_cache.size, dtype=torch.uint8, device=h.DEV)
+    opts = pa.DecodeOptions(kv_dtype=pa.PA_KV_E4M3, k_scale=1.0, v_scale=1.0, rope_theta=10000.0)
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_append_decode(h.to_dev(b2.q), h.to_dev(b2.k_new), h.to_dev(b2.v_new), kc2, kc2,
+                            torch.from_numpy(b2.block_tables).to(h.DEV),
+                            torch.from_numpy(b2.context_lens).to(h.DEV), 2048, b2.scale,
+                            torch.empty_like(h.to_dev(b2.q)), ws, desc2, opts)
+    assert e.value.status == -2

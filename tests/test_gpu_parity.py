@@ -304,8 +304,9 @@ def test_argument_errors(h):
     assert e.value.status == -4
     bad = pa.CacheDesc.make(num_blocks=8, block_size=16, num_kv_heads=1, num_q_heads=2, head_dim=96,
                             max_blocks_per_seq=3)
-    with pytest.raises(pa.PaError) as e:   # head_dim 96 not built
-        pa.pa_decode(q, kc, kc, tables, lens, 37, b.scale, out, ws, bad)
+    with pytest.raises(pa.PaError) as e:   # head_dim 96 not built (raw pointers: the C check, not
+        # the binding's pool-size check, answers; the shape is refused before any access)
+        pa.pa_decode(q, kc.data_ptr(), kc.data_ptr(), tables, lens, 37, b.scale, out, ws, bad)
     assert e.value.status == -2
     with pytest.raises(pa.PaError) as e:   # misaligned output pointer
         pa.pa_decode(q, kc, kc, tables, lens, 37, b.scale, out.data_ptr() + 2, ws, desc)
