@@ -54,9 +54,10 @@ struct SCfg {
     static constexpr int kLoadRowBytes = F8 ? D : kRowBytes;
     static constexpr int kTileBytesIn = F8 ? kGroup * kSlab * D : kTileBytes;
     static constexpr int kStageBytes = 2 * kTileBytesIn;
-    // E4M3: each warp widens its rows of a stage into a bf16 copy laid out as a bf16 stage
-    static constexpr int kStagingBytes = F8 ? 2 * kTileBytes : 0;
-    static constexpr int kStages = (D == 128 && NT == 2) ? 2 : 3;
+    static constexpr int kStagingBytes = 0;
+    // E4M3 stages carry half the bytes: more of them keep as many bytes in flight
+    static constexpr int kStages = F8 ? (D == 64 ? (NT == 1 ? 6 : 4) : (NT == 1 ? 5 : 4))
+                                      : ((D == 128 && NT == 2) ? 2 : 3);
     static constexpr int kKSteps = D / 16;
     static constexpr int kMTiles = D / 16;
     static constexpr int kMinBlocks = (D == 64 && NT == 1) ? 2 : 1;
@@ -98,18 +99,34 @@ __device__ __forceinline__ int32_t cta_of(int64_t s, int64_t S, int64_t G) {
     return (int32_t)(((s + 1) * G - 1) / S);
 }
 
-// Eight E4M3 codes (bytes 0..7) -> eight bf16 (exact: every E4M3 value is a bf16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes) {
+// Two E4M3 codes (the low 16 bits) -> two f16 (exact: every E4M3 value is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes) {
     uint32_t h2;
     asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e4m3x2 %0, c; }" : "=r"(h2) : "r"(codes & 0xFFFFu));
-    float lo, hi;
-    asm("{ .reg .f16 l, h; mov.b32 {l, h}, %2; cvt.f32.f16 %0, l; cvt.f32.f16 %1, h; }"
-        : "=f"(lo), "=f"(hi) : "r"(h2));
-    return pack_bf16x2(lo, hi);
+    return h2;
 }
-__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 q) {
-    return make_uint4(e4m3x2_to_bf16x2(q.x), e4m3x2_to_bf16x2(q.x >> 16), e4m3x2_to_bf16x2(q.y),
-                      e4m3x2_to_bf16x2(q.y >> 16));
+// Byte offset of (row, 16-byte chunk) in an E4M3 tile as TMA writes it: 64-byte rows (D=64)
+// under the 64B swizzle (chunk ^= (row >> 1) & 3), 128-byte rows (D=128) under the 128B one.
+template <int D>
+__device__ __forceinline__ uint32_t f8_off(int row, int chunk) {
+    if constexpr (D == 64) return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+    else return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// bf16 pair -> f16 pair (the E4M3 path multiplies in f16; exact for |x| in [2^-14, 65504])
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) { return pack_f16x2(bf16_lo(w), bf16_hi(w)); }
+// MMA on the stage's element type: bf16 pools multiply bf16, E4M3 pools f16
+template <bool F8>
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    if constexpr (F8) mma_f16_16816(d, a, b0, b1); else mma_bf16_16816(d, a, b0, b1);
+}
+template <bool F8>
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+    if constexpr (F8) return pack_f16x2(lo, hi); else return pack_bf16x2(lo, hi);
 }
 // Eight bf16 -> eight E4M3 codes of value * inv_scale (float product, nearest even, saturating).
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
@@ -144,8 +161,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     const int32_t Hkv = p.num_kv_heads;
     const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
-    const uint32_t staging = smem_base + C::kStages * C::kStageBytes;  // E4M3: widened stage
-    const uint32_t q_base = staging + C::kStagingBytes;                 // q ring after them
+    const uint32_t q_base = smem_base + C::kStages * C::kStageBytes;   // q ring after the stages
     const uint32_t q_slot_bytes = (uint32_t)(kGroup * G * D * 2);
     allow_dependents();
     if (threadIdx.x == kGroup * 32) {
@@ -467,8 +483,15 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
 #pragma unroll
                     for (int ks = 0; ks < C::kKSteps; ++ks) {
                         const uint32_t* qr = reinterpret_cast<const uint32_t*>(qsm + h * D + ks * 16);
-                        qf[nt][ks][0] = h < G ? qr[c] : 0u;
-                        qf[nt][ks][1] = h < G ? qr[c + 4] : 0u;
+                        if constexpr (F8) {
+                            // E4M3: the k-step's dims in the order the K fragments bring them
+                            // (lane column c holds dims 4c..4c+3 of the 16-dim chunk)
+                            qf[nt][ks][0] = h < G ? bf16x2_to_f16x2(qr[2 * c]) : 0u;
+                            qf[nt][ks][1] = h < G ? bf16x2_to_f16x2(qr[2 * c + 1]) : 0u;
+                        } else {
+                            qf[nt][ks][0] = h < G ? qr[c] : 0u;
+                            qf[nt][ks][1] = h < G ? qr[c + 4] : 0u;
+                        }
                     }
                     m_run[nt][0] = m_run[nt][1] = -INFINITY;
                     l_run[nt][0] = l_run[nt][1] = 0.f;
@@ -485,25 +508,17 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             uint32_t k_tile = smem_base + st * C::kStageBytes;
             uint32_t v_tile = k_tile + C::kTileBytes;
             if constexpr (F8) {
-                // widen this warp's 16 token rows of the E4M3 stage into the bf16 staging tile
-                // (rows past the sequence become zeros), then hand the stage back at once
-                const uint32_t f8k = k_tile, f8v = k_tile + C::kTileBytesIn;
-                k_tile = staging;
-                v_tile = staging + C::kTileBytes;
-                constexpr int kCh = D / 8;
-                for (int i = lane; i < kSlab * kCh; i += 32) {
-                    const int t = i / kCh, c = i - t * kCh;
-                    const int row = stage_row(warp, t, tb);
-                    uint4 kb = make_uint4(0, 0, 0, 0), vb = kb;
-                    if (t < valid) {
-                        kb = e4m3x8_to_bf16x8(*reinterpret_cast<const uint2*>(smem_gen + (f8k - smem_base) + row * D + c * 8));
-                        vb = e4m3x8_to_bf16x8(*reinterpret_cast<const uint2*>(smem_gen + (f8v - smem_base) + row * D + c * 8));
+                if (valid < kSlab) {
+                    // tokens past the sequence: zero their V bytes (0-probability rows add nothing)
+                    const uint32_t f8v = k_tile + C::kTileBytesIn;
+                    for (int i = lane; i < (kSlab - valid) * (D / 16); i += 32) {
+                        const int t = valid + i / (D / 16), ch = i % (D / 16);
+                        *reinterpret_cast<uint4*>(smem_gen + (f8v - smem_base) + f8_off<D>(stage_row(warp, t, tb), ch)) =
+                            make_uint4(0, 0, 0, 0);
                     }
-                    *reinterpret_cast<uint4*>(smem_gen + (swz(k_tile + (c >> 3) * C::kHalfBytes, row, c & 7) - smem_base)) = kb;
-                    *reinterpret_cast<uint4*>(smem_gen + (swz(v_tile + (c >> 3) * C::kHalfBytes, row, c & 7) - smem_base)) = vb;
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
             } else if (valid < kSlab) {
                 // tokens past the sequence: zero V so that 0-probability rows add nothing
                 for (int i = lane; i < (kSlab - valid) * 8 * C::kHalves; i += 32) {
@@ -523,13 +538,31 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+            if constexpr (F8) {
+                // E4M3 K straight from the tile: one ldmatrix.x4 brings 16 tokens x 32 dims of
+                // codes (lane (r, c): 4 codes, dims 4c..4c+3 of a chunk), widened to f16 pairs
 #pragma unroll
-            for (int ks = 0; ks < C::kKSteps; ++ks) {
-                const int ch = 2 * ks + (mi >> 1);
-                uint32_t a[4];
-                ldmatrix_x4(swz(k_tile + (ch >> 3) * C::kHalfBytes, row_a, ch), a);
+                for (int ks = 0; ks < C::kKSteps; ks += 2) {
+                    uint32_t w[4];
+                    ldmatrix_x4(k_tile + f8_off<D>(row_a, ks + (mi >> 1)), w);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const uint32_t a[4] = {e4m3x2_to_f16x2(w[2 * h2]), e4m3x2_to_f16x2(w[2 * h2 + 1]),
+                                               e4m3x2_to_f16x2(w[2 * h2] >> 16), e4m3x2_to_f16x2(w[2 * h2 + 1] >> 16)};
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            mma_16816<F8>(sacc[nt], a, qf[nt][ks + h2][0], qf[nt][ks + h2][1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < C::kKSteps; ++ks) {
+                    const int ch = 2 * ks + (mi >> 1);
+                    uint32_t a[4];
+                    ldmatrix_x4(swz(k_tile + (ch >> 3) * C::kHalfBytes, row_a, ch), a);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_16816<F8>(sacc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+                }
             }
             // ---- online softmax over the 16 rows (tokens) per head column ----
             const bool v_lo = r < valid, v_hi = (r + 8) < valid;
@@ -561,20 +594,45 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     o_acc[nt][mt][2] *= al0;
                     o_acc[nt][mt][3] *= al1;
                 }
-                pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));   // tokens 0-7
-                pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));   // tokens 8-15
+                pb[nt][0] = movmatrix_trans(pack_p<F8>(p0, p1));   // tokens 0-7
+                pb[nt][1] = movmatrix_trans(pack_p<F8>(p2, p3));   // tokens 8-15
             }
             // ---- O^T += V^T P : 16 head-dim rows x 8 heads per (m-tile, n-tile) ----
+            if constexpr (F8) {
+                // E4M3 V: ldmatrix.trans over byte pairs gives lane (r, c) tokens 2c, 2c+1 of dims
+                // 2r, 2r+1; byte permutes split even and odd dims into two m-tiles (o_acc[2j]:
+                // dims 32j + 2r (+16), o_acc[2j+1]: dims 32j + 2r + 1 (+16))
+                const uint32_t f8v = k_tile + C::kTileBytesIn;
 #pragma unroll
-            for (int mt = 0; mt < C::kMTiles; ++mt) {
-                const int ch = 2 * mt + (mi & 1);
-                uint32_t a[4];
-                ldmatrix_x4_trans(swz(v_tile + (ch >> 3) * C::kHalfBytes, row_b, ch), a);
+                for (int j = 0; j < D / 32; ++j) {
+                    uint32_t w[4];
+                    ldmatrix_x4_trans(f8v + f8_off<D>(row_b, 2 * j + (mi & 1)), w);
+                    const uint32_t ae[4] = {e4m3x2_to_f16x2(__byte_perm(w[0], 0u, 0x20u)),
+                                            e4m3x2_to_f16x2(__byte_perm(w[1], 0u, 0x20u)),
+                                            e4m3x2_to_f16x2(__byte_perm(w[2], 0u, 0x20u)),
+                                            e4m3x2_to_f16x2(__byte_perm(w[3], 0u, 0x20u))};
+                    const uint32_t ao[4] = {e4m3x2_to_f16x2(__byte_perm(w[0], 0u, 0x31u)),
+                                            e4m3x2_to_f16x2(__byte_perm(w[1], 0u, 0x31u)),
+                                            e4m3x2_to_f16x2(__byte_perm(w[2], 0u, 0x31u)),
+                                            e4m3x2_to_f16x2(__byte_perm(w[3], 0u, 0x31u))};
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o_acc[nt][mt], a, pb[nt][0], pb[nt][1]);
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma_16816<F8>(o_acc[nt][2 * j], ae, pb[nt][0], pb[nt][1]);
+                        mma_16816<F8>(o_acc[nt][2 * j + 1], ao, pb[nt][0], pb[nt][1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int mt = 0; mt < C::kMTiles; ++mt) {
+                    const int ch = 2 * mt + (mi & 1);
+                    uint32_t a[4];
+                    ldmatrix_x4_trans(swz(v_tile + (ch >> 3) * C::kHalfBytes, row_b, ch), a);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_16816<F8>(o_acc[nt][mt], a, pb[nt][0], pb[nt][1]);
+                }
             }
             __syncwarp();
-            if (!F8 && lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+            if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
             if (!(hd.flags & kLast)) continue;
 
             // ======== end of this warp's segment: store, or publish a partial ========
@@ -595,10 +653,19 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                         const int h = nt * 8 + 2 * c + jj;
                         if (h >= G) continue;
                         const float inv = p.out_scale / l_run[nt][jj];
+                        if constexpr (F8) {   // m-tiles 2j / 2j+1 hold dims 32j + 2r / + 1 (and + 16)
 #pragma unroll
-                        for (int mt = 0; mt < C::kMTiles; ++mt) {
-                            out[(size_t)h * D + mt * 16 + r] = f32_to_bf16_rn(o_acc[nt][mt][jj] * inv);
-                            out[(size_t)h * D + mt * 16 + r + 8] = f32_to_bf16_rn(o_acc[nt][mt][jj + 2] * inv);
+                            for (int j = 0; j < D / 32; ++j) {
+                                uint32_t* o32 = reinterpret_cast<uint32_t*>(out + (size_t)h * D + 32 * j + 2 * r);
+                                o32[0] = pack_bf16x2(o_acc[nt][2 * j][jj] * inv, o_acc[nt][2 * j + 1][jj] * inv);
+                                o32[8] = pack_bf16x2(o_acc[nt][2 * j][jj + 2] * inv, o_acc[nt][2 * j + 1][jj + 2] * inv);
+                            }
+                        } else {
+#pragma unroll
+                            for (int mt = 0; mt < C::kMTiles; ++mt) {
+                                out[(size_t)h * D + mt * 16 + r] = f32_to_bf16_rn(o_acc[nt][mt][jj] * inv);
+                                out[(size_t)h * D + mt * 16 + r + 8] = f32_to_bf16_rn(o_acc[nt][mt][jj + 2] * inv);
+                            }
                         }
                     }
                 continue;
@@ -612,10 +679,19 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     if (h >= G) continue;
                     const float inv = p.out_scale / l_run[nt][jj];
                     float* po = p.part_o + (prow + h) * D;
+                    if constexpr (F8) {
 #pragma unroll
-                    for (int mt = 0; mt < C::kMTiles; ++mt) {
-                        po[mt * 16 + r] = o_acc[nt][mt][jj] * inv;
-                        po[mt * 16 + r + 8] = o_acc[nt][mt][jj + 2] * inv;
+                        for (int j = 0; j < D / 32; ++j) {
+                            float2* p2 = reinterpret_cast<float2*>(po + 32 * j + 2 * r);
+                            p2[0] = make_float2(o_acc[nt][2 * j][jj] * inv, o_acc[nt][2 * j + 1][jj] * inv);
+                            p2[8] = make_float2(o_acc[nt][2 * j][jj + 2] * inv, o_acc[nt][2 * j + 1][jj + 2] * inv);
+                        }
+                    } else {
+#pragma unroll
+                        for (int mt = 0; mt < C::kMTiles; ++mt) {
+                            po[mt * 16 + r] = o_acc[nt][mt][jj] * inv;
+                            po[mt * 16 + r + 8] = o_acc[nt][mt][jj + 2] * inv;
+                        }
                     }
                     if (r == 0) p.part_lse[prow + h] = m_run[nt][jj] + __log2f(l_run[nt][jj]);
                 }
@@ -646,7 +722,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D view [blocks * Hkv][block_size][head_dim]; box = 64 dims x tb tokens x 8 kv heads.
-// bf16 pools: boxes of 64 dims in 128-byte swizzled rows; E4M3 pools: whole D-byte rows, no swizzle.
+// bf16 pools: boxes of 64 dims in 128-byte swizzled rows; E4M3 pools: whole D-byte rows,
+// 64-byte rows (D=64) under the 64B swizzle, 128-byte rows under the 128B one.
 bool make_map(CUtensorMap* map, const void* base, const DecodeParams& p) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -659,9 +736,11 @@ bool make_map(CUtensorMap* map, const void* base, const DecodeParams& p) {
                                (cuuint32_t)(p.block_size < kSlab ? p.block_size : kSlab),
                                (cuuint32_t)kGroup};
     const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle swz_mode = !p.kv_fp8          ? CU_TENSOR_MAP_SWIZZLE_128B
+                                        : p.head_dim == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                           : CU_TENSOR_MAP_SWIZZLE_128B;
     return fn(map, p.kv_fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              p.kv_fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz_mode,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
