@@ -55,12 +55,14 @@ struct SCfg {
     static constexpr int kTileBytesIn = F8 ? kGroup * kSlab * D : kTileBytes;
     static constexpr int kStageBytes = 2 * kTileBytesIn;
     static constexpr int kStagingBytes = 0;
-    // E4M3 stages carry half the bytes: more of them keep as many bytes in flight
-    static constexpr int kStages = F8 ? (D == 64 ? (NT == 1 ? 6 : 4) : (NT == 1 ? 5 : 4))
+    // E4M3 stages carry half the bytes: more of them keep as many bytes in flight, except at
+    // D=128, G<=8, where two CTAs of two stages per SM beat one of five (a CTA retires TMA
+    // requests at a bounded rate, so more CTAs issue more of them)
+    static constexpr int kStages = F8 ? (D == 64 ? (NT == 1 ? 6 : 4) : (NT == 1 ? 2 : 4))
                                       : ((D == 128 && NT == 2) ? 2 : 3);
     static constexpr int kKSteps = D / 16;
     static constexpr int kMTiles = D / 16;
-    static constexpr int kMinBlocks = (D == 64 && NT == 1) ? 2 : 1;
+    static constexpr int kMinBlocks = ((D == 64 && NT == 1) || (F8 && D == 128 && NT == 1)) ? 2 : 1;
     // dynamic shared memory for query group size g
     static constexpr size_t smem_bytes(int g) {
         return (size_t)kStages * kStageBytes + kStagingBytes + (size_t)kQSlots * kGroup * g * D * 2 + 1024;
