@@ -523,7 +523,7 @@ def run_ours(args, rank, world, dist):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
-                     "traffic": profiled_traffic(args.config, kernel_name),
+                     "traffic": profiled_traffic(args.config + ("-e4m3" if e4m3 else ""), kernel_name),
                      "kernel": ("pa_append_decode (%s)" if fused else "pa_decode (%s)") % kernel_name,
                      "algorithmic_bytes_per_launch": kv_bytes,
                      "avg_launch_ms": dec_avg_ms,
