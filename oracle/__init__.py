@@ -77,6 +77,8 @@ def _lib():
         lib.oracle_paged_decode_e4m3.argtypes = [vp, vp, vp, dbl, dbl, vp, vp, i64, i64, i64, i64, i64,
                                                  i64, dbl, vp]
         lib.oracle_paged_decode_e4m3.restype = ctypes.c_int
+        lib.oracle_paged_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, dbl, vp]
+        lib.oracle_paged_prefill.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_num_threads.restype = None
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -298,4 +300,25 @@ def paged_decode_e4m3(q, k_cache, v_cache, k_scale: float, v_scale: float, block
                                          Bs, bt.shape[1], float(scale), out.ctypes.data)
     if rc != 0:
         raise RuntimeError("oracle_paged_decode_e4m3 failed (%d)" % rc)
+    return out
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, cu_q, context_lens, scale: float) -> np.ndarray:
+    """fp64 causal attention of each sequence's last Tq = cu_q[b+1]-cu_q[b] tokens (queries,
+    rows of q [total_q, Hq, D]) over its paged cache of context_lens[b] tokens."""
+    q = _c(q, np.uint16)
+    kc = _c(k_cache, np.uint16)
+    vc = _c(v_cache, np.uint16)
+    bt = _c(block_tables, np.int32)
+    cq = _c(cu_q, np.int32)
+    lens = _c(context_lens, np.int32)
+    T, Hq, D = q.shape
+    N, Hkv, Bs, _ = kc.shape
+    B = lens.shape[0]
+    assert cq.shape == (B + 1,) and cq[-1] == T
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    rc = _lib().oracle_paged_prefill(q.ctypes.data, kc.ctypes.data, vc.ctypes.data, bt.ctypes.data, cq.ctypes.data,
+                                     lens.ctypes.data, B, Hq, Hkv, D, Bs, bt.shape[1], float(scale), out.ctypes.data)
+    if rc != 0:
+        raise RuntimeError("oracle_paged_prefill failed (%d)" % rc)
     return out

@@ -492,3 +492,62 @@ int oracle_paged_decode_e4m3(const uint16_t* q, const uint8_t* k_cache, const ui
     }
     return failed ? -2 : 0;
 }
+
+/*
+ * ---- paged prefill (chunked prefill) ----
+ * "Nano-vLLM로 배우는 vLLM 추론 엔진 작동 원리 한눈에 정리" (tilnote.io), section
+ * "Prefill vs Decode: 추론이 '한 번에 읽고, 한 글자씩 쓴다'": prefill processes the
+ * whole input at once; the Tiny-vLLM summary page, section "고성능 추론을 위한 고급
+ * 최적화 기법", fixes the attention formula and the causal mask (a token sees only
+ * itself and earlier tokens).  Reading: sequence b holds context_lens[b] = L
+ * tokens in the paged cache after this step's append, the last Tq of them are
+ * this step's queries (q rows cu_q[b] .. cu_q[b+1]-1, positions L-Tq .. L-1),
+ * and the query at position p attends to cache tokens 0..p.
+ *   q   [total_q][Hq][D] bf16      out [total_q][Hq][D] double
+ */
+int oracle_paged_prefill(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                         const int32_t* block_tables, const int32_t* cu_q, const int32_t* context_lens,
+                         int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                         int64_t block_size, int64_t max_blocks_per_seq, double scale, double* out) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return -1;
+    const int64_t pairs = num_seqs * num_kv_heads;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_num_threads())
+    for (int64_t pair = 0; pair < pairs; ++pair) {
+        const int64_t b = pair / num_kv_heads, kvh = pair % num_kv_heads;
+        const int64_t L = context_lens[b];
+        const int64_t q0 = cu_q[b], Tq = cu_q[b + 1] - cu_q[b];
+        if (Tq <= 0) continue;
+        if (Tq > L) {
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        const int32_t* table_row = block_tables + b * max_blocks_per_seq;
+        double* K = (double*)malloc(sizeof(double) * (size_t)(L * head_dim));
+        double* V = (double*)malloc(sizeof(double) * (size_t)(L * head_dim));
+        double* s = (double*)malloc(sizeof(double) * (size_t)L);
+        double* qd = (double*)malloc(sizeof(double) * (size_t)head_dim);
+        if (!K || !V || !s || !qd) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            gather_sequence(k_cache, table_row, L, kvh, num_kv_heads, block_size, head_dim, K);
+            gather_sequence(v_cache, table_row, L, kvh, num_kv_heads, block_size, head_dim, V);
+            for (int64_t i = 0; i < Tq; ++i) {
+                const int64_t pos = L - Tq + i;             /* the query's position */
+                for (int64_t h = 0; h < num_q_heads; ++h) {
+                    if (kv_head_of(h, num_q_heads, num_kv_heads) != kvh) continue;
+                    const int64_t row = (q0 + i) * num_q_heads + h;
+                    for (int64_t d = 0; d < head_dim; ++d) qd[d] = oracle_bf16_to_double(q[row * head_dim + d]);
+                    attend(qd, K, V, 0, pos + 1, head_dim, scale, s, out + row * head_dim, NULL);
+                }
+            }
+        }
+        free(K);
+        free(V);
+        free(s);
+        free(qd);
+    }
+    return failed ? -2 : 0;
+}

@@ -1,6 +1,6 @@
 """The oracle pins have teeth: each plausible mistake, planted in a copy of the
 oracle's C source and compiled on the CPU, must make at least one pin fail
-(pins of tests/test_oracle.py, tests/test_oracle_rope.py and tests/test_oracle_fp8.py).
+(pins of tests/test_oracle.py, test_oracle_rope.py, test_oracle_fp8.py and test_oracle_prefill.py).
 
 The mutant library replaces the oracle's loaded library only for the duration
 of one test; the real oracle source is never modified.
@@ -15,6 +15,7 @@ import pytest
 import oracle
 from tests import test_oracle as pins
 from tests import test_oracle_fp8 as fp8_pins
+from tests import test_oracle_prefill as prefill_pins
 from tests import test_oracle_rope as rope_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.c")
@@ -73,6 +74,10 @@ MUTANTS = {
     # FP8 decode: V scale dropped; K and V scales swapped
     "e4m3_decode_v_scale": ("gather_sequence_e4m3(v_cache, v_scale,", "gather_sequence_e4m3(v_cache, 1.0,"),
     "e4m3_decode_scales_swapped": ("gather_sequence_e4m3(k_cache, k_scale,", "gather_sequence_e4m3(k_cache, v_scale,"),
+    # prefill: causal limit off by one, query positions from 0, query rows not offset
+    "prefill_causal": ("attend(qd, K, V, 0, pos + 1, head_dim", "attend(qd, K, V, 0, pos, head_dim"),
+    "prefill_position": ("const int64_t pos = L - Tq + i;", "const int64_t pos = i;"),
+    "prefill_rows": ("const int64_t row = (q0 + i) * num_q_heads + h;", "const int64_t row = i * num_q_heads + h;"),
     # bf16 rounding breaks ties away from zero instead of to even
     "round_ties_away": ("v = ldexp(rint(ldexp(v, -qexp)), qexp);", "v = ldexp(round(ldexp(v, -qexp)), qexp);"),
 }
@@ -82,7 +87,8 @@ def _pin_calls():
     """Every pin in test_oracle as a zero-argument callable (parametrised ones expanded)."""
     calls = []
     members = (inspect.getmembers(pins, inspect.isfunction) + inspect.getmembers(rope_pins, inspect.isfunction)
-               + inspect.getmembers(fp8_pins, inspect.isfunction))
+               + inspect.getmembers(fp8_pins, inspect.isfunction)
+               + inspect.getmembers(prefill_pins, inspect.isfunction))
     for name, fn in members:
         if not name.startswith("test_"):
             continue
@@ -124,7 +130,8 @@ def test_pins_catch_planted_mistake(mutant, monkeypatch):
                     "oracle_append_kv", "oracle_paged_decode", "oracle_paged_decode_partial",
                     "oracle_merge_partials", "oracle_set_num_threads", "oracle_num_threads",
                     "oracle_rope", "oracle_round_bf16", "oracle_e4m3_to_double", "oracle_e4m3_from_float",
-                    "oracle_quantize_e4m3", "oracle_append_kv_e4m3", "oracle_paged_decode_e4m3"):
+                    "oracle_quantize_e4m3", "oracle_append_kv_e4m3", "oracle_paged_decode_e4m3",
+                    "oracle_paged_prefill"):
             f_real, f_mut = getattr(real, sym), getattr(mut, sym)
             f_mut.argtypes = f_real.argtypes
             f_mut.restype = f_real.restype

@@ -1,0 +1,69 @@
+"""Pins of the oracle's paged (chunked) prefill against what its definition fixes.
+
+Reading: sequence b holds context_lens[b] = L tokens after this step's append; its
+last Tq tokens are the queries (positions L-Tq .. L-1) and the query at position p
+attends to cache tokens 0..p (the causal mask of the Tiny-vLLM summary page, section
+"고성능 추론을 위한 고급 최적화 기법").  Pinned by: per-query decodes over the
+truncated context (a different loop of the oracle), the one-query case, causality
+(keys after p do not matter, keys up to p do), and chunk splitting.
+"""
+import numpy as np
+
+import oracle
+import workloads as wl
+
+
+def _case(seed, lens, q_lens, **kw):
+    b = wl.small_batch(seed, lens, **kw)
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    q = (rng.standard_normal((int(cu[-1]), b.num_q_heads, b.head_dim)).astype(np.float32)
+         .view(np.uint32) >> 16).astype(np.uint16)
+    return b, q, cu
+
+
+def test_each_query_is_a_decode_over_its_prefix():
+    lens, q_lens = [37, 90, 16], [5, 33, 16]
+    b, q, cu = _case(3, lens, q_lens, num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16)
+    out = oracle.paged_prefill(q, b.k_cache, b.v_cache, b.block_tables, cu, b.context_lens, b.scale)
+    for s in range(len(lens)):
+        L = int(b.context_lens[s])
+        for i in range(q_lens[s]):
+            pos = L - q_lens[s] + i
+            row = int(cu[s]) + i
+            want = oracle.paged_decode(q[row:row + 1], b.k_cache, b.v_cache, b.block_tables[s:s + 1],
+                                       np.array([pos + 1], dtype=np.int32), b.scale)
+            np.testing.assert_allclose(out[row], want[0], rtol=0, atol=1e-13)
+
+
+def test_one_query_per_sequence_is_the_decode():
+    b = wl.small_batch(4, [20, 7, 100], num_q_heads=4, num_kv_heads=4, head_dim=128, block_size=8)
+    cu = np.arange(4, dtype=np.int32)
+    out = oracle.paged_prefill(b.q, b.k_cache, b.v_cache, b.block_tables, cu, b.context_lens, b.scale)
+    want = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale)
+    np.testing.assert_array_equal(out, want)
+
+
+def test_causality():
+    b, q, cu = _case(5, [48], [48], num_q_heads=2, num_kv_heads=1, head_dim=64, block_size=16)
+    out = oracle.paged_prefill(q, b.k_cache, b.v_cache, b.block_tables, cu, b.context_lens, b.scale)
+    k2, v2 = b.k_cache.copy(), b.v_cache.copy()
+    p = 20                                        # change every key and value after position 20
+    for pos in range(p + 1, 48):
+        blk, off = b.block_tables[0][pos // 16], pos % 16
+        k2[blk, :, off, :] ^= 0x0040
+        v2[blk, :, off, :] ^= 0x0040
+    out2 = oracle.paged_prefill(q, k2, v2, b.block_tables, cu, b.context_lens, b.scale)
+    np.testing.assert_array_equal(out2[:p + 1], out[:p + 1])   # queries 0..20 see only 0..p
+    assert np.abs(out2[p + 1:] - out[p + 1:]).max() > 1e-6      # later ones see the change
+
+
+def test_a_prefill_split_into_chunks_gives_the_same_outputs():
+    b, q, cu = _case(6, [70], [70], num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16)
+    whole = oracle.paged_prefill(q, b.k_cache, b.v_cache, b.block_tables, cu, b.context_lens, b.scale)
+    a = 29
+    first = oracle.paged_prefill(q[:a], b.k_cache, b.v_cache, b.block_tables, np.array([0, a], dtype=np.int32),
+                                 np.array([a], dtype=np.int32), b.scale)
+    second = oracle.paged_prefill(q[a:], b.k_cache, b.v_cache, b.block_tables,
+                                  np.array([0, 70 - a], dtype=np.int32), np.array([70], dtype=np.int32), b.scale)
+    np.testing.assert_array_equal(np.concatenate([first, second]), whole)
