@@ -55,6 +55,8 @@ WORKLOAD_TEXT = {
     "c5": "continuous-batching trace: 16 layers (own pools), 256 live sequences, lognormal L (median 512, "
           "sigma 1, <=16384), 100 decode steps, finish p=0.01 per step with replacement, Hq=32, Hkv=8, "
           "D=64, Bs=16",
+    "pf": "paged chunked prefill, Llama-3.2-1B-shaped layer: 4 sequences, 2048 new tokens each after "
+          "0/512/1024/1536 cached, Hq=32, Hkv=8, D=64, Bs=16 (append of the chunk + causal attention)",
     "pc": "prefix caching + copy-on-write: host admission by token ids of 32 C3-shaped requests "
           "(1024-token shared prefix + suffix~U[256,7168], Bs=256); device copy of 8192 random "
           "blocks of the C2 geometry (Hkv=8, Bs=16, D=64) per step",
@@ -67,7 +69,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4", "c5", "pc"], default="c2",
+    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4", "c5", "pc", "pf"], default="c2",
                     help="pc: prefix caching + copy-on-write (host admission by token ids on the "
                          "C3 request mix, device block copies)")
     ap.add_argument("--trace-steps", type=int, default=200,
@@ -828,6 +830,141 @@ def run_pc(args, rank, world, dist):
     }
 
 
+PF_CACHED, PF_NEW = [0, 512, 1024, 1536], 2048
+
+
+def prefill_flops(lens, q_lens, num_q_heads, head_dim):
+    """4 * (p + 1) * D per query head and query at position p (q.K and p.V, 2 flops a MAC)."""
+    f = 0
+    for L, T in zip(lens, q_lens):
+        pos = np.arange(L - T, L, dtype=np.int64)
+        f += int(4 * (pos + 1).sum()) * head_dim * num_q_heads
+    return f
+
+
+def run_pf(args, rank, world, dist):
+    """Chunked prefill: a step appends each sequence's new chunk and runs the causal attention."""
+    import torch
+    import pagedattention_kv_cache_pa_b200 as pa
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    lens = [c + PF_NEW for c in PF_CACHED]
+    q_lens = [PF_NEW] * len(lens)
+    b = wl.make_batch("PF", wl.CONFIG_SEED_BASE + 41, [L - 1 for L in lens], num_q_heads=32, num_kv_heads=8,
+                      head_dim=64, block_size=16)
+    Hq, Hkv, D, Bs = b.num_q_heads, b.num_kv_heads, b.head_dim, b.block_size
+    B = len(lens)
+    rng = np.random.default_rng(wl.CONFIG_SEED_BASE + 42)
+    T = sum(q_lens)
+    bits = lambda shape: (rng.standard_normal(shape).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    q_h, k_h, v_h = bits((T, Hq, D)), bits((T, Hkv, D)), bits((T, Hkv, D))
+    slots = np.concatenate([[int(b.block_tables[s_][p // Bs]) * Bs + p % Bs for p in range(L - Tq, L)]
+                            for s_, (L, Tq) in enumerate(zip(lens, q_lens))]).astype(np.int64)
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    kc, vc = to(b.k_cache), to(b.v_cache)
+    q, k, v = to(q_h), to(k_h), to(v_h)
+    slots_d, cu_d = torch.from_numpy(slots).to(dev), torch.from_numpy(cu).to(dev)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device=dev)
+    tables_d = torch.from_numpy(b.block_tables).to(dev)
+    desc = pa.CacheDesc.make(num_blocks=b.num_blocks, block_size=Bs, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D,
+                             max_blocks_per_seq=b.max_blocks_per_seq)
+    out = torch.empty_like(q)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+
+    def step(qq, kk, vv):
+        pa.pa_append_kv(kk, vv, slots_d, kc, vc, desc, stream=stream)
+        pa.pa_prefill(qq, kc, vc, tables_d, cu_d, lens_d, PF_NEW, b.scale, out, ws, desc, stream=stream)
+
+    step(q, k, v)
+    torch.cuda.synchronize()
+    if pa.pa_decode_status(ws) != 0:
+        raise RuntimeError("prefill reported an error")
+    for _ in range(args.warmup):
+        step(q, k, v)
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
+    e0.record(stream)
+    for i in range(K):
+        pa.pa_append_kv(k, v, slots_d, kc, vc, desc, stream=stream)
+        ev[i][0].record(stream)
+        pa.pa_prefill(q, kc, vc, tables_d, cu_d, lens_d, PF_NEW, b.scale, out, ws, desc, stream=stream)
+        ev[i][1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    att_ms = float(np.mean([a.elapsed_time(c) for a, c in ev]))
+    if dist is not None:
+        t = torch.tensor([ms, att_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, att_ms = float(t[0]), float(t[1])
+    # e2e: q, k, v from pinned host memory every step, the output back
+    hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q_h, k_h, v_h))
+    hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    E = max(1, min(args.e2e_steps, 200))
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(E):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        step(dq, dk, dv)
+        hout.copy_(out, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if rank != 0:
+        return None
+    flops = prefill_flops(lens, q_lens, Hq, D)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    peak, kind = (float(peaks["bf16_tflops"]), "measured") if "bf16_tflops" in peaks else (1590.0, "fallback")
+    achieved = flops / (att_ms / 1e3) / 1e12
+    res = {
+        "metric": "paged prefill tokens/s and TFLOP/s (fraction of B200 bf16 peak)",
+        "value": world * T * K / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT["pf"], "config": "pf", "sequences": B, "new_tokens": q_lens,
+                   "context": lens, "call": "pa_append_kv + pa_prefill",
+                   "l2": "working set (%.0f MB of KV) fits L2: prefill is compute-bound" % (2 * b.k_cache.nbytes / 1e6)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_kind": kind, "traffic": None, "kernel": "pa_prefill (mma.sync bf16)",
+                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_ms},
+        "e2e": {"value": world * T * E / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int((q_h.nbytes + k_h.nbytes + v_h.nbytes)), "d2h_bytes_per_step": int(q_h.nbytes),
+                "steps": E},
+        "gpu_launches": 2 * K, "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        import oracle
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < max(1.0, args.cpu_seconds) and n < 8:
+            s_ = n % B
+            lo = lens[s_] - 64                        # the chunk's last 64 queries of one sequence
+            qs = q_h[int(cu[s_]) + PF_NEW - 64: int(cu[s_]) + PF_NEW]
+            oracle.paged_prefill(qs, b.k_cache, b.v_cache, b.block_tables[s_:s_ + 1], np.array([0, 64], np.int32),
+                                 np.array([lens[s_]], np.int32), b.scale)
+            n += 1
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": 64 * n / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+                               "kind": "oracle", "sample": "%d x 64 query tokens at the end of a chunk (the "
+                               "costliest positions), %.1f s" % (n, dt)}
+    return res
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -847,7 +984,7 @@ def main(argv=None):
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = dist_mod
     try:
-        runner = {"c5": run_c5, "pc": run_pc}.get(args.config, run_ours)
+        runner = {"c5": run_c5, "pc": run_pc, "pf": run_pf}.get(args.config, run_ours)
         res = runner(args, rank, world, dist)
         if res is not None:
             print(json.dumps(res), flush=True)

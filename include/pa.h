@@ -261,6 +261,31 @@ PA_API int pa_append_decode(const pa_bf16* q, const pa_bf16* k, const pa_bf16* v
                             void* stream);
 
 /*
+ * Paged (chunked) prefill attention.  Prefill processes a prompt, or a chunk of
+ * it, at once (Nano-vLLM page, "Nano-vLLM로 배우는 vLLM 추론 엔진 작동 원리 한눈에
+ * 정리", section "Prefill vs Decode"); the causal mask lets a token see only
+ * itself and earlier tokens (Tiny-vLLM summary page, section "고성능 추론을 위한
+ * 고급 최적화 기법").  Sequence b holds L = context_lens[b] tokens in the paged
+ * cache, this chunk's K/V included (append them first, e.g. pa_append_kv with
+ * their slots); its Tq = cu_seqlens_q[b+1] - cu_seqlens_q[b] query rows of q
+ * ([total_q][Hq][D] bf16, rows cu_seqlens_q[b] ..) sit at positions L-Tq .. L-1,
+ * and the query at position p attends to cache tokens 0..p:
+ *   out[row][h] = bf16( sum_{j<=p} softmax_j(scale * q[row][h] . K_j) V_j ),
+ * K_j, V_j of kv head h / (Hq/Hkv).  fp32 accumulation, online softmax.
+ * cu_seqlens_q: [num_seqs + 1] int32 device array (0 first, non-decreasing);
+ * max_q_len >= every Tq (sizes the grid).  workspace: >= 256 bytes, 256-byte
+ * aligned, its status word as for pa_decode (a block id outside the pool, or
+ * L < Tq or L past the table: the sequence's rows are left unwritten and
+ * pa_decode_status reports it).  head_dim 64 or 128.
+ * Errors: PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA.
+ */
+PA_API int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
+                      const int32_t* block_tables, const int32_t* cu_seqlens_q,
+                      const int32_t* context_lens, int32_t num_seqs, int32_t max_q_len, float scale,
+                      pa_bf16* out, void* workspace, size_t workspace_bytes,
+                      const pa_cache_desc* desc, void* stream);
+
+/*
  * Synchronises `stream`, reads and clears the workspace's device status word.
  * Returns PA_OK, PA_ERR_BAD_BLOCK, PA_ERR_BAD_LENGTH or PA_ERR_TIMEOUT (the
  * first set, in that order), or PA_ERR_CUDA if the read fails.

@@ -226,6 +226,49 @@ extern "C" int pa_append_kv_e4m3(const pa_bf16* k, const pa_bf16* v, const int64
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+extern "C" int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
+                          const int32_t* block_tables, const int32_t* cu_seqlens_q,
+                          const int32_t* context_lens, int32_t num_seqs, int32_t max_q_len, float scale,
+                          pa_bf16* out, void* workspace, size_t workspace_bytes,
+                          const pa_cache_desc* desc, void* stream) {
+    int rc = check_desc(desc);
+    if (rc != PA_OK) return rc;
+    if (num_seqs < 0 || num_seqs > 65535 || max_q_len < 0 || !(scale > 0.f) || !(scale < INFINITY))
+        return PA_ERR_INVALID;
+    if (desc->head_dim != 64 && desc->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (desc->num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || max_q_len == 0) return PA_OK;
+    if ((int64_t)max_q_len * (desc->num_q_heads / desc->num_kv_heads) > (int64_t)64 * 65535)
+        return PA_ERR_UNSUPPORTED;
+    if (!q || !k_cache || !v_cache || !block_tables || !cu_seqlens_q || !context_lens || !out)
+        return PA_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(cu_seqlens_q, 4) || !aligned(context_lens, 4))
+        return PA_ERR_INVALID;
+    if (!workspace || !aligned(workspace, kWorkspaceAlign) || workspace_bytes < kWorkspaceAlign)
+        return PA_ERR_WORKSPACE;
+    PrefillParams p;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.cu_q = cu_seqlens_q;
+    p.context_lens = context_lens;
+    p.out = out;
+    p.status = static_cast<int32_t*>(workspace);
+    p.num_seqs = num_seqs;
+    p.num_blocks = desc->num_blocks;
+    p.block_size = desc->block_size;
+    p.num_kv_heads = desc->num_kv_heads;
+    p.num_q_heads = desc->num_q_heads;
+    p.head_dim = desc->head_dim;
+    p.group = desc->num_q_heads / desc->num_kv_heads;
+    p.max_blocks_per_seq = desc->max_blocks_per_seq;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const cudaError_t e = launch_prefill(p, max_q_len, (cudaStream_t)stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 extern "C" int pa_copy_blocks(pa_bf16* k_cache, pa_bf16* v_cache, const int32_t* copies, int32_t n,
                               const pa_cache_desc* desc, void* stream) {
     int rc = check_desc(desc);

@@ -66,6 +66,23 @@ struct DecodePlan {
     size_t off_desc, off_lse, off_o, off_qrot, bytes;
 };
 
+// Paged prefill: sequence b's last cu_q[b+1] - cu_q[b] tokens attend causally to its
+// context_lens[b] cached tokens.
+struct PrefillParams {
+    const uint16_t* q;             // [total_q][Hq][D]
+    const uint16_t* k_cache;
+    const uint16_t* v_cache;
+    const int32_t* block_tables;
+    const int32_t* cu_q;           // [B + 1]
+    const int32_t* context_lens;   // [B]
+    uint16_t* out;                 // [total_q][Hq][D]
+    int32_t* status;
+    int32_t num_seqs, num_blocks, block_size, num_kv_heads, num_q_heads, head_dim, group;
+    int32_t max_blocks_per_seq;
+    float scale_log2;
+};
+cudaError_t launch_prefill(const PrefillParams& p, int max_q_len, cudaStream_t stream);
+
 constexpr size_t kWorkspaceAlign = 256;
 
 int num_sms_current_device(int* out);

@@ -1,0 +1,82 @@
+"""Paged (chunked) prefill through the C ABI against the fp64 oracle (needs a B200).
+
+Outputs within 1e-2 + 1e-2 * |oracle|; cases: whole prompts (Tq = L), chunks after a
+cached prefix (Tq < L), one-token chunks, lengths off the 64-key and 64-row tiles,
+GQA groups 1..16, head dims 64 and 128, block sizes 8..256; errors reported through
+the status word without a fault.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+import pagedattention_kv_cache_pa_b200 as pa
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tests import gpu_harness
+    return gpu_harness
+
+
+def _run(h, seed, lens, q_lens, **kw):
+    b = wl.small_batch(seed, lens, **kw)
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    q = (rng.standard_normal((int(cu[-1]), b.num_q_heads, b.head_dim)).astype(np.float32)
+         .view(np.uint32) >> 16).astype(np.uint16)
+    desc = h.desc_of(b)
+    out = torch.full((int(cu[-1]), b.num_q_heads, b.head_dim), 9.0, dtype=torch.bfloat16, device=h.DEV)
+    ws = torch.zeros(256, dtype=torch.uint8, device=h.DEV)
+    pa.pa_prefill(h.to_dev(q), h.to_dev(b.k_cache), h.to_dev(b.v_cache), torch.from_numpy(b.block_tables).to(h.DEV),
+                  torch.from_numpy(cu).to(h.DEV), torch.from_numpy(b.context_lens).to(h.DEV), max(q_lens),
+                  b.scale, out, ws, desc)
+    torch.cuda.synchronize()
+    assert pa.pa_decode_status(ws) == 0
+    ref = oracle.paged_prefill(q, b.k_cache, b.v_cache, b.block_tables, cu, b.context_lens, b.scale)
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    ok, ex = oracle.within_tolerance(got, ref)
+    assert ok, "prefill outside tolerance by %g" % ex
+
+
+SHAPES = [(32, 8, 64, 16), (8, 8, 64, 8), (16, 1, 128, 16), (64, 8, 128, 32), (6, 3, 64, 256), (2, 2, 128, 64),
+          (24, 8, 64, 16)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "Hq%d-Hkv%d-D%d-Bs%d" % s)
+def test_prefill_shapes(h, shape):
+    Hq, Hkv, D, Bs = shape
+    lens = [1, 64, 65, 200, 333, 130]
+    q_lens = [1, 64, 17, 200, 40, 1]                   # whole prompts, chunks, single tokens
+    _run(h, 7000 + Hq + D + Bs, lens, q_lens, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, block_size=Bs)
+
+
+def test_prefill_llama_1b_prompt_and_chunk(h):
+    _run(h, 7100, [2048, 1500], [2048, 700], num_q_heads=32, num_kv_heads=8, head_dim=64, block_size=16)
+
+
+def test_prefill_reports_bad_lengths_and_blocks(h):
+    b = wl.small_batch(7200, [40, 20], num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16)
+    desc = h.desc_of(b)
+    q = torch.zeros((10, 4, 64), dtype=torch.bfloat16, device=h.DEV)
+    out = torch.zeros_like(q)
+    ws = torch.zeros(256, dtype=torch.uint8, device=h.DEV)
+    cu = torch.tensor([0, 5, 10], dtype=torch.int32, device=h.DEV)
+    lens = torch.tensor([40, 3], dtype=torch.int32, device=h.DEV)      # second: fewer tokens than queries
+    kc, vc = h.to_dev(b.k_cache), h.to_dev(b.v_cache)
+    tables = torch.from_numpy(b.block_tables).to(h.DEV)
+    pa.pa_prefill(q, kc, vc, tables, cu, lens, 5, b.scale, out, ws, desc)
+    torch.cuda.synchronize()
+    assert pa.pa_decode_status(ws) == -8
+    bad = b.block_tables.copy()
+    bad[0, 1] = b.num_blocks + 5
+    lens = torch.tensor([40, 20], dtype=torch.int32, device=h.DEV)
+    pa.pa_prefill(q, kc, vc, torch.from_numpy(bad).to(h.DEV), cu, lens, 5, b.scale, out, ws, desc)
+    torch.cuda.synchronize()
+    assert pa.pa_decode_status(ws) == -7
