@@ -110,6 +110,16 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def max_over_ranks(values, dist, device):
+    """Each value's max over all ranks: the slowest rank sets a multi-GPU job's time."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def kv_read_bytes(lens, num_kv_heads, head_dim, elem_bytes=2):
     """Algorithmic K+V bytes one decode launch must read: 2 (K,V) x L x Hkv x D x elem_bytes per
     sequence (2 for bf16 pools, 1 for E4M3)."""
@@ -442,10 +452,7 @@ def run_ours(args, rank, world, dist):
         dec_avg_ms = elapsed_ms / K
     else:
         dec_avg_ms = float(np.mean([s.elapsed_time(e) for s, e in ev_dec]))
-    if dist is not None:
-        t = torch.tensor([elapsed_ms, dec_avg_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, dec_avg_ms = float(t[0]), float(t[1])
+    elapsed_ms, dec_avg_ms = max_over_ranks([elapsed_ms, dec_avg_ms], dist, dev)
     rc = pa.pa_decode_status(ws)
     if rc != 0:
         raise RuntimeError("decode reported %s during timing" % pa.pa_status_string(rc))
@@ -492,10 +499,7 @@ def run_ours(args, rank, world, dist):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms, = max_over_ranks([e2e_ms], dist, dev)
     e2e_value = world * B * E / (e2e_ms / 1e3)
 
     if rank != 0:
@@ -649,10 +653,7 @@ def run_c5(args, rank, world, dist):
     kv_per_call = np.array([kv_read_bytes(lens[i % S], Hkv, D) for i in range(K) for _ in range(NL)],
                            dtype=np.float64)
     gbs = float(kv_per_call.sum() / (call_ms.sum() / 1e3) / 1e9)
-    if dist is not None:
-        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt[0])
+    elapsed_ms, = max_over_ranks([elapsed_ms], dist, dev)
     value = world * B * K / (elapsed_ms / 1e3)
 
     # e2e: the host block manager replays the trace inside the timed region; per step the
@@ -692,10 +693,7 @@ def run_c5(args, rank, world, dist):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt[0])
+    e2e_ms, = max_over_ranks([e2e_ms], dist, dev)
     if rank != 0:
         return None
     peak, peak_kind = measured_peaks()
@@ -803,10 +801,7 @@ def run_pc(args, rank, world, dist):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
+    ms, = max_over_ranks([ms], dist, dev)
     if rank != 0:
         return None
     bytes_step = 2 * 2 * P * Hkv * Bs * D * 2            # K and V, read + write
@@ -900,10 +895,7 @@ def run_pf(args, rank, world, dist):
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     att_ms = float(np.mean([a.elapsed_time(c) for a, c in ev]))
-    if dist is not None:
-        t = torch.tensor([ms, att_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, att_ms = float(t[0]), float(t[1])
+    ms, att_ms = max_over_ranks([ms, att_ms], dist, dev)
     # e2e: q, k, v from pinned host memory every step, the output back
     hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q_h, k_h, v_h))
     hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
@@ -920,7 +912,7 @@ def run_pf(args, rank, world, dist):
         hout.copy_(out, non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
+    e2e_ms, = max_over_ranks([f0.elapsed_time(f1)], dist, dev)
     if rank != 0:
         return None
     flops = prefill_flops(lens, q_lens, Hq, D)
