@@ -18,16 +18,16 @@
 namespace pa {
 namespace {
 
-constexpr int kPieceGroups = 4;
-
-// One CTA of D threads per (sequence, kv head, query head): 4 groups over the
-// pieces (piece k goes to group k % 4) times D/4 float4 columns of the head
+// One CTA of PG * D/4 threads per (sequence, kv head, query head): PG groups over
+// the pieces (piece k goes to group k % PG) times D/4 float4 columns of the head
 // dimension.  Each thread folds its pieces into a running (max, weight, sum)
-// state as their lse and output arrive (one round of independent loads), and
-// the 4 groups' states are merged the same way through shared memory.
-template <int D, bool kStream>
-__global__ void __launch_bounds__(D) merge_kernel(const DecodeParams p) {
+// state as their lse and output arrive (independent loads), and the groups'
+// states are merged the same way through shared memory.  Long contexts cut a
+// sequence into many pieces: 16 groups keep each thread's chain short there.
+template <int D, bool kStream, int PG>
+__global__ void __launch_bounds__(PG * D / 4) merge_kernel(const DecodeParams p) {
     constexpr int kCols = D / 4;
+    constexpr int kPieceGroups = PG;
     allow_dependents();   // a next decode call launched early may plan while this runs
     wait_prerequisite();
     __shared__ float4 s_acc[kPieceGroups][kCols];
@@ -100,27 +100,34 @@ __global__ void __launch_bounds__(D) merge_kernel(const DecodeParams p) {
     }
 }
 
-template <int D, bool kStream>
+template <int D, bool kStream, int PG>
 cudaError_t launch_m(const DecodeParams& p, bool pdl, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.num_seqs, (unsigned)p.num_kv_heads, (unsigned)p.group);
-    cfg.blockDim = dim3(D);
+    cfg.blockDim = dim3(PG * D / 4);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, merge_kernel<D, kStream>, p);
+    return cudaLaunchKernelEx(&cfg, merge_kernel<D, kStream, PG>, p);
+}
+
+template <int D, bool kStream>
+cudaError_t launch_mg(const DecodeParams& p, bool pdl, cudaStream_t stream) {
+    // contexts of 8K tokens and more are cut into many pieces per sequence
+    return p.max_context_len >= 8192 ? launch_m<D, kStream, 16>(p, pdl, stream)
+                                     : launch_m<D, kStream, 4>(p, pdl, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const DecodeParams& p, bool stream_layout, bool pdl, cudaStream_t stream) {
     if (p.head_dim == 64)
-        return stream_layout ? launch_m<64, true>(p, pdl, stream) : launch_m<64, false>(p, pdl, stream);
+        return stream_layout ? launch_mg<64, true>(p, pdl, stream) : launch_mg<64, false>(p, pdl, stream);
     if (p.head_dim == 128)
-        return stream_layout ? launch_m<128, true>(p, pdl, stream) : launch_m<128, false>(p, pdl, stream);
+        return stream_layout ? launch_mg<128, true>(p, pdl, stream) : launch_mg<128, false>(p, pdl, stream);
     return cudaErrorInvalidValue;
 }
 
