@@ -54,7 +54,6 @@ struct SCfg {
     static constexpr int kLoadRowBytes = F8 ? D : kRowBytes;
     static constexpr int kTileBytesIn = F8 ? kGroup * kSlab * D : kTileBytes;
     static constexpr int kStageBytes = 2 * kTileBytesIn;
-    static constexpr int kStagingBytes = 0;
     // E4M3 stages carry half the bytes: more of them keep as many bytes in flight, except at
     // D=128, G<=8, where two CTAs of two stages per SM beat one of five (a CTA retires TMA
     // requests at a bounded rate, so more CTAs issue more of them)
@@ -65,7 +64,7 @@ struct SCfg {
     static constexpr int kMinBlocks = ((D == 64 && NT == 1) || (F8 && D == 128 && NT == 1)) ? 2 : 1;
     // dynamic shared memory for query group size g
     static constexpr size_t smem_bytes(int g) {
-        return (size_t)kStages * kStageBytes + kStagingBytes + (size_t)kQSlots * kGroup * g * D * 2 + 1024;
+        return (size_t)kStages * kStageBytes + (size_t)kQSlots * kGroup * g * D * 2 + 1024;
     }
 };
 

@@ -17,6 +17,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "pa_ptx.cuh"
@@ -228,14 +230,14 @@ __global__ void __launch_bounds__(kThreadsPf) prefill_kernel(const PrefillParams
 template <int D>
 cudaError_t launch_pf(const PrefillParams& p, int max_q_len, cudaStream_t stream) {
     const size_t smem = (size_t)kRows * D * 2 + 4 * (size_t)kKeys * D * 2;
-    static bool attr_set[64] = {};
+    static std::atomic<uint64_t> attr_set{0};           // one bit per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
+    if (!(attr_set.load(std::memory_order_acquire) & (1ull << dev))) {
         const cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    (int)smem);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
     const int tiles = (max_q_len * p.group + kRows - 1) / kRows;
     if (tiles <= 0) return cudaSuccess;

@@ -129,6 +129,22 @@ def test_e4m3_arguments_rejected_without_a_gpu():
                                  kernel=pa.PA_KERNEL_SIMT)) == -2
 
 
+def test_prefill_rejects_bad_arguments_without_a_gpu():
+    lib = binding.lib
+    fake = ctypes.c_void_p(0x10000)
+    d = _desc()
+    call = lambda n, mq, scale, dd, ws=fake, wsb=256: lib.pa_prefill(
+        fake, fake, fake, fake, fake, fake, n, mq, ctypes.c_float(scale), fake, ws, wsb, ctypes.byref(dd), None)
+    assert call(-1, 4, 0.1, d) == -1
+    assert call(2, -1, 0.1, d) == -1
+    assert call(2, 4, 0.0, d) == -1                      # scale must be > 0
+    assert call(2, 4, 0.1, _desc(head_dim=96)) == -2
+    assert call(0, 4, 0.1, d) == 0                        # nothing to do
+    assert call(2, 0, 0.1, d) == 0
+    assert call(2, 4, 0.1, d, ws=None) == -4              # workspace (status word) missing
+    assert call(2, 4, 0.1, d, wsb=16) == -4
+
+
 def test_slot_mapping_entry_matches_oracle():
     import oracle
     rng = np.random.default_rng(0)
