@@ -66,8 +66,11 @@ __global__ void __launch_bounds__(kThreadsPf) prefill_kernel(const PrefillParams
         if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) raise_status(p.status, kStatusBadLength);
         return;
     }
-    const int rows = Tq * G, r0 = blockIdx.x * kRows;
-    if (r0 >= rows) return;
+    // the last row tiles of a chunk attend to the most keys: they take the first CTAs
+    const int rows = Tq * G, ntile = (rows + kRows - 1) / kRows;
+    const int tile = ntile - 1 - (int)blockIdx.x;
+    if (tile < 0) return;
+    const int r0 = tile * kRows;
     const int* table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
