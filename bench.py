@@ -76,6 +76,8 @@ def parse_args(argv=None):
                     help="c5: decode steps timed (the 100-step trace replayed as needed)")
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "split"], default="auto")
     ap.add_argument("--max-ctas", type=int, default=0)
+    ap.add_argument("--prefill-kernel", choices=["auto", "tcgen05", "mma"], default="auto",
+                    help="pf: tcgen05 (tensor-memory accumulators; auto) or warp-level mma.sync")
     ap.add_argument("--path", choices=["fused", "separate"], default="fused",
                     help="fused: pa_append_decode; separate: pa_append_kv then pa_decode")
     ap.add_argument("--split-tokens", type=int, default=0)
@@ -871,7 +873,8 @@ def run_pf(args, rank, world, dist):
 
     def step(qq, kk, vv):
         pa.pa_append_kv(kk, vv, slots_d, kc, vc, desc, stream=stream)
-        pa.pa_prefill(qq, kc, vc, tables_d, cu_d, lens_d, PF_NEW, b.scale, out, ws, desc, stream=stream)
+        pa.pa_prefill(qq, kc, vc, tables_d, cu_d, lens_d, PF_NEW, b.scale, out, ws, desc, stream=stream,
+                      kernel=args.prefill_kernel)
 
     step(q, k, v)
     torch.cuda.synchronize()
@@ -888,7 +891,8 @@ def run_pf(args, rank, world, dist):
     for i in range(K):
         pa.pa_append_kv(k, v, slots_d, kc, vc, desc, stream=stream)
         ev[i][0].record(stream)
-        pa.pa_prefill(q, kc, vc, tables_d, cu_d, lens_d, PF_NEW, b.scale, out, ws, desc, stream=stream)
+        pa.pa_prefill(q, kc, vc, tables_d, cu_d, lens_d, PF_NEW, b.scale, out, ws, desc, stream=stream,
+                      kernel=args.prefill_kernel)
         ev[i][1].record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -932,7 +936,8 @@ def run_pf(args, rank, world, dist):
                    "context": lens, "call": "pa_append_kv + pa_prefill",
                    "l2": "working set (%.0f MB of KV) fits L2: prefill is compute-bound" % (2 * b.k_cache.nbytes / 1e6)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_kind": kind, "traffic": None, "kernel": "pa_prefill (mma.sync bf16)",
+                     "peak_kind": kind, "traffic": None, "kernel": "pa_prefill (%s bf16)" % (
+                         "mma.sync" if args.prefill_kernel == "mma" else "tcgen05"),
                      "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_ms},
         "e2e": {"value": world * T * E / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int((q_h.nbytes + k_h.nbytes + v_h.nbytes)), "d2h_bytes_per_step": int(q_h.nbytes),

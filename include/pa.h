@@ -277,18 +277,28 @@ PA_API int pa_append_decode(const pa_bf16* q, const pa_bf16* k, const pa_bf16* v
  * aligned, its status word as for pa_decode (a block id outside the pool, or
  * L < Tq or L past the table: the sequence's rows are left unwritten and
  * pa_decode_status reports it).  head_dim 64 or 128.
- * Errors: PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA.
+ * kernel: PA_PREFILL_AUTO (= PA_PREFILL_TCGEN05), PA_PREFILL_TCGEN05 (128-row
+ * tiles on the fifth-generation tensor cores, accumulators in tensor memory) or
+ * PA_PREFILL_MMA (64-row tiles on warp-level mma.sync); both compute the same
+ * operation, with fp32 accumulation in a different order.
+ * Errors: PA_ERR_INVALID (also an unknown kernel), PA_ERR_UNSUPPORTED,
+ * PA_ERR_WORKSPACE, PA_ERR_CUDA.
  */
+#define PA_PREFILL_AUTO     0
+#define PA_PREFILL_TCGEN05  1
+#define PA_PREFILL_MMA      2
 PA_API int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
                       const int32_t* block_tables, const int32_t* cu_seqlens_q,
                       const int32_t* context_lens, int32_t num_seqs, int32_t max_q_len, float scale,
                       pa_bf16* out, void* workspace, size_t workspace_bytes,
-                      const pa_cache_desc* desc, void* stream);
+                      const pa_cache_desc* desc, int32_t kernel, void* stream);
 
 /*
  * Synchronises `stream`, reads and clears the workspace's device status word.
- * Returns PA_OK, PA_ERR_BAD_BLOCK, PA_ERR_BAD_LENGTH or PA_ERR_TIMEOUT (the
- * first set, in that order), or PA_ERR_CUDA if the read fails.
+ * Returns PA_OK, PA_ERR_BAD_BLOCK, PA_ERR_BAD_LENGTH, PA_ERR_TIMEOUT or
+ * PA_ERR_UNSUPPORTED (a tensor-core kernel found its shared memory off the
+ * 1024-byte boundary its swizzled tiles need, and wrote nothing) -- the first
+ * set, in that order -- or PA_ERR_CUDA if the read fails.
  */
 PA_API int pa_decode_status(void* workspace, size_t workspace_bytes, void* stream);
 

@@ -126,7 +126,7 @@ lib.pa_bm_append_token_ids.restype = ctypes.c_int
 lib.pa_bm_num_cached_blocks.argtypes = [_vp]
 lib.pa_bm_num_cached_blocks.restype = _i32
 lib.pa_copy_blocks.argtypes = [_vp, _vp, _vp, _i32, _DESC, _vp]
-lib.pa_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _vp, _sz, _DESC, _vp]
+lib.pa_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _vp, _sz, _DESC, _i32, _vp]
 lib.pa_prefill.restype = ctypes.c_int
 lib.pa_append_kv_e4m3.argtypes = [_vp, _vp, _vp, _i32, ctypes.c_float, ctypes.c_float, _vp, _vp, _DESC, _vp]
 lib.pa_append_kv_e4m3.restype = ctypes.c_int
@@ -234,16 +234,24 @@ def pa_copy_blocks(k_cache, v_cache, copies, desc: CacheDesc, stream=None) -> No
                               _stream(stream)), "pa_copy_blocks")
 
 
+PA_PREFILL_AUTO, PA_PREFILL_TCGEN05, PA_PREFILL_MMA = 0, 1, 2
+_PREFILL_KERNELS = {"auto": PA_PREFILL_AUTO, "tcgen05": PA_PREFILL_TCGEN05, "mma": PA_PREFILL_MMA}
+
+
 def pa_prefill(q, k_cache, v_cache, block_tables, cu_seqlens_q, context_lens, max_q_len: int, scale: float,
-               out, workspace, desc: CacheDesc, stream=None) -> None:
-    """Causal attention of each sequence's last Tq tokens over its paged cache."""
+               out, workspace, desc: CacheDesc, stream=None, kernel: str = "auto") -> None:
+    """Causal attention of each sequence's last Tq tokens over its paged cache.
+
+    kernel: "auto" (= "tcgen05"), "tcgen05" or "mma" (the warp-level mma.sync kernel)."""
     n = int(context_lens.shape[0])
+    if kernel not in _PREFILL_KERNELS:
+        raise ValueError("pa_prefill: kernel must be one of %s" % sorted(_PREFILL_KERNELS))
     _check(lib.pa_prefill(_dev(q, "bfloat16", "q"), _cache(k_cache, desc, "k_cache"),
                           _cache(v_cache, desc, "v_cache"), _dev(block_tables, "int32", "block_tables"),
                           _dev(cu_seqlens_q, "int32", "cu_seqlens_q"), _dev(context_lens, "int32", "context_lens"),
                           n, int(max_q_len), float(scale), _dev(out, "bfloat16", "out"),
                           _dev(workspace, "uint8", "workspace"), int(workspace.numel()), ctypes.byref(desc),
-                          _stream(stream)), "pa_prefill")
+                          _PREFILL_KERNELS[kernel], _stream(stream)), "pa_prefill")
 
 
 def pa_decode_workspace_size(num_seqs: int, max_context_len: int, desc: CacheDesc,

@@ -230,10 +230,12 @@ extern "C" int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf1
                           const int32_t* block_tables, const int32_t* cu_seqlens_q,
                           const int32_t* context_lens, int32_t num_seqs, int32_t max_q_len, float scale,
                           pa_bf16* out, void* workspace, size_t workspace_bytes,
-                          const pa_cache_desc* desc, void* stream) {
+                          const pa_cache_desc* desc, int32_t kernel, void* stream) {
     int rc = check_desc(desc);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || num_seqs > 65535 || max_q_len < 0 || !(scale > 0.f) || !(scale < INFINITY))
+        return PA_ERR_INVALID;
+    if (kernel != PA_PREFILL_AUTO && kernel != PA_PREFILL_TCGEN05 && kernel != PA_PREFILL_MMA)
         return PA_ERR_INVALID;
     if (desc->head_dim != 64 && desc->head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (desc->num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
@@ -265,7 +267,8 @@ extern "C" int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf1
     p.group = desc->num_q_heads / desc->num_kv_heads;
     p.max_blocks_per_seq = desc->max_blocks_per_seq;
     p.scale_log2 = scale * 1.4426950408889634f;
-    const cudaError_t e = launch_prefill(p, max_q_len, (cudaStream_t)stream);
+    const cudaError_t e = kernel == PA_PREFILL_MMA ? launch_prefill(p, max_q_len, (cudaStream_t)stream)
+                                                   : launch_prefill_tc(p, max_q_len, (cudaStream_t)stream);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -456,5 +459,6 @@ extern "C" int pa_decode_status(void* workspace, size_t workspace_bytes, void* s
     if (word & kStatusBadBlock) return PA_ERR_BAD_BLOCK;
     if (word & kStatusBadLength) return PA_ERR_BAD_LENGTH;
     if (word & kStatusTimeout) return PA_ERR_TIMEOUT;
+    if (word & kStatusSmemAlign) return PA_ERR_UNSUPPORTED;
     return PA_OK;
 }

@@ -14,6 +14,7 @@ enum : int32_t {
     kStatusBadBlock = 1,
     kStatusBadLength = 2,
     kStatusTimeout = 4,
+    kStatusSmemAlign = 8,   // shared memory off the 1024-byte boundary a swizzled operand needs
 };
 
 // Everything a decode kernel reads; passed by value as the kernel parameter.
@@ -82,6 +83,7 @@ struct PrefillParams {
     float scale_log2;
 };
 cudaError_t launch_prefill(const PrefillParams& p, int max_q_len, cudaStream_t stream);
+cudaError_t launch_prefill_tc(const PrefillParams& p, int max_q_len, cudaStream_t stream);
 
 constexpr size_t kWorkspaceAlign = 256;
 

@@ -1,0 +1,323 @@
+// Paged (chunked) prefill attention on the fifth-generation tensor cores.
+//
+// Same operation as prefill.cu: sequence b holds context_lens[b] = L tokens after this
+// step's append, its last Tq = cu_q[b+1] - cu_q[b] tokens are the queries (positions
+// L-Tq .. L-1), and the query at position p attends to cache tokens 0..p (Nano-vLLM
+// page, section "Prefill vs Decode"; causal mask: Tiny-vLLM summary page, section
+// "고성능 추론을 위한 고급 최적화 기법").
+//
+// One CTA of 128 threads per (128 query rows, kv head, sequence); a row is a (query
+// token, query head of the kv head's group) pair and thread i owns row i, which is
+// tensor-memory lane i.  Per 64-key tile t:
+//   S_t = Q K_t^T   tcgen05.mma, M=128 N=64, Q and K_t K-major in shared memory,
+//                   fp32 S_t in tensor memory;
+//   softmax         each thread loads its row of S_t, masks it causally, updates its
+//                   running max and sum in the log2 domain, and writes P_t (bf16) as a
+//                   K-major A operand into shared memory;
+//   O_t = P_t V_t   tcgen05.mma, M=128 N=D, V_t read MN-major straight from its
+//                   [key][dim] tile; each thread folds its row of O_t into fp32
+//                   registers, O = alpha O + O_t.
+// One thread issues P_t V_t and Q K_{t+1} together, so S_{t+1} is computed while the
+// rows of O_t are folded in.  K and V tiles are gathered through the block table with
+// 16-byte cp.async copies into 128-byte-swizzled tiles, two buffers each: K_{t+2} is
+// requested once S_t is done, V_{t+2} once O_t is done.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+#include "pa_ptx.cuh"
+#include "pa_umma.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int kTcRows = 128;     // query rows per CTA (tensor-memory lanes)
+constexpr int kTcKeys = 64;      // keys per tile
+constexpr int kTcThreads = 128;
+
+template <int D>
+struct TcCfg {
+    static constexpr int kQBytes = kTcRows * D * 2;
+    static constexpr int kKVBytes = kTcKeys * D * 2;       // one K (or V) tile
+    static constexpr int kPBytes = kTcRows * kTcKeys * 2;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;           // 2 buffers
+    static constexpr int kOffV = kOffK + 2 * kKVBytes;      // 2 buffers
+    static constexpr int kOffP = kOffV + 2 * kKVBytes;
+    static constexpr int kOffBar = kOffP + kPBytes;         // 2 mbarriers, tensor-memory address
+    static constexpr int kSmem = kOffBar + 32;
+    static constexpr int kColS = 0;                         // S: 64 fp32 columns
+    static constexpr int kColO = 64;                        // O_t: D fp32 columns
+    static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;
+    static constexpr int kMinBlocks = D == 64 ? 3 : 2;      // by shared memory and tensor memory
+};
+
+// Byte offset of (row, 16-byte chunk c) in a tile of `rows` rows of bf16 stored as
+// 128-byte-swizzled atoms: atom c / 8 holds 128 bytes of every row, rows at 128 bytes,
+// chunk (c % 8) XOR (row % 8).  This is the canonical K-major layout of a tcgen05
+// operand (and the MN-major one when the rows run along K, as for V).
+template <int ROWS>
+__device__ __forceinline__ uint32_t sw128(int row, int c) {
+    return (uint32_t)((c >> 3) * (ROWS * 128) + row * 128 + ((((c & 7) ^ (row & 7))) << 4));
+}
+
+__device__ __forceinline__ void cp_async16_tc(uint32_t dst, const void* src, bool live) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(live ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_tc() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_tc() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kMinBlocks) prefill_tc_kernel(const PrefillParams p) {
+    using C = TcCfg<D>;
+    constexpr int kCh = D / 8;                               // 16-byte chunks per row
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t s_q = s_base + C::kOffQ, s_k = s_base + C::kOffK, s_v = s_base + C::kOffV;
+    const uint32_t s_p = s_base + C::kOffP;
+    const uint32_t bar_s = s_base + C::kOffBar, bar_o = bar_s + 8, s_tmem = bar_s + 16;
+
+    const int b = blockIdx.z, kvh = blockIdx.y;
+    const int G = p.group, Hq = p.num_q_heads, Hkv = p.num_kv_heads, Bs = p.block_size;
+    const int q0 = p.cu_q[b], Tq = p.cu_q[b + 1] - q0;
+    const int L = p.context_lens[b];
+    const int cap = p.max_blocks_per_seq * Bs;
+    if (Tq <= 0) return;
+    if (L < Tq || L > cap) {                                 // fewer tokens than queries, or past the table
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) raise_status(p.status, kStatusBadLength);
+        return;
+    }
+    if (s_base & 1023u) {                                    // the swizzle needs 1024-byte-aligned tiles
+        if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
+        return;
+    }
+    // the last row tiles of a chunk attend to the most keys: they take the first CTAs
+    const int rows = Tq * G, ntile = (rows + kTcRows - 1) / kTcRows;
+    const int tile = ntile - 1 - (int)blockIdx.x;
+    if (tile < 0) return;
+    const int r0 = tile * kTcRows;
+    const int* table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+    const int tid = threadIdx.x, warp = tid >> 5;
+
+    const int last_tok = min(rows - 1, r0 + kTcRows - 1) / G;
+    const int kend = L - Tq + last_tok + 1;                  // keys needed: up to the last row's position
+    const int ntiles = (kend + kTcKeys - 1) / kTcKeys;
+    const int pos_first = L - Tq + r0 / G;                   // smallest position in the tile
+
+    // ---- tensor memory and barriers ----
+    if (warp == 0) {
+        tmem_alloc(s_tmem, C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    uint32_t tmem;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(tmem) : "r"(s_tmem) : "memory");
+    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's 32 lanes
+
+    // ---- loads: Q (rows past the chunk are zeros), K and V tiles through the block table ----
+    for (int i = tid; i < kTcRows * kCh; i += kTcThreads) {
+        const int row = i / kCh, c = i - row * kCh, R = r0 + row;
+        const bool live = R < rows;
+        const int tok = live ? R / G : 0, g = live ? R - tok * G : 0;
+        const uint16_t* src = p.q + (((size_t)(q0 + tok) * Hq + (size_t)kvh * G + g) * D + c * 8);
+        cp_async16_tc(s_q + sw128<kTcRows>(row, c), src, live);
+    }
+    auto load_tile = [&](const uint16_t* cache, uint32_t dst, int t) {
+        const int k0 = t * kTcKeys;
+        for (int i = tid; i < kTcKeys * kCh; i += kTcThreads) {
+            const int j = i / kCh, c = i - j * kCh, kp = k0 + j;
+            bool live = kp < L;
+            size_t off = 0;
+            if (live) {
+                const int blk = __ldg(table + kp / Bs);
+                if (blk < 0 || blk >= p.num_blocks) {
+                    raise_status(p.status, kStatusBadBlock);
+                    live = false;
+                } else {
+                    off = (((size_t)blk * Hkv + kvh) * Bs + kp % Bs) * D + c * 8;
+                }
+            }
+            cp_async16_tc(dst + sw128<kTcKeys>(j, c), cache + off, live);
+        }
+    };
+    // groups in issue order: {Q, K0, V0}, K1, V1, then K_{t+2} and V_{t+2} per tile t
+    // (empty groups past the last tile keep the count uniform)
+    load_tile(p.k_cache, s_k, 0);
+    load_tile(p.v_cache, s_v, 0);
+    cp_async_commit_tc();
+    if (ntiles > 1) load_tile(p.k_cache, s_k + C::kKVBytes, 1);
+    cp_async_commit_tc();
+    if (ntiles > 1) load_tile(p.v_cache, s_v + C::kKVBytes, 1);
+    cp_async_commit_tc();
+
+    constexpr uint32_t kIdescS = umma_idesc_bf16(kTcRows, kTcKeys, false);
+    constexpr uint32_t kIdescO = umma_idesc_bf16(kTcRows, D, true);
+    auto issue_s = [&](int t) {                              // S = Q K_t^T over D / 16 K steps
+        const uint32_t kt = s_k + (t & 1) * C::kKVBytes;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t a = umma_desc_sw128(s_q + (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd = umma_desc_sw128(kt + (ks >> 2) * (kTcKeys * 128) + (ks & 3) * 32, 16, 1024);
+            umma_bf16_ss(tmem + C::kColS, a, bd, kIdescS, ks > 0);
+        }
+        umma_commit(bar_s);
+    };
+    auto issue_o = [&](int t) {                              // O_t = P V_t over 4 K steps of 16 keys
+        const uint32_t vt = s_v + (t & 1) * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+            const uint64_t a = umma_desc_sw128(s_p + kk * 32, 16, 1024);
+            // MN-major B: 8-key groups 1024 bytes apart, 64-dim atoms one tile of keys apart
+            const uint64_t bd = umma_desc_sw128(vt + kk * 16 * 128, kTcKeys * 128, 1024);
+            umma_bf16_ss(tmem + C::kColO, a, bd, kIdescO, kk > 0);
+        }
+        umma_commit(bar_o);
+    };
+
+    cp_async_wait_tc<2>();                                   // Q, K0, V0
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+        tc_fence_after_sync();
+        issue_s(0);
+    }
+
+    const int R = r0 + tid;
+    const int pos = R < rows ? L - Tq + R / G : L - 1;      // padded rows: computed, not written
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[D];
+#pragma unroll
+    for (int j = 0; j < D; ++j) o[j] = 0.f;
+    bool failed = false;
+
+    for (int t = 0; t < ntiles; ++t) {
+        // ---- S_t ----
+        if (!mbar_wait(bar_s, (uint32_t)(t & 1), p.status)) failed = true;
+        tc_fence_after_sync();
+        if (t + 2 < ntiles) load_tile(p.k_cache, s_k + (t & 1) * C::kKVBytes, t + 2);   // K_t is consumed
+        cp_async_commit_tc();
+        uint32_t sr[64];
+        tmem_ld64(t_lane + C::kColS, sr);
+        const int k0 = t * kTcKeys;
+        float mx = -INFINITY;
+        if (k0 + kTcKeys - 1 > pos_first) {                  // a tile on the diagonal: mask
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const float v = k0 + j <= pos ? __uint_as_float(sr[j]) : -INFINITY;
+                sr[j] = __float_as_uint(v);
+                mx = fmaxf(mx, v);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(sr[j]));
+        }
+        // key 0 is in every row's range, so m_new is finite from the first tile on
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const float alpha = fast_exp2(m_run - m_new);
+        m_run = m_new;
+        float rsum = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * j]), sl2, -m_new));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * j + 1]), sl2, -m_new));
+            rsum += p0 + p1;
+            pk[j] = pack_bf16x2(p0, p1);
+        }
+        l_run = l_run * alpha + rsum;
+        const uint32_t prow = s_p + tid * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + ((c ^ (tid & 7)) << 4)),
+                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                         : "memory");
+        // ---- P_t V_t and Q K_{t+1}: K_{t+1} and V_{t+1} must have landed ----
+        cp_async_wait_tc<1>();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before_sync();
+        if (__syncthreads_or(failed)) break;
+        if (tid == 0) {
+            tc_fence_after_sync();
+            issue_o(t);
+            if (t + 1 < ntiles) issue_s(t + 1);
+        }
+        // ---- O = alpha O + O_t ----
+        if (!mbar_wait(bar_o, (uint32_t)(t & 1), p.status)) failed = true;
+        tc_fence_after_sync();
+        if (t + 2 < ntiles) load_tile(p.v_cache, s_v + (t & 1) * C::kKVBytes, t + 2);   // V_t is consumed
+        cp_async_commit_tc();
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+            uint32_t orow[64];
+            tmem_ld64(t_lane + C::kColO + h * 64, orow);
+#pragma unroll
+            for (int j = 0; j < 64; ++j) o[h * 64 + j] = fmaf(o[h * 64 + j], alpha, __uint_as_float(orow[j]));
+        }
+        tc_fence_before_sync();
+    }
+    cp_async_wait_tc<0>();
+    tc_fence_before_sync();
+    const bool aborted = __syncthreads_or(failed);
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+    if (aborted || R >= rows) return;
+    // ---- out = O / l ----
+    const int tok = R / G, g = R - tok * G;
+    const float inv = 1.f / l_run;
+    uint16_t* out = p.out + ((size_t)(q0 + tok) * Hq + (size_t)kvh * G + g) * D;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        uint4 w;
+        w.x = pack_bf16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
+        w.y = pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+        w.z = pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+        w.w = pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+        *reinterpret_cast<uint4*>(out + 8 * c) = w;
+    }
+}
+
+template <int D>
+cudaError_t launch_pf_tc(const PrefillParams& p, int max_q_len, cudaStream_t stream) {
+    constexpr size_t smem = TcCfg<D>::kSmem;
+    static std::atomic<uint64_t> attr_set{0};               // one bit per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!(attr_set.load(std::memory_order_acquire) & (1ull << dev))) {
+        const cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(1ull << dev, std::memory_order_acq_rel);
+    }
+    const int tiles = (max_q_len * p.group + kTcRows - 1) / kTcRows;
+    if (tiles <= 0) return cudaSuccess;
+    dim3 grid((unsigned)tiles, (unsigned)p.num_kv_heads, (unsigned)p.num_seqs);
+    prefill_tc_kernel<D><<<grid, kTcThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const PrefillParams& p, int max_q_len, cudaStream_t stream) {
+    if (p.head_dim == 64) return launch_pf_tc<64>(p, max_q_len, stream);
+    if (p.head_dim == 128) return launch_pf_tc<128>(p, max_q_len, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pa

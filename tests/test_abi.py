@@ -133,9 +133,13 @@ def test_prefill_rejects_bad_arguments_without_a_gpu():
     lib = binding.lib
     fake = ctypes.c_void_p(0x10000)
     d = _desc()
-    call = lambda n, mq, scale, dd, ws=fake, wsb=256: lib.pa_prefill(
-        fake, fake, fake, fake, fake, fake, n, mq, ctypes.c_float(scale), fake, ws, wsb, ctypes.byref(dd), None)
+    call = lambda n, mq, scale, dd, ws=fake, wsb=256, kernel=0: lib.pa_prefill(
+        fake, fake, fake, fake, fake, fake, n, mq, ctypes.c_float(scale), fake, ws, wsb, ctypes.byref(dd), kernel,
+        None)
     assert call(-1, 4, 0.1, d) == -1
+    assert call(2, 4, 0.1, d, kernel=3) == -1            # unknown kernel
+    assert call(2, 4, 0.1, d, kernel=-1) == -1
+    assert call(0, 4, 0.1, d, kernel=pa.PA_PREFILL_MMA) == 0
     assert call(2, -1, 0.1, d) == -1
     assert call(2, 4, 0.0, d) == -1                      # scale must be > 0
     assert call(2, 4, 0.1, _desc(head_dim=96)) == -2

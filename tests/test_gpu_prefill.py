@@ -1,9 +1,10 @@
 """Paged (chunked) prefill through the C ABI against the fp64 oracle (needs a B200).
 
-Outputs within 1e-2 + 1e-2 * |oracle|; cases: whole prompts (Tq = L), chunks after a
-cached prefix (Tq < L), one-token chunks, lengths off the 64-key and 64-row tiles,
-GQA groups 1..16, head dims 64 and 128, block sizes 8..256; errors reported through
-the status word without a fault.
+Both kernels (tcgen05 with tensor-memory accumulators, and warp-level mma.sync), each
+within 1e-2 + 1e-2 * |oracle|; cases: whole prompts (Tq = L), chunks after a cached
+prefix (Tq < L), one-token chunks, lengths off the 64-key and 64/128-row tiles, GQA
+groups 1..16, head dims 64 and 128, block sizes 8..256; errors reported through the
+status word without a fault.
 """
 import numpy as np
 import pytest
@@ -24,7 +25,10 @@ def h():
     return gpu_harness
 
 
-def _run(h, seed, lens, q_lens, **kw):
+KERNELS = ["tcgen05", "mma"]
+
+
+def _run(h, seed, lens, q_lens, kernel="auto", **kw):
     b = wl.small_batch(seed, lens, **kw)
     rng = np.random.default_rng(seed)
     cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
@@ -35,7 +39,7 @@ def _run(h, seed, lens, q_lens, **kw):
     ws = torch.zeros(256, dtype=torch.uint8, device=h.DEV)
     pa.pa_prefill(h.to_dev(q), h.to_dev(b.k_cache), h.to_dev(b.v_cache), torch.from_numpy(b.block_tables).to(h.DEV),
                   torch.from_numpy(cu).to(h.DEV), torch.from_numpy(b.context_lens).to(h.DEV), max(q_lens),
-                  b.scale, out, ws, desc)
+                  b.scale, out, ws, desc, kernel=kernel)
     torch.cuda.synchronize()
     assert pa.pa_decode_status(ws) == 0
     ref = oracle.paged_prefill(q, b.k_cache, b.v_cache, b.block_tables, cu, b.context_lens, b.scale)
@@ -49,19 +53,31 @@ SHAPES = [(32, 8, 64, 16), (8, 8, 64, 8), (16, 1, 128, 16), (64, 8, 128, 32), (6
           (24, 8, 64, 16)]
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "Hq%d-Hkv%d-D%d-Bs%d" % s)
-def test_prefill_shapes(h, shape):
+def test_prefill_shapes(h, shape, kernel):
     Hq, Hkv, D, Bs = shape
     lens = [1, 64, 65, 200, 333, 130]
     q_lens = [1, 64, 17, 200, 40, 1]                   # whole prompts, chunks, single tokens
-    _run(h, 7000 + Hq + D + Bs, lens, q_lens, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, block_size=Bs)
+    _run(h, 7000 + Hq + D + Bs, lens, q_lens, kernel=kernel, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+         block_size=Bs)
 
 
-def test_prefill_llama_1b_prompt_and_chunk(h):
-    _run(h, 7100, [2048, 1500], [2048, 700], num_q_heads=32, num_kv_heads=8, head_dim=64, block_size=16)
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_llama_1b_prompt_and_chunk(h, kernel):
+    _run(h, 7100, [2048, 1500], [2048, 700], kernel=kernel, num_q_heads=32, num_kv_heads=8, head_dim=64,
+         block_size=16)
 
 
-def test_prefill_reports_bad_lengths_and_blocks(h):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_head_dim_128_long_chunk(h, kernel):
+    # several 128-row tiles and 64-key tiles with ragged ends, G = 4, blocks of 32
+    _run(h, 7150, [1000, 777], [600, 777], kernel=kernel, num_q_heads=16, num_kv_heads=4, head_dim=128,
+         block_size=32)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_reports_bad_lengths_and_blocks(h, kernel):
     b = wl.small_batch(7200, [40, 20], num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16)
     desc = h.desc_of(b)
     q = torch.zeros((10, 4, 64), dtype=torch.bfloat16, device=h.DEV)
@@ -71,12 +87,12 @@ def test_prefill_reports_bad_lengths_and_blocks(h):
     lens = torch.tensor([40, 3], dtype=torch.int32, device=h.DEV)      # second: fewer tokens than queries
     kc, vc = h.to_dev(b.k_cache), h.to_dev(b.v_cache)
     tables = torch.from_numpy(b.block_tables).to(h.DEV)
-    pa.pa_prefill(q, kc, vc, tables, cu, lens, 5, b.scale, out, ws, desc)
+    pa.pa_prefill(q, kc, vc, tables, cu, lens, 5, b.scale, out, ws, desc, kernel=kernel)
     torch.cuda.synchronize()
     assert pa.pa_decode_status(ws) == -8
     bad = b.block_tables.copy()
     bad[0, 1] = b.num_blocks + 5
     lens = torch.tensor([40, 20], dtype=torch.int32, device=h.DEV)
-    pa.pa_prefill(q, kc, vc, torch.from_numpy(bad).to(h.DEV), cu, lens, 5, b.scale, out, ws, desc)
+    pa.pa_prefill(q, kc, vc, torch.from_numpy(bad).to(h.DEV), cu, lens, 5, b.scale, out, ws, desc, kernel=kernel)
     torch.cuda.synchronize()
     assert pa.pa_decode_status(ws) == -7
