@@ -28,8 +28,10 @@ def h():
 KERNELS = ["tcgen05", "mma"]
 
 
-def _run(h, seed, lens, q_lens, kernel="auto", **kw):
+def _run(h, seed, lens, q_lens, kernel="auto", mutate=None, **kw):
     b = wl.small_batch(seed, lens, **kw)
+    if mutate is not None:
+        mutate(b)
     rng = np.random.default_rng(seed)
     cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
     q = (rng.standard_normal((int(cu[-1]), b.num_q_heads, b.head_dim)).astype(np.float32)
@@ -49,8 +51,10 @@ def _run(h, seed, lens, q_lens, kernel="auto", **kw):
     assert ok, "prefill outside tolerance by %g" % ex
 
 
+# block sizes 8..256 that tile 64 keys (copied by TMA in the tcgen05 kernel) and 24, 4
+# that do not (gathered with cp.async)
 SHAPES = [(32, 8, 64, 16), (8, 8, 64, 8), (16, 1, 128, 16), (64, 8, 128, 32), (6, 3, 64, 256), (2, 2, 128, 64),
-          (24, 8, 64, 16)]
+          (24, 8, 64, 16), (8, 2, 64, 24), (4, 4, 128, 4), (8, 1, 64, 128)]
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
@@ -74,6 +78,28 @@ def test_prefill_head_dim_128_long_chunk(h, kernel):
     # several 128-row tiles and 64-key tiles with ragged ends, G = 4, blocks of 32
     _run(h, 7150, [1000, 777], [600, 777], kernel=kernel, num_q_heads=16, num_kv_heads=4, head_dim=128,
          block_size=32)
+
+
+def _poison_unused_rows(b):
+    """NaN (bf16 0x7FC0) in every pool row no sequence holds: free blocks and the tail of
+    each sequence's last block.  The attention must not read them into the output."""
+    used = np.zeros(b.k_cache.shape[0], dtype=bool)
+    for s, L in enumerate(b.context_lens):
+        nb = (int(L) + b.block_size - 1) // b.block_size
+        used[b.block_tables[s, :nb]] = True
+    for cache in (b.k_cache, b.v_cache):
+        cache[~used] = 0x7FC0
+        for s, L in enumerate(b.context_lens):
+            L = int(L)
+            if L % b.block_size:
+                cache[b.block_tables[s, (L - 1) // b.block_size], :, L % b.block_size:, :] = 0x7FC0
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("Bs", [16, 24, 128])
+def test_prefill_ignores_pool_rows_past_each_sequence(h, kernel, Bs):
+    _run(h, 7300 + Bs, [37, 130, 64, 201], [37, 9, 64, 100], kernel=kernel, mutate=_poison_unused_rows,
+         num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=Bs)
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
