@@ -20,9 +20,11 @@
 // One thread issues P_t V_t and Q K_{t+1} together, so S_{t+1} is computed while the
 // rows of O_t are folded in.  K and V tiles have two buffers each: K_{t+2} is requested
 // once S_t is done, V_{t+2} once O_t is done, from block ids read a tile ahead.  When
-// the block size tiles 64 keys (8, 16, 32, 64 or a multiple of 64) warp 0 moves them
-// with TMA, one box of 64 dims x min(Bs, 64) tokens per block and 64-dim atom, swizzled
-// by the copy engine; otherwise every thread gathers them with 16-byte cp.async copies.
+// the block size tiles 64 keys (8, 16, 32, 64 or a multiple of 64) they move by TMA, one
+// box of 64 dims x min(Bs, 64) tokens per block and 64-dim atom, swizzled by the copy
+// engine: warp 1 issues the K boxes and warp 2 the V boxes, so that warp 0, whose
+// thread 0 issues the MMAs, carries no copy work; otherwise every thread gathers them
+// with 16-byte cp.async copies.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -151,14 +153,15 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kMinBlocks)
     constexpr int kKPT = kTcKeys / kJStep;                   // keys per thread per tile: 4 or 8
     const int j0 = tid / kCh, c_ld = tid - (tid / kCh) * kCh;
     int ids[kKPT];
-    // TMA: lane i of warp 0 moves slot i of a tile (rb tokens of one block) with one box
-    // per 64-dim atom; slot_id is that block's id for the next tile to request.
+    // TMA: lane i of warp 1 (K) and of warp 2 (V) moves slot i of a tile (rb tokens of one
+    // block) with one box per 64-dim atom; slot_id is that block's id for the next tile to
+    // request.
     const int rb = Bs < kTcKeys ? Bs : kTcKeys, nslot = kTcKeys / rb;
     int slot_id = 0;
     auto fetch_ids = [&](int t) {
         if constexpr (kTma) {
             const int kp = t * kTcKeys + lane * rb;
-            if (warp == 0 && lane < nslot && kp < L) slot_id = __ldg(table + kp / Bs);
+            if ((warp == 1 || warp == 2) && lane < nslot && kp < L) slot_id = __ldg(table + kp / Bs);
         } else {
 #pragma unroll
             for (int k = 0; k < kKPT; ++k) {
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kMinBlocks)
             }
         }
     };
-    auto tma_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int t) {   // warp 0
+    auto tma_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int t) {   // one warp
         const int kp = t * kTcKeys + lane * rb;
         bool valid = lane < nslot && kp < L;
         if (valid && (slot_id < 0 || slot_id >= p.num_blocks)) {
@@ -202,13 +205,13 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kMinBlocks)
         }
     };
     // request K_t into buffer t & 1 (TMA: barrier bar_k[t & 1]; cp.async: one group)
-    // TMA tiles requested and waited for, as thread 0 (lane 0 of the issuing warp) saw them:
-    // on an aborted run it drains the difference before the CTA exits
+    // TMA tiles requested (every thread counts them) and waited for by thread 0: on an
+    // aborted run thread 0 drains the difference before the CTA exits
     int k_req = -1, v_req = -1, k_seen = -1, v_seen = -1;
     auto request_k = [&](int t) {
         if constexpr (kTma) {
             k_req = t;
-            if (warp == 0) tma_tile(&kmap, s_k + (t & 1) * C::kKVBytes, bar_k + 8 * (t & 1), t);
+            if (warp == 1) tma_tile(&kmap, s_k + (t & 1) * C::kKVBytes, bar_k + 8 * (t & 1), t);
         } else {
             load_tile(p.k_cache, s_k + (t & 1) * C::kKVBytes, t);
         }
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kMinBlocks)
     auto request_v = [&](int t) {
         if constexpr (kTma) {
             v_req = t;
-            if (warp == 0) tma_tile(&vmap, s_v + (t & 1) * C::kKVBytes, bar_v + 8 * (t & 1), t);
+            if (warp == 2) tma_tile(&vmap, s_v + (t & 1) * C::kKVBytes, bar_v + 8 * (t & 1), t);
         } else {
             load_tile(p.v_cache, s_v + (t & 1) * C::kKVBytes, t);
         }
