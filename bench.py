@@ -131,7 +131,8 @@ def kv_read_bytes(lens, num_kv_heads, head_dim, elem_bytes=2):
 def kernel_source_hash(kernel_name):
     files = {"tensor": ["decode_stream.cu", "pa_ptx.cuh", "merge.cu"],
              "split": ["decode_tensor.cu", "pa_ptx.cuh", "merge.cu"],
-             "simt": ["decode_simt.cu", "merge.cu"]}[kernel_name]
+             "simt": ["decode_simt.cu", "merge.cu"],
+             "prefill": ["prefill_tc.cu", "pa_umma.cuh", "pa_ptx.cuh"]}[kernel_name]
     files = files + ["pa_device.cuh", "pa_internal.h", "api.cu"]
     h = hashlib.sha256()
     for f in files:
@@ -936,8 +937,9 @@ def run_pf(args, rank, world, dist):
                    "context": lens, "call": "pa_append_kv + pa_prefill",
                    "l2": "working set (%.0f MB of KV) fits L2: prefill is compute-bound" % (2 * b.k_cache.nbytes / 1e6)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_kind": kind, "traffic": None, "kernel": "pa_prefill (%s bf16)" % (
-                         "mma.sync" if args.prefill_kernel == "mma" else "tcgen05"),
+                     "peak_kind": kind,
+                     "traffic": None if args.prefill_kernel == "mma" else profiled_traffic("pf", "prefill"),
+                     "kernel": "pa_prefill (%s bf16)" % ("mma.sync" if args.prefill_kernel == "mma" else "tcgen05"),
                      "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_ms},
         "e2e": {"value": world * T * E / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int((q_h.nbytes + k_h.nbytes + v_h.nbytes)), "d2h_bytes_per_step": int(q_h.nbytes),
