@@ -140,6 +140,10 @@ def test_prefill_rejects_bad_arguments_without_a_gpu():
     assert call(2, 4, 0.1, d, kernel=3) == -1            # unknown kernel
     assert call(2, 4, 0.1, d, kernel=-1) == -1
     assert call(0, 4, 0.1, d, kernel=pa.PA_PREFILL_MMA) == 0
+    # the binding refuses an unknown kernel name before it touches any buffer
+    with pytest.raises(ValueError):
+        pa.pa_prefill(None, None, None, None, None, np.zeros(2, np.int32), 4, 0.1, None, None, d,
+                      kernel="wgmma")
     assert call(2, -1, 0.1, d) == -1
     assert call(2, 4, 0.0, d) == -1                      # scale must be > 0
     assert call(2, 4, 0.1, _desc(head_dim=96)) == -2
