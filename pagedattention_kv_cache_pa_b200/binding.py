@@ -21,7 +21,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "pa.h")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libpa.so is not built (%s); run __graft_entry__.build() or "
-                      "python -m pagedattention_kv_cache_pa_b200._build" % LIB_PATH)
+                      "python pagedattention_kv_cache_pa_b200/_build.py" % LIB_PATH)
 
 lib = ctypes.CDLL(LIB_PATH)
 
