@@ -840,6 +840,28 @@ def prefill_flops(lens, q_lens, num_q_heads, head_dim):
     return f
 
 
+def pf_cpu_baseline(b, q_h, cu, lens, B, seconds):
+    """The oracle's prefill on windows of 64 consecutive queries of the chunks, for about
+    `seconds`.  Visit n takes sequence n % B and window 13 (n // B) mod (chunk / 64) of it, so
+    every sequence steps through its whole chunk and a cut-short run still samples early,
+    middle and late positions evenly."""
+    import oracle
+    windows = PF_NEW // 64
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < max(1.0, seconds):
+        s_ = n % B
+        w = (13 * (n // B)) % windows
+        end = lens[s_] - PF_NEW + 64 * (w + 1)       # the window's queries are the last 64 of `end` tokens
+        qs = q_h[int(cu[s_]) + 64 * w: int(cu[s_]) + 64 * (w + 1)]
+        oracle.paged_prefill(qs, b.k_cache, b.v_cache, b.block_tables[s_:s_ + 1], np.array([0, 64], np.int32),
+                             np.array([end], np.int32), b.scale)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": 64 * n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d windows of 64 query tokens spread evenly over the %d chunks, %.1f s" % (n, B, dt)}
+
+
 def run_pf(args, rank, world, dist):
     """Chunked prefill: a step appends each sequence's new chunk and runs the causal attention."""
     import torch
@@ -947,20 +969,7 @@ def run_pf(args, rank, world, dist):
         "gpu_launches": 2 * K, "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:
-        import oracle
-        t0 = time.perf_counter()
-        n = 0
-        while time.perf_counter() - t0 < max(1.0, args.cpu_seconds) and n < 8:
-            s_ = n % B
-            lo = lens[s_] - 64                        # the chunk's last 64 queries of one sequence
-            qs = q_h[int(cu[s_]) + PF_NEW - 64: int(cu[s_]) + PF_NEW]
-            oracle.paged_prefill(qs, b.k_cache, b.v_cache, b.block_tables[s_:s_ + 1], np.array([0, 64], np.int32),
-                                 np.array([lens[s_]], np.int32), b.scale)
-            n += 1
-        dt = time.perf_counter() - t0
-        res["cpu_baseline"] = {"value": 64 * n / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
-                               "kind": "oracle", "sample": "%d x 64 query tokens at the end of a chunk (the "
-                               "costliest positions), %.1f s" % (n, dt)}
+        res["cpu_baseline"] = pf_cpu_baseline(b, q_h, cu, lens, B, args.cpu_seconds)
     return res
 
 
