@@ -153,6 +153,14 @@ PA_API int pa_rope_append_kv(const pa_bf16* q, pa_bf16* q_out, const pa_bf16* k,
 
 #define PA_FLAG_CHECK     1   /* synchronise after the launch and report device-side errors     */
 #define PA_FLAG_PDL       2   /* early start (programmatic dependent launch), see pa_decode     */
+/* Failure-handling self-test (whole-group tensor kernel only, else PA_ERR_UNSUPPORTED): the
+ * producer warp of the kernel's CTA 0 issues no copy and signals nothing, so that CTA's
+ * consumer warps find their first wait unanswered; their waits give up after 10 ms (instead
+ * of 2 s), raise the timeout bit and the CTA exits with no copy in flight.  The other CTAs run
+ * normally.  The call then reports PA_ERR_TIMEOUT (through PA_FLAG_CHECK or pa_decode_status)
+ * and its output is unspecified; the workspace serves the next call as it is.  For tests of
+ * the error path; never set in normal use. */
+#define PA_FLAG_SELFTEST_STALL 4
 
 #define PA_KV_BF16        0   /* caches hold bf16 values                                         */
 #define PA_KV_E4M3        1   /* caches hold E4M3 codes (uint8), see pa_append_kv_e4m3           */
@@ -189,8 +197,10 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * over the context_lens[b] tokens the table row block_tables[b] reaches,
  * with K_j, V_j the rows of kv head h / (Hq/Hkv).  fp32 accumulation, online
  * softmax, the result rounded to nearest-even bf16.  A sequence with
- * context_lens[b] == 0 outputs zeros.  Long contexts are split across CTAs;
- * the partial states are merged (log-sum-exp) inside the same launch.
+ * context_lens[b] == 0 outputs zeros.  Long contexts are split across CTAs:
+ * each piece leaves an fp32 partial state in the workspace, and a second
+ * kernel, launched by the same call on the same stream, merges them
+ * (log-sum-exp) into out.
  *
  * workspace: caller-owned device buffer of at least
  * pa_decode_workspace_size(...) bytes, 256-byte aligned, ZERO-FILLED BEFORE
@@ -306,6 +316,29 @@ PA_API int pa_decode_status(void* workspace, size_t workspace_bytes, void* strea
 PA_API int32_t pa_decode_max_splits(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc* desc,
                              const pa_decode_options* options);
 
+/*
+ * How pa_decode (and pa_append_decode, pa_decode_noalloc) will partition the work of a call
+ * of this shape on the current device, for callers that size, test or profile around it.
+ *  kernel:       PA_KERNEL_TENSOR for the stream-partitioned whole-group kernel (Hkv a
+ *                multiple of 8), PA_KERNEL_TENSOR_SPLIT or PA_KERNEL_SIMT for the split ones.
+ *  ctas:         stream kernel: CTAs of its persistent grid.  The work is the concatenation,
+ *                over groups of 8 kv heads and then sequences, of 16-token slabs (an empty
+ *                sequence counts one); CTA i of G = min(ctas, slabs S) takes slabs
+ *                [i S / G, (i + 1) S / G).  0 for the split kernels.
+ *  split_tokens: split kernels: tokens per split (split k covers [k C, (k + 1) C)); else 0.
+ *  max_splits:   split kernels: splits per (sequence, kv head) at most; else 1.
+ * Returns PA_OK, or the error the decode call itself would return for these arguments.
+ */
+typedef struct pa_decode_plan_info {
+    int32_t kernel;
+    int32_t ctas;
+    int32_t split_tokens;
+    int32_t max_splits;
+} pa_decode_plan_info;
+
+PA_API int pa_decode_describe(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc* desc,
+                              const pa_decode_options* options, pa_decode_plan_info* out);
+
 /* ---- paged decode without allocation ------------------------------------------------------ */
 /*
  * (The pages have no counterpart: this is a deployment convenience.)
@@ -327,6 +360,15 @@ PA_API int32_t pa_decode_max_splits(int32_t num_seqs, int32_t max_context_len, c
  *  - Every call shares the one array and it keeps the previous call's
  *    contents (the words that must start at zero are cleared on `stream`), so
  *    calls that may overlap on the GPU race: serialise them (one stream).
+ *  - Device-side errors (a block id outside the pool, a clipped length, a
+ *    timed-out wait) are reported only with PA_FLAG_CHECK, which synchronises
+ *    `stream` and returns them; without it they are dropped, because the next
+ *    call clears the array's status word before it runs.
+ *  - The clearing is a memset on `stream` between the previous kernel and the
+ *    decode, so PA_FLAG_PDL gives no early start here.
+ *  - The cached address is that of the device's primary context (the one the
+ *    CUDA runtime uses); do not call this from another driver-API context on the
+ *    same device.
  */
 #define PA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 

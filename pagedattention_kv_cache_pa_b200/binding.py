@@ -32,6 +32,7 @@ STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ER
 PA_KERNEL_AUTO, PA_KERNEL_SIMT, PA_KERNEL_TENSOR, PA_KERNEL_TENSOR_SPLIT = 0, 1, 2, 3
 PA_FLAG_CHECK = 1
 PA_FLAG_PDL = 2
+PA_FLAG_SELFTEST_STALL = 4
 PA_KV_BF16 = 0
 PA_KV_E4M3 = 1
 
@@ -58,6 +59,11 @@ class DecodeOptions(ctypes.Structure):
                 ("flags", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
                 ("rope_theta", ctypes.c_float), ("kv_dtype", ctypes.c_int32),
                 ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
+
+
+class DecodePlanInfo(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("ctas", ctypes.c_int32),
+                ("split_tokens", ctypes.c_int32), ("max_splits", ctypes.c_int32)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -91,6 +97,8 @@ lib.pa_decode_status.argtypes = [_vp, _sz, _vp]
 lib.pa_decode_status.restype = ctypes.c_int
 lib.pa_decode_max_splits.argtypes = [_i32, _i32, _DESC, _OPTS]
 lib.pa_decode_max_splits.restype = _i32
+lib.pa_decode_describe.argtypes = [_i32, _i32, _DESC, _OPTS, ctypes.POINTER(DecodePlanInfo)]
+lib.pa_decode_describe.restype = ctypes.c_int
 lib.pa_slot_mapping.argtypes = [_vp, _i32, _vp, _i32, _i32, _vp]
 lib.pa_slot_mapping.restype = ctypes.c_int
 lib.pa_bm_create.argtypes = [_i32, _i32, _i32, _i32, _vp, _i32, ctypes.POINTER(_vp)]
@@ -267,6 +275,17 @@ def pa_decode_max_splits(num_seqs: int, max_context_len: int, desc: CacheDesc,
                          options: DecodeOptions | None = None) -> int:
     return int(lib.pa_decode_max_splits(int(num_seqs), int(max_context_len), ctypes.byref(desc),
                                         ctypes.byref(options) if options is not None else None))
+
+
+def pa_decode_describe(num_seqs: int, max_context_len: int, desc: CacheDesc,
+                       options: DecodeOptions | None = None) -> DecodePlanInfo:
+    """The decode kernel and partition a call of this shape runs (kernel, ctas, split_tokens,
+    max_splits)."""
+    info = DecodePlanInfo()
+    _check(lib.pa_decode_describe(int(num_seqs), int(max_context_len), ctypes.byref(desc),
+                                  ctypes.byref(options) if options is not None else None,
+                                  ctypes.byref(info)), "pa_decode_describe")
+    return info
 
 
 def pa_decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,

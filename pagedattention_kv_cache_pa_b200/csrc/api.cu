@@ -319,6 +319,23 @@ extern "C" int32_t pa_decode_max_splits(int32_t num_seqs, int32_t max_context_le
     return plan.max_splits;
 }
 
+extern "C" int pa_decode_describe(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc* desc,
+                                  const pa_decode_options* options, pa_decode_plan_info* out) {
+    if (!out) return PA_ERR_INVALID;
+    int rc = check_decode_shape(num_seqs, max_context_len, desc);
+    if (rc != PA_OK) return rc;
+    DecodePlan plan;
+    rc = make_decode_plan(num_seqs, max_context_len, *desc, options, &plan);
+    if (rc != PA_OK) return rc;
+    out->kernel = plan.kernel == DecodeKernel::kStream  ? PA_KERNEL_TENSOR
+                  : plan.kernel == DecodeKernel::kSplit ? PA_KERNEL_TENSOR_SPLIT
+                                                        : PA_KERNEL_SIMT;
+    out->ctas = plan.kernel == DecodeKernel::kStream ? plan.grid : 0;
+    out->split_tokens = plan.kernel == DecodeKernel::kStream ? 0 : plan.split_tokens;
+    out->max_splits = plan.max_splits;
+    return PA_OK;
+}
+
 // Shared by pa_decode_ex (k_new == v_new == null) and pa_append_decode.
 static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_new,
                        const pa_bf16* k_cache, const pa_bf16* v_cache, const int32_t* block_tables,
@@ -328,7 +345,7 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     int rc = check_decode_shape(num_seqs, max_context_len, desc);
     if (rc != PA_OK) return rc;
     if (options && (options->max_ctas < 0 || options->kernel < 0 || options->kernel > 3 ||
-                    (options->flags & ~(PA_FLAG_CHECK | PA_FLAG_PDL)) != 0 ||
+                    (options->flags & ~(PA_FLAG_CHECK | PA_FLAG_PDL | PA_FLAG_SELFTEST_STALL)) != 0 ||
                     !(options->rope_theta >= 0.f) || !(options->rope_theta < INFINITY) ||
                     (options->kv_dtype != PA_KV_BF16 && options->kv_dtype != PA_KV_E4M3)))
         return PA_ERR_INVALID;
@@ -348,10 +365,15 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     DecodePlan plan;
     rc = make_decode_plan(num_seqs, max_context_len, *desc, options, &plan);
     if (rc != PA_OK) return rc;
+    const bool stall = options && (options->flags & PA_FLAG_SELFTEST_STALL);
+    if (stall && plan.kernel != DecodeKernel::kStream) return PA_ERR_UNSUPPORTED;
     if (!workspace || !aligned(workspace, kWorkspaceAlign) || workspace_bytes < plan.bytes)
         return PA_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     DecodeParams p;
+    p.grid = plan.grid;
+    p.selftest_stall = stall ? 1 : 0;
+    p.wait_ns = stall ? kSelftestWaitNs : kDecodeWaitNs;
     p.q = q;
     p.k_cache = k_cache;
     p.v_cache = v_cache;

@@ -18,6 +18,9 @@
 // current, its address is looked up once with cudaGetSymbolAddress and cached.
 // Calls share the array and it keeps the previous call's contents; the words
 // that must start at zero are cleared by a cudaMemsetAsync on the call's stream.
+// The address belongs to the device's primary context (the runtime API's
+// context); a caller that makes another driver-API context current on the same
+// device must not call this entry point from it.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -63,7 +66,10 @@ extern "C" int pa_decode_noalloc(const pa_bf16* q, const pa_bf16* k_cache, const
                                  const pa_decode_options* options, void* stream) {
     if (num_seqs == 0) return PA_OK;
     const size_t need = pa_decode_workspace_size_ex(num_seqs, max_context_len, desc, options);
-    if (need == 0) return PA_ERR_INVALID;
+    if (need == 0)   // arguments pa_decode_ex refuses: let it name the error (it fails before
+                     // touching the workspace, so nothing is launched)
+        return pa_decode_ex(q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                            max_context_len, scale, out, nullptr, 0, desc, options, stream);
     if (need > kNoAllocScratchBytes) return PA_ERR_WORKSPACE;   // shape needs more than the array
     void* scratch = nullptr;
     const int rc = scratch_address(&scratch);

@@ -41,6 +41,9 @@ __global__ void __launch_bounds__(PG * D / 4) merge_kernel(const DecodeParams p)
         const int4 dsc = reinterpret_cast<const int4*>(p.seq_desc)[(size_t)(kvh / 8) * p.num_seqs + b];
         nsplit = dsc.x;
         if (nsplit <= 1) return;
+        // a descriptor this launch's decode did not write (it gave up on a timed-out wait)
+        // may be left from an earlier call: read nothing outside this launch's partial rows
+        if (dsc.y < 0 || dsc.z < 0 || dsc.z > 1 || (int64_t)dsc.y + nsplit > p.grid) return;
         // CTA i_first + k wrote slot 0 for k > 0; the first CTA used slot dsc.z
         first_row = (((size_t)dsc.y * 2 + dsc.z) * Hkv + kvh) * G + h;
         row0 = (((size_t)(dsc.y + 1) * 2) * Hkv + kvh) * G + h;

@@ -50,6 +50,9 @@ struct DecodeParams {
     int32_t kv_fp8;                // caches hold E4M3 codes (uint8), values = code * scale
     float k_inv_scale, v_inv_scale;  // E4M3: float(1/scale) applied when quantizing new rows
     float out_scale;               // multiplies the normalised output (E4M3: the V scale; else 1)
+    int32_t grid;                  // stream kernel: CTAs of the launch (bounds the merge's reads)
+    int32_t selftest_stall;        // PA_FLAG_SELFTEST_STALL: CTA 0 of the stream kernel idles
+    unsigned long long wait_ns;    // limit of every bounded wait in the stream kernel
 };
 
 // Which decode kernel a plan runs.
@@ -86,6 +89,10 @@ cudaError_t launch_prefill(const PrefillParams& p, int max_q_len, cudaStream_t s
 cudaError_t launch_prefill_tc(const PrefillParams& p, int max_q_len, cudaStream_t stream);
 
 constexpr size_t kWorkspaceAlign = 256;
+// Limits of the decode kernels' bounded waits: normal calls, and PA_FLAG_SELFTEST_STALL calls
+// (whose stalled waits are meant to run out quickly).
+constexpr unsigned long long kDecodeWaitNs = 2000000000ull;   // 2 s
+constexpr unsigned long long kSelftestWaitNs = 10000000ull;   // 10 ms
 
 int num_sms_current_device(int* out);
 int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc& d,

@@ -11,7 +11,7 @@
 
 namespace pa {
 
-constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
+constexpr unsigned long long kWaitTimeoutNs = kDecodeWaitNs;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -49,13 +49,14 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 }
 
 // Bounded wait: false (and the timeout status bit) if the phase does not
-// complete within kWaitTimeoutNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* status) {
+// complete within limit_ns (kWaitTimeoutNs unless the caller asks for less).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* status,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 255u && globaltimer() - t0 > kWaitTimeoutNs) {
+        if ((it & 255u) == 255u && globaltimer() - t0 > limit_ns) {
             raise_status(status, kStatusTimeout);
             return false;
         }
@@ -154,8 +155,9 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 
 // Bounded wait polled by every lane of the warp (each lane acquires the
 // phase itself); the warp-uniform result is lane 0's.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int32_t* status) {
-    const bool ok = mbar_wait(bar, parity, status);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int32_t* status,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
+    const bool ok = mbar_wait(bar, parity, status, limit_ns);
     return __shfl_sync(0xffffffffu, ok, 0);
 }
 

@@ -110,7 +110,7 @@ def rope_pool_matches(gpu: np.ndarray, initial: np.ndarray, k_new: np.ndarray, s
 
 def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int = 0,
              max_ctas: int = 0, check_pool: bool = True, sample=None, fused: bool = False,
-             pdl: bool = False, rope_theta: float = 0.0):
+             pdl: bool = False, rope_theta: float = 0.0, ref_out=None):
     """Runs one step on both sides; returns a dict of results and checks.
 
     fused=False: pa_append_kv through the host slot mapping, then pa_decode.
@@ -118,6 +118,8 @@ def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int =
     pdl=True: PA_FLAG_PDL (the decode kernel may start while the append kernel runs).
     rope_theta > 0 (fused only): q and the new K rows turned by RoPE at position L-1; the
     rotated K rows are held to rope_close's bound, every other byte must be identical.
+    ref_out: the oracle's decode of this very step, when the caller already has it (it is
+    computed here otherwise); returned as res["ref"] either way.
     """
     assert rope_theta == 0.0 or fused
     (slots, tables, lens), (o_slots, o_tables, o_lens) = host_step(b)
@@ -165,7 +167,10 @@ def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int =
             res["pool_equal"] = (np.array_equal(to_host_bits(k_cache), ref_k) and
                                  np.array_equal(to_host_bits(v_cache), ref_v))
     got = out.float().cpu().numpy().astype(np.float64)
-    if sample is None:
+    if ref_out is not None:
+        ref = ref_out
+        res["ok"], res["excess"] = oracle.within_tolerance(got, ref)
+    elif sample is None:
         ref = oracle.paged_decode(q_ref, ref_k, ref_v, o_tables, o_lens, b.scale)
         res["ok"], res["excess"] = oracle.within_tolerance(got, ref)
     else:
@@ -173,5 +178,6 @@ def run_step(b: wl.DecodeBatch, *, kernel=pa.PA_KERNEL_AUTO, split_tokens: int =
         ref = oracle.paged_decode(q_ref[idx], ref_k, ref_v, o_tables[idx], o_lens[idx], b.scale)
         res["ok"], res["excess"] = oracle.within_tolerance(got[idx], ref)
     res["out"] = got
+    res["ref"] = ref
     res["finite"] = bool(np.isfinite(got).all())
     return res

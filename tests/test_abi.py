@@ -72,10 +72,40 @@ def test_decode_rejects_unsupported_shapes_without_a_gpu():
     opts = pa.DecodeOptions(split_tokens=128, kernel=pa.PA_KERNEL_SIMT)  # no device query needed
     assert lib.pa_decode_max_splits(1, 1000, ctypes.byref(d), ctypes.byref(opts)) == 8
     assert pa.pa_decode_workspace_size(2, 1000, d, opts) > 0
-    for bad in (4, 1 << 30, -1):                       # flag bits outside CHECK | PDL
+    for bad in (8, 1 << 30, -1):                       # flag bits outside CHECK | PDL | SELFTEST_STALL
         o = pa.DecodeOptions(flags=bad)
         assert lib.pa_decode_ex(fake, fake, fake, fake, fake, 1, 16, ctypes.c_float(0.1), fake, fake,
                                 1 << 20, ctypes.byref(d), ctypes.byref(o), None) == -1, bad
+
+
+def test_decode_describe_without_a_gpu():
+    d = _desc()
+    opts = pa.DecodeOptions(split_tokens=128, kernel=pa.PA_KERNEL_SIMT)   # no device query needed
+    info = pa.pa_decode_describe(2, 1000, d, opts)
+    assert (info.kernel, info.ctas, info.split_tokens, info.max_splits) == (pa.PA_KERNEL_SIMT, 0, 128, 8)
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode_describe(2, 1000, _desc(head_dim=96), opts)
+    assert e.value.status == -2
+    assert binding.lib.pa_decode_describe(2, 1000, ctypes.byref(d), ctypes.byref(opts), None) == -1
+
+
+def test_noalloc_returns_pa_decode_errors_without_a_gpu():
+    # refused before any device work: the same codes pa_decode_ex gives
+    lib = binding.lib
+    fake = ctypes.c_void_p(0x10000)
+    cases = [(_desc(head_dim=96), None, -2),                                   # head_dim not built
+             (_desc(num_q_heads=34, num_kv_heads=2), None, -2),                # group of 17
+             (_desc(), pa.DecodeOptions(kernel=pa.PA_KERNEL_SIMT, kv_dtype=pa.PA_KV_E4M3,
+                                        k_scale=1.0, v_scale=1.0), -2),        # E4M3 needs the tensor kernel
+             (_desc(), pa.DecodeOptions(split_tokens=100, kernel=pa.PA_KERNEL_SIMT), -1),
+             (_desc(), pa.DecodeOptions(flags=8), -1)]
+    for d, o, want in cases:
+        ob = ctypes.byref(o) if o is not None else None
+        got = lib.pa_decode_noalloc(fake, fake, fake, fake, fake, 1, 16, ctypes.c_float(0.1), fake,
+                                    ctypes.byref(d), ob, None)
+        ref = lib.pa_decode_ex(fake, fake, fake, fake, fake, 1, 16, ctypes.c_float(0.1), fake, fake,
+                               1 << 20, ctypes.byref(d), ob, None)
+        assert got == ref == want, (want, got, ref)
 
 
 def test_rope_append_rejects_bad_arguments_without_a_gpu():
