@@ -386,6 +386,34 @@ PA_API int pa_decode_noalloc(const pa_bf16* q, const pa_bf16* k_cache, const pa_
 PA_API int pa_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
                     const int32_t* lengths, int32_t num_seqs, int32_t block_size, int64_t* slots);
 
+/* ---- host block pool --------------------------------------------------------------------- */
+/*
+ * The allocator of the paged pool on its own (host memory): the KV cache is divided into
+ * fixed-size blocks handed out only as tokens need them, and one block may sit in several
+ * block tables at once (vLLM overview page, "vLLM — PagedAttention으로 LLM 추론 성능을 2~4배
+ * 끌어올린 서빙 엔진" (dev.to), section "PagedAttention — OS 가상 메모리에서 영감"; Nano-vLLM
+ * page, section "KV 캐시와 Block Manager", shared prefix blocks).  For callers that keep
+ * their own block tables; pa_bm_* below applies the same policy and keeps the tables too.
+ * Policy: free ids form a stack with free_order[0] on top; pa_pool_alloc takes n ids from the
+ * top (all or nothing: PA_ERR_OOM_BLOCKS and no change when fewer are free) and gives each a
+ * reference count of 1; pa_pool_share adds one holder to an allocated block; pa_pool_free
+ * drops one, and at zero the block goes back on top of the stack.  Blocks not listed in
+ * free_order start allocated with a count of 1.  Sharing or freeing a free block, or an id
+ * outside [0, num_blocks), is PA_ERR_INVALID and changes nothing.  Not thread-safe.
+ */
+typedef struct pa_block_pool pa_block_pool;
+
+PA_API int pa_pool_create(int32_t num_blocks, const int32_t* free_order, int32_t num_free,
+                          pa_block_pool** out);
+PA_API void pa_pool_destroy(pa_block_pool* pool);
+/* n free blocks, top of the stack first, into blocks[0..n). */
+PA_API int pa_pool_alloc(pa_block_pool* pool, int32_t n, int32_t* blocks);
+PA_API int pa_pool_share(pa_block_pool* pool, int32_t block);
+PA_API int pa_pool_free(pa_block_pool* pool, int32_t block);
+PA_API int32_t pa_pool_num_free(const pa_block_pool* pool);
+/* Holders of a block (0 = free), or -1 for an id outside the pool. */
+PA_API int32_t pa_pool_refcount(const pa_block_pool* pool, int32_t block);
+
 /* ---- host block manager ---------------------------------------------------------------- */
 /*
  * Host-memory bookkeeping of a block pool shared by up to max_seqs sequence

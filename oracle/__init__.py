@@ -20,7 +20,7 @@ import subprocess
 
 import numpy as np
 
-from .block_manager import BlockManagerModel, OutOfBlocks, SharedBlockWrite  # noqa: F401
+from .block_manager import BlockManagerModel, BlockPoolModel, OutOfBlocks, SharedBlockWrite  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "pa_oracle.c")

@@ -274,3 +274,48 @@ class BlockManagerModel:
     def table_array(self, seq: int):
         row = list(self.tables[seq])
         return row + [-1] * (self.max_blocks_per_seq - len(row))
+
+
+class BlockPoolModel:
+    """Model of the per-block pool (pa_pool_*): a stack of free ids and a count of holders.
+
+    The pages give the idea (blocks handed out one at a time as tokens need them; a block of a
+    shared prefix sits in several tables); the policy is the one the block manager above
+    follows: free_order[0] is on top of the stack and handed out first, alloc of n is all or
+    nothing, share adds a holder to an allocated block, free drops one and a block whose count
+    reaches zero goes back on top.  Blocks not in free_order start allocated once.
+    """
+
+    def __init__(self, num_blocks: int, free_order=None):
+        order = list(range(num_blocks)) if free_order is None else [int(b) for b in free_order]
+        assert len(set(order)) == len(order) and all(0 <= b < num_blocks for b in order)
+        self.num_blocks = num_blocks
+        self.refcount = [1] * num_blocks
+        for b in order:
+            self.refcount[b] = 0
+        self.stack = list(reversed(order))          # top = end of the list
+
+    def alloc(self, n: int):
+        if n > len(self.stack):
+            raise OutOfBlocks(n)
+        out = []
+        for _ in range(n):
+            b = self.stack.pop()
+            self.refcount[b] = 1
+            out.append(b)
+        return out
+
+    def share(self, block: int) -> None:
+        if not (0 <= block < self.num_blocks) or self.refcount[block] == 0:
+            raise ValueError("share of a free or unknown block")
+        self.refcount[block] += 1
+
+    def free(self, block: int) -> None:
+        if not (0 <= block < self.num_blocks) or self.refcount[block] == 0:
+            raise ValueError("free of a free or unknown block")
+        self.refcount[block] -= 1
+        if self.refcount[block] == 0:
+            self.stack.append(block)
+
+    def num_free(self) -> int:
+        return len(self.stack)

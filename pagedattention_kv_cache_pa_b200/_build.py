@@ -13,7 +13,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpa.so")
 
 CUDA_SOURCES = ["api.cu", "append.cu", "decode_simt.cu", "decode_tensor.cu", "decode_stream.cu", "merge.cu", "decode_noalloc.cu", "rope.cu", "prefill.cu", "prefill_tc.cu"]
-CXX_SOURCES = ["block_manager.cpp"]
+CXX_SOURCES = ["block_manager.cpp", "block_pool.cpp"]
 HEADERS = ["pa_internal.h", "pa_device.cuh", "pa_ptx.cuh", "pa_umma.cuh"]
 
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",

@@ -139,6 +139,20 @@ lib.pa_prefill.restype = ctypes.c_int
 lib.pa_append_kv_e4m3.argtypes = [_vp, _vp, _vp, _i32, ctypes.c_float, ctypes.c_float, _vp, _vp, _DESC, _vp]
 lib.pa_append_kv_e4m3.restype = ctypes.c_int
 lib.pa_copy_blocks.restype = ctypes.c_int
+lib.pa_pool_create.argtypes = [_i32, _vp, _i32, ctypes.POINTER(_vp)]
+lib.pa_pool_create.restype = ctypes.c_int
+lib.pa_pool_destroy.argtypes = [_vp]
+lib.pa_pool_destroy.restype = None
+lib.pa_pool_alloc.argtypes = [_vp, _i32, _vp]
+lib.pa_pool_alloc.restype = ctypes.c_int
+lib.pa_pool_share.argtypes = [_vp, _i32]
+lib.pa_pool_share.restype = ctypes.c_int
+lib.pa_pool_free.argtypes = [_vp, _i32]
+lib.pa_pool_free.restype = ctypes.c_int
+lib.pa_pool_num_free.argtypes = [_vp]
+lib.pa_pool_num_free.restype = _i32
+lib.pa_pool_refcount.argtypes = [_vp, _i32]
+lib.pa_pool_refcount.restype = _i32
 
 
 def pa_status_string(status: int) -> str:
@@ -444,3 +458,40 @@ class BlockManager:
         rows = np.empty(self.max_seqs, dtype=np.int32)
         n = lib.pa_bm_take_dirty_rows(self._h, rows.ctypes.data, self.max_seqs)
         return rows[:n]
+
+
+class BlockPool:
+    """Owner of a pa_block_pool handle: per-block alloc / share / free (host memory only)."""
+
+    def __init__(self, num_blocks: int, free_order=None):
+        fo = _host(np.asarray(range(num_blocks) if free_order is None else free_order, dtype=np.int32),
+                   np.int32, "free_order")
+        h = _vp()
+        _check(lib.pa_pool_create(int(num_blocks), fo.ctypes.data if fo.size else None, int(fo.size),
+                                  ctypes.byref(h)), "pa_pool_create")
+        self._h = h
+        self.num_blocks = int(num_blocks)
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib.pa_pool_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def alloc(self, n: int) -> np.ndarray:
+        out = np.empty(max(int(n), 1), dtype=np.int32)
+        _check(lib.pa_pool_alloc(self._h, int(n), out.ctypes.data), "pa_pool_alloc")
+        return out[:int(n)]
+
+    def share(self, block: int) -> None:
+        _check(lib.pa_pool_share(self._h, int(block)), "pa_pool_share")
+
+    def free(self, block: int) -> None:
+        _check(lib.pa_pool_free(self._h, int(block)), "pa_pool_free")
+
+    def num_free(self) -> int:
+        return int(lib.pa_pool_num_free(self._h))
+
+    def refcount(self, block: int) -> int:
+        return int(lib.pa_pool_refcount(self._h, int(block)))
