@@ -1,22 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the paged decode step (KV append + paged decode attention).
 
-One step = one decode step of one attention layer for the whole batch:
-append each sequence's new token into its slot (pa_append_kv), then paged
-decode attention over every cached token (pa_decode; long contexts split
-across CTAs and merged in the same launch).  The default workload is the
-Llama-3.2-1B-shaped layer: 64 sequences, Hq=32, Hkv=8, head_dim 64, block
-size 16, cached lengths uniform in [128, 2048], blocks scattered over a pool
-10 % larger than needed.  Successive steps rotate over independent copies of
-the layer's pool (different addresses, > 1 GB together) so that the 126 MB L2
-cannot serve the K/V reads.
+The default line is the 16-layer continuous-batching trace (C5): 256 live
+sequences of the Llama-3.2-1B attention shape (Hq=32, Hkv=8, head_dim 64, block
+size 16) with lognormal lengths, each step appending one token per sequence and
+running paged decode attention in every layer (pa_append_decode per layer;
+the 100-step trace, with sequences finishing and being replaced, replayed as
+often as --steps asks).  A step is one decode step of all 16 layers; the 16
+layer pools (about 7.5 GB) keep the 126 MB L2 from serving the K/V reads.
 
 Prints one JSON line (rank 0).  `value` is seq-steps/s over all ranks with
-inputs resident in HBM; `e2e` repeats the measurement with each step's inputs
-copied from pinned host memory and the output copied back inside the timed
-region.  `roofline` reports the decode kernel's KV-read bandwidth against the
-measured HBM copy bandwidth.  `cpu_baseline` times the fp64 CPU oracle on a
-bounded sample.  With --impl reference the oracle alone is timed.
+inputs resident in HBM; `e2e` repeats the measurement through the host block
+manager, with each step's inputs copied up from pinned host memory in one copy
+and the outputs copied back in one, inside the timed region.  `roofline`
+reports the decode kernel's KV-read bandwidth against the measured HBM copy
+bandwidth.  `cpu_baseline` times the fp64 CPU oracle on a bounded sample.
+`also` carries the other decode workloads of the same run (C2, C3, C4; bf16
+and E4M3 pools), device-timed the same way.  --config c1..c4 / pc / pf measure
+one other workload as the line itself.  With --impl reference the oracle alone
+is timed.
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the
 path has no exchange step); the timed region is bracketed by barriers and the
@@ -66,18 +68,21 @@ WORKLOAD_TEXT = {
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: per config, a few hundred ms of device time)")
+    ap.add_argument("--warmup", type=int, default=None, help="untimed steps after the settle period")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4", "c5", "pc", "pf"], default="c2",
-                    help="pc: prefix caching + copy-on-write (host admission by token ids on the "
-                         "C3 request mix, device block copies)")
-    ap.add_argument("--trace-steps", type=int, default=200,
-                    help="c5: decode steps timed (the 100-step trace replayed as needed)")
+    ap.add_argument("--config", choices=["c1", "c2", "c3", "c4", "c5", "pc", "pf"], default="c5",
+                    help="c5 (default): the 16-layer continuous-batching trace, one step = all 16 "
+                         "layers; pc: prefix caching + copy-on-write (host admission by token ids "
+                         "on the C3 request mix, device block copies)")
+    ap.add_argument("--no-also", action="store_true",
+                    help="c5: skip the C2/C3/C4 (bf16 and E4M3) lines measured after the headline")
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "split"], default="auto")
     ap.add_argument("--max-ctas", type=int, default=0)
-    ap.add_argument("--prefill-kernel", choices=["auto", "tcgen05", "mma"], default="auto",
-                    help="pf: tcgen05 (tensor-memory accumulators; auto) or warp-level mma.sync")
+    ap.add_argument("--prefill-kernel", choices=["auto", "tcgen05", "tcgen05_ws", "mma"], default="auto",
+                    help="pf: tcgen05 (tensor-memory accumulators), tcgen05_ws (one job per warp, O in "
+                         "tensor memory) or warp-level mma.sync")
     ap.add_argument("--path", choices=["fused", "separate"], default="fused",
                     help="fused: pa_append_decode; separate: pa_append_kv then pa_decode")
     ap.add_argument("--split-tokens", type=int, default=0)
@@ -96,7 +101,18 @@ def parse_args(argv=None):
                          "runs; tables and lengths are written once before the timed region, as "
                          "the flag requires (per-call events are then left out: they would "
                          "serialise the calls)")
-    return ap.parse_args(argv)
+    args = ap.parse_args(argv)
+    steps, warmup = DEFAULT_STEPS[args.config]
+    if args.steps is None:
+        args.steps = steps
+    if args.warmup is None:
+        args.warmup = warmup
+    return args
+
+
+# (steps, warm-up steps) when the command line gives none
+DEFAULT_STEPS = {"c1": (20000, 50), "c2": (20000, 50), "c3": (10000, 50), "c4": (2000, 20),
+                 "c5": (300, 10), "pc": (200, 10), "pf": (200, 10)}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -132,7 +148,8 @@ def kernel_source_hash(kernel_name):
     files = {"tensor": ["decode_stream.cu", "pa_ptx.cuh", "merge.cu"],
              "split": ["decode_tensor.cu", "pa_ptx.cuh", "merge.cu"],
              "simt": ["decode_simt.cu", "merge.cu"],
-             "prefill": ["prefill_tc.cu", "pa_umma.cuh", "pa_ptx.cuh"]}[kernel_name]
+             "prefill": ["prefill_tc.cu", "pa_umma.cuh", "pa_ptx.cuh"],
+             "prefill_ws": ["prefill_ws.cu", "pa_umma.cuh", "pa_ptx.cuh"]}[kernel_name]
     files = files + ["pa_device.cuh", "pa_internal.h", "api.cu"]
     h = hashlib.sha256()
     for f in files:
@@ -318,16 +335,74 @@ def cpu_baseline(b, slots, tables, lens, budget_s):
 # ---------------------------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------------------------
-def run_ours(args, rank, world, dist):
+def unique_kv_bytes(tables, lens, block_size, num_kv_heads, head_dim, elem_bytes=2):
+    """K+V bytes of the distinct pool rows a decode launch reads: a block shared by several
+    tables (a common prefix) counts once, with the most tokens any sequence uses in it."""
+    used = {}
+    for row, L in zip(tables, lens):
+        L = int(L)
+        for i in range(-(-L // block_size)):
+            blk = int(row[i])
+            used[blk] = max(used.get(blk, 0), min(block_size, L - i * block_size))
+    return int(2 * sum(used.values()) * num_kv_heads * head_dim * elem_bytes)
+
+
+def settle(fn, seconds=0.2):
+    """Untimed calls for about `seconds` of wall time before the warm-up: clocks, caches and
+    the launch path reach their steady state."""
+    import torch
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn(n)
+        n += 1
+        if n % 32 == 0:
+            torch.cuda.synchronize()
+            if time.perf_counter() - t0 >= seconds:
+                return n
+
+
+def _pack(specs, device):
+    """One pinned host buffer and one device buffer holding several arrays at 256-byte aligned
+    offsets: a step's inputs go up in one copy.  specs: [(name, numpy array)]; returns (host
+    buffer, device buffer, {name: (host numpy view, device tensor view)})."""
+    import torch
+    offs, off = {}, 0
+    for name, a in specs:
+        offs[name] = off
+        off += -(-a.nbytes // 256) * 256
+    h_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
+    d_buf = torch.empty(off, dtype=torch.uint8, device=device)
+    views = {}
+    tdt = {np.dtype(np.uint16): torch.bfloat16, np.dtype(np.int32): torch.int32,
+           np.dtype(np.int64): torch.int64}
+    for name, a in specs:
+        o, n = offs[name], a.nbytes
+        hv = h_buf.numpy()[o:o + n].view(a.dtype).reshape(a.shape)
+        hv[...] = a
+        dv = d_buf[o:o + n].view(tdt[a.dtype]).view(a.shape)
+        views[name] = (hv, dv)
+    return h_buf, d_buf, views
+
+
+def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_steps=None, kv=None,
+               with_cpu=True):
+    """A decode configuration (c1..c4): one step = pa_append_decode (or the separate calls) of
+    one layer for the whole batch, rotating over layer pools larger than L2 together."""
     import torch
     import pagedattention_kv_cache_pa_b200 as pa
 
+    cfg = cfg or args.config
+    K = args.steps if steps is None else steps
+    W = args.warmup if warmup is None else warmup
+    E = args.e2e_steps if e2e_steps is None else e2e_steps
+    kv = kv or args.kv
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
 
-    b = wl.CONFIGS[args.config]()
+    b = wl.CONFIGS[cfg]()
     B, Bs, MB = b.batch, b.block_size, b.max_blocks_per_seq
     Hq, Hkv, D = b.num_q_heads, b.num_kv_heads, b.head_dim
 
@@ -345,12 +420,12 @@ def run_ours(args, rank, world, dist):
     def to_dev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    e4m3 = args.kv == "e4m3"
+    e4m3 = kv == "e4m3"
     KS = VS = 5.0 / 448                                  # N(0,1) data: |x| <= 5 fills the E4M3 range
     pool_bytes = 2 * b.k_cache.nbytes // (2 if e4m3 else 1)
     layers = max(1, min(8, math.ceil(1.0e9 / pool_bytes)))
-    desc0 = pa.CacheDesc.make(num_blocks=b.num_blocks, block_size=Bs, num_kv_heads=Hkv, num_q_heads=Hq,
-                              head_dim=D, max_blocks_per_seq=MB)
+    desc = pa.CacheDesc.make(num_blocks=b.num_blocks, block_size=Bs, num_kv_heads=Hkv, num_q_heads=Hq,
+                             head_dim=D, max_blocks_per_seq=MB)
 
     def pool(a):
         t = to_dev(a)
@@ -360,18 +435,18 @@ def run_ours(args, rank, world, dist):
         rows = t.permute(0, 2, 1, 3).reshape(-1, Hkv, D).contiguous()
         qp = torch.empty(t.shape, dtype=torch.uint8, device=dev)
         pa.pa_append_kv_e4m3(rows, rows, torch.arange(rows.shape[0], dtype=torch.int64, device=dev), KS, KS,
-                             qp, qp, desc0)
+                             qp, qp, desc)
         return qp
     kcs = [pool(b.k_cache) for _ in range(layers)]
     vcs = [pool(b.v_cache) for _ in range(layers)]
     torch.cuda.synchronize()
-    q, k_new, v_new = to_dev(b.q), to_dev(b.k_new), to_dev(b.v_new)
-    slots_d = torch.from_numpy(slots).to(dev)
-    tables_d = torch.from_numpy(tables).to(dev)
-    lens_d = torch.from_numpy(lens).to(dev)
+    # every input of a step in one buffer (the e2e leg uploads it whole, in one copy)
+    h_buf, d_buf, io = _pack([("q", b.q), ("k", b.k_new), ("v", b.v_new), ("slots", slots),
+                              ("tables", tables), ("lens", lens)], dev)
+    d_buf.copy_(h_buf)
+    q, k_new, v_new = io["q"][1], io["k"][1], io["v"][1]
+    slots_d, tables_d, lens_d = io["slots"][1], io["tables"][1], io["lens"][1]
     out = torch.empty_like(q)
-    desc = pa.CacheDesc.make(num_blocks=b.num_blocks, block_size=Bs, num_kv_heads=Hkv,
-                             num_q_heads=Hq, head_dim=D, max_blocks_per_seq=MB)
     kernel = {"auto": pa.PA_KERNEL_AUTO, "simt": pa.PA_KERNEL_SIMT,
               "tensor": pa.PA_KERNEL_TENSOR, "split": pa.PA_KERNEL_TENSOR_SPLIT}[args.kernel]
     pdl = args.pdl == "on"
@@ -380,7 +455,7 @@ def run_ours(args, rank, world, dist):
                             flags=pa.PA_FLAG_PDL if pdl else 0, rope_theta=args.rope, **kvo)
     wsb = pa.pa_decode_workspace_size(B, max_len, desc, opts)
     ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
-    splits = pa.pa_decode_max_splits(B, max_len, desc, opts)
+    plan = pa.pa_decode_describe(B, max_len, desc, opts)
 
     fused = args.path == "fused"
     # separate path: pa_append_kv (or pa_rope_append_kv) through the slot mapping, then pa_decode
@@ -389,40 +464,41 @@ def run_ours(args, rank, world, dist):
     pos_d = torch.from_numpy(np.maximum(lens - 1, 0).astype(np.int32)).to(dev)
     q_rot = torch.empty_like(q)
 
-    def separate(qq, kk, vv, sl, tb, ln, L, ev=None):
+    def call(L, ev=None):
+        if fused:
+            if ev is not None:
+                ev[0].record(stream)
+            pa.pa_append_decode(q, k_new, v_new, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale,
+                                out, ws, desc, opts, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            return
+        qq = q
         if args.rope > 0:
-            pa.pa_rope_append_kv(qq, q_rot, kk, vv, pos_d, sl, args.rope, kcs[L], vcs[L], desc,
+            pa.pa_rope_append_kv(q, q_rot, k_new, v_new, pos_d, slots_d, args.rope, kcs[L], vcs[L], desc,
                                  stream=stream)
             qq = q_rot
         elif e4m3:
-            pa.pa_append_kv_e4m3(kk, vv, sl, KS, VS, kcs[L], vcs[L], desc, stream=stream)
+            pa.pa_append_kv_e4m3(k_new, v_new, slots_d, KS, VS, kcs[L], vcs[L], desc, stream=stream)
         else:
-            pa.pa_append_kv(kk, vv, sl, kcs[L], vcs[L], desc, stream=stream)
+            pa.pa_append_kv(k_new, v_new, slots_d, kcs[L], vcs[L], desc, stream=stream)
         if ev is not None:
             ev[0].record(stream)
-        pa.pa_decode(qq, kcs[L], vcs[L], tb, ln, max_len, b.scale, out, ws, desc, opts_dec,
+        pa.pa_decode(qq, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale, out, ws, desc, opts_dec,
                      stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
-    def step(i):
-        L = i % layers
-        if fused:
-            pa.pa_append_decode(q, k_new, v_new, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale,
-                                out, ws, desc, opts, stream=stream)
-        else:
-            separate(q, k_new, v_new, slots_d, tables_d, lens_d, L)
-
     # correctness guard before timing: the kernel must not report device errors
-    step(0)
+    call(0)
     torch.cuda.synchronize()
     rc = pa.pa_decode_status(ws)
     if rc != 0:
         raise RuntimeError("decode reported %s" % pa.pa_status_string(rc))
 
-    for i in range(args.warmup):
-        step(i)
-    K = args.steps
+    settle(lambda i: call(i % layers))
+    for i in range(W):
+        call(i % layers)
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -433,16 +509,7 @@ def run_ours(args, rank, world, dist):
     clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
     t_start.record(stream)
     for i in range(K):
-        L = i % layers
-        if fused:
-            if not pdl:
-                ev_dec[i][0].record(stream)
-            pa.pa_append_decode(q, k_new, v_new, kcs[L], vcs[L], tables_d, lens_d, max_len, b.scale,
-                                out, ws, desc, opts, stream=stream)
-            if not pdl:
-                ev_dec[i][1].record(stream)
-        else:
-            separate(q, k_new, v_new, slots_d, tables_d, lens_d, L, None if pdl else ev_dec[i])
+        call(i % layers, None if pdl else ev_dec[i])
     t_end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -459,101 +526,119 @@ def run_ours(args, rank, world, dist):
     rc = pa.pa_decode_status(ws)
     if rc != 0:
         raise RuntimeError("decode reported %s during timing" % pa.pa_status_string(rc))
-
     value = world * B * K / (elapsed_ms / 1e3)
 
-    # ---- e2e: host buffers in, result out, every step -----------------------------------
-    E = args.e2e_steps
-    h_q = torch.from_numpy(b.q.view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_k = torch.from_numpy(b.k_new.view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_v = torch.from_numpy(b.v_new.view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_slots = torch.from_numpy(slots).pin_memory()
-    h_tables = torch.from_numpy(tables).pin_memory()
-    h_lens = torch.from_numpy(lens).pin_memory()
-    h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
-    d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
-    d_slots, d_tables, d_lens = (torch.empty_like(slots_d), torch.empty_like(tables_d),
-                                 torch.empty_like(lens_d))
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_tables, h_lens))
-    d2h = h_out.numel() * h_out.element_size()
+    # ---- e2e: the step's inputs up from pinned host memory in one copy, the output back in one
+    e2e = None
+    if E > 0:
+        h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
 
-    def e2e_step(i):
-        L = i % layers
-        for dst, src in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_slots, h_slots),
-                         (d_tables, h_tables), (d_lens, h_lens)):
-            dst.copy_(src, non_blocking=True)
-        if fused:
-            pa.pa_append_decode(d_q, d_k, d_v, kcs[L], vcs[L], d_tables, d_lens, max_len, b.scale,
-                                out, ws, desc, opts, stream=stream)
-        else:
-            separate(d_q, d_k, d_v, d_slots, d_tables, d_lens, L)
-        h_out.copy_(out, non_blocking=True)
+        def e2e_step(i):
+            d_buf.copy_(h_buf, non_blocking=True)
+            call(i % layers)
+            h_out.copy_(out, non_blocking=True)
 
-    for i in range(min(args.warmup, 20)):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(E):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms, = max_over_ranks([e2e_ms], dist, dev)
-    e2e_value = world * B * E / (e2e_ms / 1e3)
+        for i in range(min(W, 20)):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(E):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms, = max_over_ranks([e0.elapsed_time(e1)], dist, dev)
+        e2e = {"value": world * B * E / (e2e_ms / 1e3), "unit": "seq-steps/s",
+               "h2d_bytes_per_step": int(h_buf.numel()), "d2h_bytes_per_step": int(h_out.numel() * 2),
+               "copies_per_step": {"h2d": 1, "d2h": 1}, "steps": E}
 
     if rank != 0:
         return None
 
-    # PA_KERNEL_AUTO runs the tensor-core kernel; with Hkv a multiple of 8 (every
-    # workload here) that is the whole-group, stream-partitioned one
-    kernel_name = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR_SPLIT: "split"}.get(kernel, "tensor")
+    kernel_name = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR_SPLIT: "split"}.get(plan.kernel, "tensor")
     peak, peak_kind = measured_peaks()
-    kv_bytes = kv_read_bytes(lens, Hkv, D, 1 if e4m3 else 2)
+    elem = 1 if e4m3 else 2
+    logical = kv_read_bytes(lens, Hkv, D, elem)
+    unique = unique_kv_bytes(tables, lens, Bs, Hkv, D, elem)
+    kv_bytes = unique                                    # equal to logical unless blocks are shared
     achieved = kv_bytes / (dec_avg_ms / 1e3) / 1e9
     res = {
         "metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+        "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 kv, bf16 q/out" if e4m3 else "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT[args.config], "config": args.config,
+        "config": {"workload": WORKLOAD_TEXT[cfg], "config": cfg,
                    "batch": B, "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
                    "block_size": Bs, "num_blocks": b.num_blocks, "mean_context": float(lens.mean()),
-                   "max_context": max_len, "decode_kernel": kernel_name,
-                   "split_tokens": args.split_tokens or "auto", "max_splits": splits,
+                   "max_context": max_len, "decode_kernel": kernel_name, "ctas": plan.ctas,
+                   "split_tokens": args.split_tokens or "auto", "max_splits": plan.max_splits,
                    "call": "pa_append_decode" if fused else
                            ("pa_rope_append_kv + pa_decode" if args.rope > 0 else "pa_append_kv + pa_decode"),
-                   "pdl": pdl, "rope_theta": args.rope, "kv_dtype": args.kv,
+                   "pdl": pdl, "rope_theta": args.rope, "kv_dtype": kv,
                    "l2": "inputs larger than L2: %d rotating layer pools of %.0f MB" % (layers, pool_bytes / 1e6),
                    "parallelism": "replicas x%d" % world},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
-                     "traffic": profiled_traffic(args.config + ("-e4m3" if e4m3 else ""), kernel_name),
+                     "traffic": profiled_traffic(cfg + ("-e4m3" if e4m3 else ""), kernel_name),
                      "kernel": ("pa_append_decode (%s)" if fused else "pa_decode (%s)") % kernel_name,
                      "algorithmic_bytes_per_launch": kv_bytes,
+                     "bytes_basis": "unique pool rows (a shared prefix counted once)" if unique != logical
+                                    else "K+V rows of every context",
+                     "logical_bytes_per_launch": logical,
                      "avg_launch_ms": dec_avg_ms,
                      "launch_timing": "timed region / calls" if pdl else "CUDA events around each call"},
         "kv_read_gbs_step": kv_bytes * K / (elapsed_ms / 1e3) / 1e9,
-        "e2e": {"value": e2e_value, "unit": "seq-steps/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": E},
-        # per step: the append (its own kernel unless the tensor kernel fuses it), the decode
+        "e2e": e2e,
+        # per step: the append (its own kernel unless the stream kernel fuses it), the decode
         # kernel and (when any sequence can be cut) the merge kernel
         "gpu_launches": K * ((0 if (fused and kernel_name == "tensor") else 1) + 1 +
-                             (1 if (kernel_name == "tensor" or splits > 1) else 0)),
+                             (1 if (kernel_name == "tensor" or plan.max_splits > 1) else 0)),
         "clocks": clk,
     }
-    if not args.no_cpu_baseline and world == 1:
+    if with_cpu and not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(b, slots, tables, lens, args.cpu_seconds)
+    del kcs, vcs
     return res
+
+
+def run_ours(args, rank, world, dist):
+    return run_decode(args, rank, world, dist)
+
+
+# The other decode workloads, measured in the same run as the headline line (device time,
+# inputs resident in HBM), so that one bench run records all of them.
+ALSO = [("c2", "bf16", 6000), ("c3", "bf16", 4000), ("c4", "bf16", 1000), ("c2", "e4m3", 6000),
+        ("c4", "e4m3", 1000)]
+
+
+def run_also(args, rank, world, dist):
+    import torch
+    out = {}
+    for cfg, kv, steps in ALSO:
+        r = run_decode(args, rank, world, dist, cfg=cfg, steps=steps, warmup=20, e2e_steps=0, kv=kv,
+                       with_cpu=False)
+        torch.cuda.empty_cache()
+        if r is None:
+            continue
+        rf = r["roofline"]
+        out[cfg + ("-e4m3" if kv == "e4m3" else "")] = {
+            "workload": r["config"]["workload"], "value": r["value"], "unit": r["unit"],
+            "steps": r["steps"], "warmup": r["warmup"], "ms_per_step": r["ms_per_step"],
+            "kv_dtype": kv, "roofline": {k: rf[k] for k in ("achieved", "peak", "frac", "unit",
+                                                           "algorithmic_bytes_per_launch", "bytes_basis",
+                                                           "avg_launch_ms", "traffic")},
+            "clocks": r["clocks"]}
+    return out
 
 
 def run_c5(args, rank, world, dist):
     """C5: the continuous-batching trace.  One step = one decode step of all 16 layers for the
-    256 live sequences (host block manager, then pa_append_decode per layer)."""
+    256 live sequences (host block manager, then pa_append_decode per layer).  The 100-step
+    trace is replayed as often as --steps asks."""
     import torch
     import pagedattention_kv_cache_pa_b200 as pa
 
@@ -593,17 +678,23 @@ def run_c5(args, rank, world, dist):
     def to_dev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    kcs, vcs, qs, ks, vs, outs = [], [], [], [], [], []
+    kcs, vcs, tok = [], [], []
     for layer in range(NL):
         kc, vc = t.pool(layer)
         kcs.append(to_dev(kc))
         vcs.append(to_dev(vc))
         del kc, vc
-        q, k, v = t.token_inputs(layer, 0)
-        qs.append(to_dev(q))
-        ks.append(to_dev(k))
-        vs.append(to_dev(v))
-        outs.append(torch.empty_like(qs[-1]))
+        tok.append(t.token_inputs(layer, 0))
+    # q, k, v of every layer in one buffer, the outputs of every layer in another: the e2e leg
+    # moves a step's inputs up in one copy and its outputs down in one
+    h_tok, d_tok, io = _pack([(n % l, a) for l in range(NL) for n, a in zip(("q%d", "k%d", "v%d"), tok[l])],
+                             dev)
+    d_tok.copy_(h_tok)
+    qs = [io["q%d" % l][1] for l in range(NL)]
+    ks = [io["k%d" % l][1] for l in range(NL)]
+    vs = [io["v%d" % l][1] for l in range(NL)]
+    outs_all = torch.empty((NL,) + tuple(qs[0].shape), dtype=torch.bfloat16, device=dev)
+    outs = [outs_all[l] for l in range(NL)]
     desc = pa.CacheDesc.make(num_blocks=N, block_size=Bs, num_kv_heads=Hkv, num_q_heads=Hq,
                              head_dim=D, max_blocks_per_seq=MB)
     kernel = {"auto": pa.PA_KERNEL_AUTO, "simt": pa.PA_KERNEL_SIMT,
@@ -613,20 +704,27 @@ def run_c5(args, rank, world, dist):
                             flags=pa.PA_FLAG_PDL if pdl else 0, rope_theta=args.rope)
     ws = torch.zeros(pa.pa_decode_workspace_size(B, int(lens.max()), desc, opts), dtype=torch.uint8,
                      device=dev)
+    plan = pa.pa_decode_describe(B, int(lens.max()), desc, opts)
 
-    def call(s, layer):
-        pa.pa_append_decode(qs[layer], ks[layer], vs[layer], kcs[layer], vcs[layer], tables_d[s],
-                            lens_d[s], step_max[s], t.scale, outs[layer], ws, desc, opts,
+    def call(s, layer, tb=None, ln=None, mx=None):
+        pa.pa_append_decode(qs[layer], ks[layer], vs[layer], kcs[layer], vcs[layer],
+                            tables_d[s] if tb is None else tb, lens_d[s] if ln is None else ln,
+                            step_max[s] if mx is None else mx, t.scale, outs[layer], ws, desc, opts,
                             stream=stream)
 
-    for s in range(3):
+    def trace_step(i):
         for layer in range(NL):
-            call(s, layer)
+            call(i % S, layer)
+
+    trace_step(0)
     torch.cuda.synchronize()
     rc = pa.pa_decode_status(ws)
     if rc != 0:
         raise RuntimeError("decode reported %s" % pa.pa_status_string(rc))
-    K = args.trace_steps
+    K, W = args.steps, args.warmup
+    settle(trace_step)
+    for i in range(W):
+        trace_step(i)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K * NL)]
     t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -658,20 +756,20 @@ def run_c5(args, rank, world, dist):
     gbs = float(kv_per_call.sum() / (call_ms.sum() / 1e3) / 1e9)
     elapsed_ms, = max_over_ranks([elapsed_ms], dist, dev)
     value = world * B * K / (elapsed_ms / 1e3)
+    rc = pa.pa_decode_status(ws)
+    if rc != 0:
+        raise RuntimeError("decode reported %s during timing" % pa.pa_status_string(rc))
 
-    # e2e: the host block manager replays the trace inside the timed region; per step the
-    # table rows and lengths go up, per layer q/k/v go up and the output comes back
+    # e2e: the host block manager replays the trace inside the timed region.  Per step one copy
+    # up (table rows, lengths, every layer's q/k/v) and one copy down (every layer's output),
+    # through two pinned staging buffers so that the host prepares step i+1 while step i runs.
     E = min(args.e2e_steps, S)
-    h_q = [torch.from_numpy(np.ascontiguousarray(t.token_inputs(l, 0)[0]).view(np.int16)).view(torch.bfloat16).pin_memory() for l in range(NL)]
-    h_k = [torch.from_numpy(np.ascontiguousarray(t.token_inputs(l, 0)[1]).view(np.int16)).view(torch.bfloat16).pin_memory() for l in range(NL)]
-    h_v = [torch.from_numpy(np.ascontiguousarray(t.token_inputs(l, 0)[2]).view(np.int16)).view(torch.bfloat16).pin_memory() for l in range(NL)]
-    h_out = torch.empty(outs[0].shape, dtype=torch.bfloat16).pin_memory()
-    h_tab = torch.empty((B, MB), dtype=torch.int32).pin_memory()
-    h_len = torch.empty((B,), dtype=torch.int32).pin_memory()
-    d_q, d_k, d_v = torch.empty_like(qs[0]), torch.empty_like(ks[0]), torch.empty_like(vs[0])
-    d_tab, d_len = torch.empty((B, MB), dtype=torch.int32, device=dev), torch.empty((B,), dtype=torch.int32, device=dev)
-    h2d = h_tab.numel() * 4 + h_len.numel() * 4 + NL * (h_q[0].numel() + h_k[0].numel() + h_v[0].numel()) * 2
-    d2h = NL * h_out.numel() * 2
+    stage = []
+    for _ in range(2):
+        hb, db, v2 = _pack([("tables", tables[0]), ("lens", lens[0])] +
+                           [(n % l, a) for l in range(NL) for n, a in zip(("q%d", "k%d", "v%d"), tok[l])], dev)
+        stage.append((hb, db, v2, torch.cuda.Event()))
+    h_outs = [torch.empty(outs_all.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -680,19 +778,18 @@ def run_c5(args, rank, world, dist):
     for step, bm in replay():
         if step >= E:
             break
-        torch.cuda.current_stream().synchronize()   # pinned staging is reused each step
-        h_tab.numpy()[:] = bm.block_tables()
-        h_len.numpy()[:] = bm.context_lens()
-        d_tab.copy_(h_tab, non_blocking=True)
-        d_len.copy_(h_len, non_blocking=True)
-        mx = int(h_len.numpy().max())
+        hb, db, v2, done = stage[step & 1]
+        done.synchronize()                       # the copy that last read this staging buffer is over
+        v2["tables"][0][...] = bm.block_tables()
+        v2["lens"][0][...] = bm.context_lens()
+        mx = int(v2["lens"][0].max())
+        db.copy_(hb, non_blocking=True)
         for layer in range(NL):
-            d_q.copy_(h_q[layer], non_blocking=True)
-            d_k.copy_(h_k[layer], non_blocking=True)
-            d_v.copy_(h_v[layer], non_blocking=True)
-            pa.pa_append_decode(d_q, d_k, d_v, kcs[layer], vcs[layer], d_tab, d_len, mx, t.scale,
+            pa.pa_append_decode(v2["q%d" % layer][1], v2["k%d" % layer][1], v2["v%d" % layer][1],
+                                kcs[layer], vcs[layer], v2["tables"][1], v2["lens"][1], mx, t.scale,
                                 outs[layer], ws, desc, opts, stream=stream)
-            h_out.copy_(outs[layer], non_blocking=True)
+        h_outs[step & 1].copy_(outs_all, non_blocking=True)
+        done.record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -700,15 +797,16 @@ def run_c5(args, rank, world, dist):
     if rank != 0:
         return None
     peak, peak_kind = measured_peaks()
-    kernel_name = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR_SPLIT: "split"}.get(kernel, "tensor")
+    kernel_name = {pa.PA_KERNEL_SIMT: "simt", pa.PA_KERNEL_TENSOR_SPLIT: "split"}.get(plan.kernel, "tensor")
     res = {
         "metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": world, "steps": K,
-        "warmup": 3, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
+        "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT["c5"], "config": "c5", "batch": B, "layers": NL,
-                   "trace_steps": S, "num_blocks": N, "mean_context": float(lens.mean()),
-                   "decode_kernel": kernel_name, "call": "pa_append_decode per layer", "pdl": pdl,
-                   "rope_theta": args.rope,
+                   "trace_steps": S, "step": "one decode step of all 16 layers (trace replayed as needed)",
+                   "num_blocks": N, "mean_context": float(lens.mean()),
+                   "decode_kernel": kernel_name, "ctas": plan.ctas, "call": "pa_append_decode per layer",
+                   "pdl": pdl, "rope_theta": args.rope,
                    "l2": "inputs larger than L2: 16 layer pools of %.0f MB" % (2 * kcs[0].numel() * 2 / 1e6),
                    "parallelism": "replicas x%d" % world},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
@@ -717,16 +815,20 @@ def run_c5(args, rank, world, dist):
                      "traffic": profiled_traffic("c5", kernel_name),
                      "kernel": "pa_append_decode (%s)" % kernel_name,
                      "algorithmic_bytes_per_launch": float(kv_per_call.mean()),
+                     "bytes_basis": "K+V rows of every context",
                      "avg_launch_ms": float(call_ms.mean()),
                      "launch_timing": "timed region / calls" if pdl else "CUDA events around each call"},
         "e2e": {"value": world * B * E / (e2e_ms / 1e3), "unit": "seq-steps/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": E,
+                "h2d_bytes_per_step": int(stage[0][0].numel()),
+                "d2h_bytes_per_step": int(h_outs[0].numel() * 2),
+                "copies_per_step": {"h2d": 1, "d2h": 1}, "steps": E,
                 "includes": "host block manager (retire, admit, append) per step"},
         "gpu_launches": K * NL * 2,
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline_c5(t, tables, lens, args.cpu_seconds)
+    del kcs, vcs
     return res
 
 
@@ -943,6 +1045,7 @@ def run_pf(args, rank, world, dist):
     if rank != 0:
         return None
     flops = prefill_flops(lens, q_lens, Hq, D)
+    pk = "tcgen05" if args.prefill_kernel == "auto" else args.prefill_kernel
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -960,8 +1063,10 @@ def run_pf(args, rank, world, dist):
                    "l2": "working set (%.0f MB of KV) fits L2: prefill is compute-bound" % (2 * b.k_cache.nbytes / 1e6)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": kind,
-                     "traffic": None if args.prefill_kernel == "mma" else profiled_traffic("pf", "prefill"),
-                     "kernel": "pa_prefill (%s bf16)" % ("mma.sync" if args.prefill_kernel == "mma" else "tcgen05"),
+                     "traffic": profiled_traffic("pf", "prefill_ws" if pk == "tcgen05_ws" else "prefill")
+                                if pk in ("tcgen05", "tcgen05_ws") else None,
+                     "kernel": "pa_prefill (%s bf16)" % {"mma": "mma.sync", "tcgen05": "tcgen05",
+                                                         "tcgen05_ws": "tcgen05, warp-specialized"}[pk],
                      "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_ms},
         "e2e": {"value": world * T * E / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int((q_h.nbytes + k_h.nbytes + v_h.nbytes)), "d2h_bytes_per_step": int(q_h.nbytes),
@@ -994,6 +1099,10 @@ def main(argv=None):
     try:
         runner = {"c5": run_c5, "pc": run_pc, "pf": run_pf}.get(args.config, run_ours)
         res = runner(args, rank, world, dist)
+        if args.config == "c5" and not args.no_also:
+            also = run_also(args, rank, world, dist)
+            if res is not None:
+                res["also"] = also
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

@@ -176,7 +176,7 @@ typedef struct pa_decode_options {
                            /* 0 = no rotation.  pa_decode(_ex) rejects a nonzero value.         */
     int32_t kv_dtype;      /* PA_KV_BF16 (default) or PA_KV_E4M3: the caches are uint8 E4M3     */
                            /* pools of the same [N][Hkv][Bs][D] shape (the pointers are read as */
-                           /* bytes); the whole-group tensor kernel only, no RoPE               */
+                           /* bytes); the whole-group tensor kernel only                        */
     float k_scale;         /* PA_KV_E4M3: K value = code value * k_scale (> 0)                  */
     float v_scale;         /* PA_KV_E4M3: V value = code value * v_scale (> 0)                  */
 } pa_decode_options;
@@ -198,15 +198,18 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * with K_j, V_j the rows of kv head h / (Hq/Hkv).  fp32 accumulation, online
  * softmax, the result rounded to nearest-even bf16.  A sequence with
  * context_lens[b] == 0 outputs zeros.  Long contexts are split across CTAs:
- * each piece leaves an fp32 partial state in the workspace, and a second
- * kernel, launched by the same call on the same stream, merges them
- * (log-sum-exp) into out.
+ * each piece leaves an fp32 partial state in the workspace, and the pieces are
+ * merged (log-sum-exp) into out: by the CTA that finishes a sequence's last
+ * piece, inside the same launch, for the whole-group tensor kernel; by a
+ * second kernel, launched by the same call on the same stream, for the others.
  *
  * workspace: caller-owned device buffer of at least
  * pa_decode_workspace_size(...) bytes, 256-byte aligned, ZERO-FILLED BEFORE
- * ITS FIRST USE.  The kernel leaves its counters at zero when it completes,
- * so the buffer can be reused by later calls without clearing; calls that
- * may overlap on the GPU need separate workspaces.
+ * ITS FIRST USE.  The kernels leave their work counters at zero when they
+ * complete, and the merge counters of the whole-group tensor kernel carry the
+ * call's number (so a workspace left by a call that gave up on a wait serves
+ * the next call as it is); the buffer can be reused by later calls without
+ * clearing.  Calls that may overlap on the GPU need separate workspaces.
  *
  * Built shapes: head_dim 64 or 128; block_size 8, 16, 32, 64, 128 or 256;
  * Hq / Hkv <= 16.  Others return PA_ERR_UNSUPPORTED.  The tensor-core
@@ -222,8 +225,9 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * options->kv_dtype == PA_KV_E4M3: the caches are E4M3 pools (see
  * pa_append_kv_e4m3) and the attention reads K = code value * k_scale,
  * V = code value * v_scale; only the whole-group tensor kernel serves it
- * (PA_ERR_UNSUPPORTED otherwise, and with rope_theta).  pa_append_decode then
- * quantizes the new rows with the same scales as it writes them.
+ * (PA_ERR_UNSUPPORTED otherwise).  pa_append_decode then quantizes the new
+ * rows with the same scales as it writes them; with rope_theta > 0 the new K
+ * row is turned and rounded to bf16 first, and that bf16 row is quantized.
  *
  * PA_FLAG_PDL (whole-group tensor kernel only; ignored by the others): the
  * decode kernel is launched as a programmatic dependent of the kernel before
@@ -233,7 +237,8 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * workspace are touched after the wait.  Set the flag only when context_lens
  * and block_tables were complete before the previous kernel on `stream`
  * started (host-written metadata, as in a serving step's layer loop).  The
- * library's own kernels (append, merge) let such a launch start early.
+ * library's own kernels (append, merge, the decode itself) let such a launch
+ * start early.
  */
 PA_API int pa_decode(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
               const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
@@ -297,6 +302,9 @@ PA_API int pa_append_decode(const pa_bf16* q, const pa_bf16* k, const pa_bf16* v
 #define PA_PREFILL_AUTO     0
 #define PA_PREFILL_TCGEN05  1
 #define PA_PREFILL_MMA      2
+#define PA_PREFILL_TCGEN05_WS 3   /* tcgen05 with one job per warp (softmax, MMA issue, TMA) and */
+                                  /* O accumulated in tensor memory; block sizes 8, 16, 32, 64  */
+                                  /* or multiples of 64 (PA_ERR_UNSUPPORTED otherwise)          */
 PA_API int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
                       const int32_t* block_tables, const int32_t* cu_seqlens_q,
                       const int32_t* context_lens, int32_t num_seqs, int32_t max_q_len, float scale,

@@ -12,7 +12,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpa.so")
 
-CUDA_SOURCES = ["api.cu", "append.cu", "decode_simt.cu", "decode_tensor.cu", "decode_stream.cu", "merge.cu", "decode_noalloc.cu", "rope.cu", "prefill.cu", "prefill_tc.cu"]
+CUDA_SOURCES = ["api.cu", "append.cu", "decode_simt.cu", "decode_tensor.cu", "decode_stream.cu", "merge.cu", "decode_noalloc.cu", "rope.cu", "prefill.cu", "prefill_tc.cu", "prefill_ws.cu"]
 CXX_SOURCES = ["block_manager.cpp", "block_pool.cpp"]
 HEADERS = ["pa_internal.h", "pa_device.cuh", "pa_ptx.cuh", "pa_umma.cuh"]
 

@@ -256,8 +256,9 @@ def pa_copy_blocks(k_cache, v_cache, copies, desc: CacheDesc, stream=None) -> No
                               _stream(stream)), "pa_copy_blocks")
 
 
-PA_PREFILL_AUTO, PA_PREFILL_TCGEN05, PA_PREFILL_MMA = 0, 1, 2
-_PREFILL_KERNELS = {"auto": PA_PREFILL_AUTO, "tcgen05": PA_PREFILL_TCGEN05, "mma": PA_PREFILL_MMA}
+PA_PREFILL_AUTO, PA_PREFILL_TCGEN05, PA_PREFILL_MMA, PA_PREFILL_TCGEN05_WS = 0, 1, 2, 3
+_PREFILL_KERNELS = {"auto": PA_PREFILL_AUTO, "tcgen05": PA_PREFILL_TCGEN05, "mma": PA_PREFILL_MMA,
+                    "tcgen05_ws": PA_PREFILL_TCGEN05_WS}
 
 
 def pa_prefill(q, k_cache, v_cache, block_tables, cu_seqlens_q, context_lens, max_q_len: int, scale: float,

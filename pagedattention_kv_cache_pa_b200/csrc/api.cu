@@ -46,6 +46,15 @@ int32_t env_split_tokens() {
     return v;
 }
 
+// Call numbers for the stream kernel's merge counters: never 0 (a zero-filled workspace holds
+// counters of call 0), distinct for 2^32 - 1 calls in a row.
+uint32_t next_epoch() {
+    static std::atomic<uint32_t> n{0};
+    uint32_t e = n.fetch_add(1, std::memory_order_relaxed) + 1;
+    if (e == 0) e = n.fetch_add(1, std::memory_order_relaxed) + 1;
+    return e;
+}
+
 int32_t env_kernel() {
     static int32_t v = [] {
         const char* s = getenv("PA_DECODE_KERNEL");
@@ -98,6 +107,7 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
     plan->off_desc = kWorkspaceAlign;
     plan->off_lse = plan->off_desc;
     plan->off_qrot = 0;
+    plan->off_mcnt = plan->off_gcnt = 0;
     plan->grid = 0;
     plan->split_tokens = 0;
     plan->max_splits = 1;
@@ -112,7 +122,9 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
         plan->off_lse = plan->off_desc + up((size_t)(d.num_kv_heads / 8) * num_seqs * 16);
         const size_t rows = (size_t)plan->grid * 2 * d.num_kv_heads * G;
         plan->off_o = plan->off_lse + up(rows * sizeof(float));
-        plan->bytes = plan->off_o + up(rows * (size_t)d.head_dim * sizeof(float));
+        plan->off_mcnt = plan->off_o + up(rows * (size_t)d.head_dim * sizeof(float));
+        plan->off_gcnt = plan->off_mcnt + up((size_t)(d.num_kv_heads / 8) * num_seqs * sizeof(uint64_t));
+        plan->bytes = plan->off_gcnt + up((size_t)plan->grid * 2 * sizeof(uint64_t));
         return PA_OK;
     }
     if (kernel == PA_KERNEL_TENSOR || kernel == PA_KERNEL_TENSOR_SPLIT) {
@@ -235,8 +247,10 @@ extern "C" int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf1
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || num_seqs > 65535 || max_q_len < 0 || !(scale > 0.f) || !(scale < INFINITY))
         return PA_ERR_INVALID;
-    if (kernel != PA_PREFILL_AUTO && kernel != PA_PREFILL_TCGEN05 && kernel != PA_PREFILL_MMA)
+    if (kernel != PA_PREFILL_AUTO && kernel != PA_PREFILL_TCGEN05 && kernel != PA_PREFILL_MMA &&
+        kernel != PA_PREFILL_TCGEN05_WS)
         return PA_ERR_INVALID;
+    if (kernel == PA_PREFILL_TCGEN05_WS && !prefill_ws_supports(desc->block_size)) return PA_ERR_UNSUPPORTED;
     if (desc->head_dim != 64 && desc->head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (desc->num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
     if (num_seqs == 0 || max_q_len == 0) return PA_OK;
@@ -267,8 +281,10 @@ extern "C" int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf1
     p.group = desc->num_q_heads / desc->num_kv_heads;
     p.max_blocks_per_seq = desc->max_blocks_per_seq;
     p.scale_log2 = scale * 1.4426950408889634f;
-    const cudaError_t e = kernel == PA_PREFILL_MMA ? launch_prefill(p, max_q_len, (cudaStream_t)stream)
-                                                   : launch_prefill_tc(p, max_q_len, (cudaStream_t)stream);
+    const cudaStream_t st = (cudaStream_t)stream;
+    const cudaError_t e = kernel == PA_PREFILL_MMA          ? launch_prefill(p, max_q_len, st)
+                          : kernel == PA_PREFILL_TCGEN05_WS ? launch_prefill_ws(p, max_q_len, st)
+                                                            : launch_prefill_tc(p, max_q_len, st);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -354,7 +370,6 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     if (fp8 && (!(options->k_scale > 0.f) || !(options->k_scale < INFINITY) ||
                 !(options->v_scale > 0.f) || !(options->v_scale < INFINITY)))
         return PA_ERR_INVALID;
-    if (fp8 && rope_theta > 0.f) return PA_ERR_UNSUPPORTED;   // RoPE on E4M3 pools: not built
     if (rope_theta > 0.f && !k_new) return PA_ERR_INVALID;   // RoPE needs the new token (pa_append_decode)
     if (num_seqs == 0) return PA_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
@@ -372,6 +387,10 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     char* ws = static_cast<char*>(workspace);
     DecodeParams p;
     p.grid = plan.grid;
+    p.inline_merge = plan.kernel == DecodeKernel::kStream ? 1 : 0;
+    p.epoch = next_epoch();
+    p.merge_cnt = reinterpret_cast<unsigned long long*>(ws + plan.off_mcnt);
+    p.group_cnt = reinterpret_cast<unsigned long long*>(ws + plan.off_gcnt);
     p.selftest_stall = stall ? 1 : 0;
     p.wait_ns = stall ? kSelftestWaitNs : kDecodeWaitNs;
     p.q = q;
@@ -428,8 +447,10 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
         case DecodeKernel::kSplit: e = launch_decode_tensor(p, st); break;
         default: e = launch_decode_simt(p, st); break;
     }
-    // second pass: merge the pieces of every sequence that was cut
-    if (e == cudaSuccess && (plan.kernel == DecodeKernel::kStream || plan.max_splits > 1))
+    // second pass: merge the pieces of every sequence that was cut (the stream kernel merges
+    // its own)
+    if (e == cudaSuccess && ((plan.kernel == DecodeKernel::kStream && !p.inline_merge) ||
+                             (plan.kernel != DecodeKernel::kStream && plan.max_splits > 1)))
         e = launch_merge(p, plan.kernel == DecodeKernel::kStream,
                          plan.kernel != DecodeKernel::kSimt, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;

@@ -1,9 +1,9 @@
 // Paged decode attention, stream-partitioned: the main tensor-core kernel.
 //
 // Shaped by two facts measured on the B200: HBM streams at full rate through
-// TMA only when each request is large (about 16 KB; a CTA retires roughly one
-// request every 0.4 us whatever its size), and a decode step is short, so any
-// imbalance between CTAs is paid in full.
+// TMA only when each request is large (about 16 KB: one 2 KB box per page and
+// kv head, as in decode_tensor.cu, leaves the CTAs' request rate the limit),
+// and a decode step is short, so any imbalance between CTAs is paid in full.
 //
 //  * A CTA covers a group of 8 kv heads at once.  In the pool layout
 //    [block][kv head][token][head dim], the 16 tokens x 8 heads of a block are
@@ -144,6 +144,134 @@ __device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 x, float inv_scale) {
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
+// ---- merging the pieces of cut sequences, inside the decode kernel ----------------------
+// A sequence cut across CTAs i_first .. i_first + n - 1 leaves one normalised partial state per
+// piece: piece 0 in partial slot `fslot` of CTA i_first, piece k >= 1 in slot 0 of CTA
+// i_first + k (rows of part_o / part_lse).  Each CTA, once its pieces are written, counts them
+// on the sequence's counter; the CTA whose count completes it merges all pieces (log-sum-exp,
+// the same arithmetic as merge.cu) into out.  A sequence of more than kMergeFan pieces is
+// merged in two levels: the pieces are counted per group of kMergeFan on a counter of the
+// group's first piece; the CTA completing a group merges it into that first piece's rows and
+// counts the group on the sequence's counter, and the CTA completing that merges the groups.
+// Counters hold (call number << 32 | count): a counter left by an earlier call (one that gave
+// up on a wait, say) reads as zero, so they never need clearing.
+constexpr int32_t kMergeFan = 16;
+
+__device__ __forceinline__ int32_t counter_add(unsigned long long* c, uint32_t epoch, int32_t* status) {
+    unsigned long long old = __ldcg(c);
+    for (int it = 0; it < (1 << 20); ++it) {
+        const unsigned long long nw =
+            (uint32_t)(old >> 32) == epoch ? old + 1 : (((unsigned long long)epoch << 32) | 1ull);
+        const unsigned long long prev = atomicCAS(c, old, nw);
+        if (prev == old) return (int32_t)(uint32_t)nw;
+        old = prev;
+    }
+    raise_status(status, kStatusTimeout);
+    return -1;
+}
+
+// Merges pieces k = k0, k0 + step, ... < k1 of one sequence for the 8 kv heads of group gi:
+// into out (bf16) when lead < 0, else into the partial rows of piece `lead` (fp32 + lse).
+template <int D>
+__device__ void merge_pieces(const DecodeParams& p, int32_t b, int32_t gi, int32_t i_first, int32_t fslot,
+                             int32_t k0, int32_t k1, int32_t step, int32_t lead, float* s_lse) {
+    const int32_t G = p.group, Hkv = p.num_kv_heads;
+    constexpr int kCols = D / 4;
+    const int32_t units = 8 * G * kCols;
+    auto row_of = [&](int32_t k) -> size_t {
+        const int32_t cta = i_first + k, slot = k == 0 ? fslot : 0;
+        return ((size_t)cta * 2 + slot) * Hkv;
+    };
+    for (int32_t u = threadIdx.x; u < units; u += blockDim.x) {
+        const int32_t kvl = u / (G * kCols), rem = u - kvl * (G * kCols);
+        const int32_t h = rem / kCols, c4 = rem - h * kCols;
+        const int32_t kvh = gi * 8 + kvl;
+        float m = -INFINITY, W = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int32_t k = k0; k < k1; k += step) {
+            const size_t r = (row_of(k) + kvh) * G + h;
+            const float lse = __ldcg(p.part_lse + r);
+            const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + r * D) + c4);
+            const float mn = fmaxf(m, lse);
+            const float sc = fast_exp2(m - mn), w = fast_exp2(lse - mn);
+            W = W * sc + w;
+            acc.x = acc.x * sc + w * o.x;
+            acc.y = acc.y * sc + w * o.y;
+            acc.z = acc.z * sc + w * o.z;
+            acc.w = acc.w * sc + w * o.w;
+            m = mn;
+        }
+        const float inv = 1.f / W;
+        if (lead < 0) {
+            uint2 packed;
+            packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+            packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+            reinterpret_cast<uint2*>(p.out + ((size_t)b * p.num_q_heads + (size_t)kvh * G + h) * D)[c4] = packed;
+        } else {
+            // the group's state replaces its first piece's (each thread wrote back only what it
+            // read itself; the lse, read by every column, is written after the barrier below)
+            const size_t r = (row_of(lead) + kvh) * G + h;
+            reinterpret_cast<float4*>(p.part_o + r * D)[c4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+            if (c4 == 0) s_lse[kvl * G + h] = m + __log2f(W);
+        }
+    }
+    if (lead >= 0) {
+        __syncthreads();
+        for (int32_t i = threadIdx.x; i < 8 * G; i += blockDim.x)
+            p.part_lse[(row_of(lead) + gi * 8 + i / G) * G + i % G] = s_lse[i];
+    }
+}
+
+// The CTA's share of the merging, after its own pieces are written (called by every thread).
+template <int D>
+__device__ void merge_tail(const DecodeParams& p, const int4* s_cut, const int32_t* s_cut_fslot, bool failed) {
+    __shared__ int32_t s_todo[2], s_final;
+    __shared__ float s_lse[8 * 16];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            const int4 c = s_cut[s];
+            int32_t todo = 0;
+            if (!failed && c.z > 1) {
+                const int32_t n = c.z, i_first = c.w, k = (int32_t)blockIdx.x - i_first;
+                if (n <= kMergeFan) {
+                    todo = counter_add(p.merge_cnt + (size_t)c.y * p.num_seqs + c.x, p.epoch, p.status) == n ? 1 : 0;
+                } else {
+                    const int32_t lead = k / kMergeFan * kMergeFan, size = min(kMergeFan, n - lead);
+                    const int32_t cta = i_first + lead, slot = lead == 0 ? s_cut_fslot[s] : 0;
+                    todo = counter_add(p.group_cnt + (size_t)cta * 2 + slot, p.epoch, p.status) == size ? 2 : 0;
+                }
+            }
+            s_todo[s] = todo;
+        }
+    }
+    __syncthreads();
+    for (int s = 0; s < 2; ++s) {
+        const int32_t todo = s_todo[s];
+        if (todo == 0) continue;
+        const int4 c = s_cut[s];
+        const int32_t n = c.z, i_first = c.w, fslot = s_cut_fslot[s];
+        __threadfence();   // the other pieces' states, counted before this CTA's, are visible
+        if (todo == 1) {
+            merge_pieces<D>(p, c.x, c.y, i_first, fslot, 0, n, 1, -1, s_lse);
+            continue;
+        }
+        const int32_t k = (int32_t)blockIdx.x - i_first, lead = k / kMergeFan * kMergeFan;
+        merge_pieces<D>(p, c.x, c.y, i_first, fslot, lead, min(n, lead + kMergeFan), 1, lead, s_lse);
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+            s_final = counter_add(p.merge_cnt + (size_t)c.y * p.num_seqs + c.x, p.epoch, p.status) ==
+                      (n + kMergeFan - 1) / kMergeFan;
+        __syncthreads();
+        if (s_final) {
+            __threadfence();
+            merge_pieces<D>(p, c.x, c.y, i_first, fslot, 0, n, kMergeFan, -1, s_lse);
+        }
+        __syncthreads();
+    }
+}
+
 template <int D, int NT, bool F8>
 __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     decode_stream_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
@@ -156,6 +284,9 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     __shared__ __align__(8) uint64_t qfull_bar[kQSlots];
     __shared__ __align__(8) uint64_t qempty_bar[kQSlots];
     __shared__ double s_rope_inv[64];   // RoPE inverse frequencies of the D/2 pairs
+    __shared__ int4 s_cut[2];            // per partial slot: {sequence, kv group, pieces, first CTA}
+    __shared__ int32_t s_cut_fslot[2];   //   and the partial slot the sequence's first CTA used
+    __shared__ int32_t s_failed;         // a wait of this CTA gave up: it merges nothing
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t G = p.group;
@@ -179,6 +310,8 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             mbar_init(smem_u32(&qfull_bar[s]), 1);
             mbar_init(smem_u32(&qempty_bar[s]), kGroup);
         }
+        s_cut[0] = s_cut[1] = make_int4(0, 0, 0, 0);
+        s_failed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (p.rope_theta > 0.f)
@@ -188,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     if (warp == kGroup && p.selftest_stall && blockIdx.x == 0) {
         // failure-handling self-test: this CTA's producer issues no copy and signals nothing,
         // so its consumers' first waits run out with no copy in flight
+        if (lane == 0) s_failed = 1;
     } else if (warp == kGroup) {
         // ================================ producer ================================
         const int32_t B = p.num_seqs, Bs = p.block_size;
@@ -291,7 +425,11 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     seg_slot = P < lo ? 0 : 1;
                     seg_ifirst = i_first;
                     seg_fslot = P < (int64_t)i_first * S / Gc ? 0 : 1;
-                    if (P >= lo && lane == 0)   // this CTA holds the sequence's first slab
+                    if (lane == 0 && seg_nsplit > 1) {   // a cut sequence: this CTA holds one piece
+                        s_cut[seg_slot] = make_int4(b, gi, seg_nsplit, i_first);
+                        s_cut_fslot[seg_slot] = seg_fslot;
+                    }
+                    if (!p.inline_merge && P >= lo && lane == 0)   // the merge kernel's descriptor
                         reinterpret_cast<int4*>(p.seq_desc)[(size_t)gi * B + b] =
                             make_int4(seg_nsplit, i_first, seg_fslot, 0);
                     if (s != lo) {
@@ -300,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     }
                     if (L > 0) {
                         int qs;
-                        if (!acquire(qempty_bar, qk, kQSlots, qs)) { alive = false; break; }
+                        if (!acquire(qempty_bar, qk, kQSlots, qs)) { alive = false; s_failed = 1; break; }
                         seg_q = qs;
                         if (lane == 0) {
                             const uint32_t bar = smem_u32(&qfull_bar[qs]);
@@ -313,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     }
                 }
                 int st;
-                if (!acquire(empty_bar, gtile, C::kStages, st)) { alive = false; break; }
+                if (!acquire(empty_bar, gtile, C::kStages, st)) { alive = false; s_failed = 1; break; }
                 const int32_t t0 = j * kSlab;
                 const int32_t valid = L == 0 ? 0 : min(kSlab, L - t0);
                 const uint32_t fbar = smem_u32(&full_bar[st]);
@@ -336,15 +474,33 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                         const size_t row0 = ((size_t)blk * Hkv + gi * kGroup) * Bs + (pos - lbn * Bs);
                         const size_t src0 = ((size_t)b * Hkv + gi * kGroup) * D;
                         if constexpr (F8) {
-                            // E4M3 pools: the new rows quantized with the caches' scales
+                            // E4M3 pools: the new rows quantized with the caches' scales (K first
+                            // turned by RoPE and rounded to bf16 when the call asks for it)
                             uint8_t* kq = reinterpret_cast<uint8_t*>(kc);
                             uint8_t* vq = reinterpret_cast<uint8_t*>(vc);
+                            if (p.rope_theta > 0.f) {
+                                constexpr int kHalfChunks = D / 16;
+                                for (int i = lane; i < kGroup * kHalfChunks; i += 32) {
+                                    const int hh = i / kHalfChunks, cc = i - hh * kHalfChunks;
+                                    float cs[8], sn[8];
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) rope_cos_sin(pos, s_rope_inv[cc * 8 + e], &cs[e], &sn[e]);
+                                    const uint16_t* src = p.k_new + src0 + (size_t)hh * D + cc * 8;
+                                    uint4 x1 = __ldg(reinterpret_cast<const uint4*>(src));
+                                    uint4 x2 = __ldg(reinterpret_cast<const uint4*>(src + D / 2));
+                                    rope_rotate8(x1, x2, cs, sn);
+                                    uint8_t* dst = kq + (row0 + (size_t)hh * Bs) * D + cc * 8;
+                                    *reinterpret_cast<uint2*>(dst) = bf16x8_to_e4m3x8(x1, p.k_inv_scale);
+                                    *reinterpret_cast<uint2*>(dst + D / 2) = bf16x8_to_e4m3x8(x2, p.k_inv_scale);
+                                }
+                            }
                             for (int i = lane; i < kGroup * kChunks; i += 32) {
                                 const int hh = i / kChunks, cc = i - hh * kChunks;
                                 const size_t dst = (row0 + (size_t)hh * Bs) * D + cc * 8;
                                 const size_t src = src0 + (size_t)hh * D + cc * 8;
-                                *reinterpret_cast<uint2*>(kq + dst) = bf16x8_to_e4m3x8(
-                                    __ldg(reinterpret_cast<const uint4*>(p.k_new + src)), p.k_inv_scale);
+                                if (p.rope_theta <= 0.f)
+                                    *reinterpret_cast<uint2*>(kq + dst) = bf16x8_to_e4m3x8(
+                                        __ldg(reinterpret_cast<const uint4*>(p.k_new + src)), p.k_inv_scale);
                                 *reinterpret_cast<uint2*>(vq + dst) = bf16x8_to_e4m3x8(
                                     __ldg(reinterpret_cast<const uint4*>(p.v_new + src)), p.v_inv_scale);
                             }
@@ -450,7 +606,10 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
         const int row_b = stage_row(warp, rr + ((mi >> 1) << 3), tb);    // V: tokens rr (+8)
         for (uint32_t gtile = 0;; ++gtile) {
             const int st = gtile % C::kStages;
-            if (!warp_wait(smem_u32(&full_bar[st]), (gtile / C::kStages) & 1, p.status, p.wait_ns)) break;
+            if (!warp_wait(smem_u32(&full_bar[st]), (gtile / C::kStages) & 1, p.status, p.wait_ns)) {
+                s_failed = 1;
+                break;
+            }
             const Hdr hd = s_hdr[st];
             if (hd.flags & kEnd) break;
             const int32_t kvh = hd.kvh0 + warp;
@@ -462,7 +621,10 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             }
             if (hd.flags & kFirst) {
                 const int qs = qk % kQSlots;
-                if (!warp_wait(smem_u32(&qfull_bar[qs]), (qk / kQSlots) & 1, p.status, p.wait_ns)) break;
+                if (!warp_wait(smem_u32(&qfull_bar[qs]), (qk / kQSlots) & 1, p.status, p.wait_ns)) {
+                    s_failed = 1;
+                    break;
+                }
                 uint16_t* qsm = reinterpret_cast<uint16_t*>(
                     smem_gen + (q_base - smem_base) + qs * (size_t)(kGroup * G * D * 2)) + (size_t)warp * G * D;
                 if (p.rope_theta > 0.f) {
@@ -700,6 +862,11 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     if (r == 0) p.part_lse[prow + h] = m_run[nt][jj] + __log2f(l_run[nt][jj]);
                 }
         }
+    }
+    if (p.inline_merge) {
+        __threadfence();   // this CTA's partial states, before its pieces are counted
+        __syncthreads();
+        merge_tail<D>(p, s_cut, s_cut_fslot, s_failed != 0);
     }
     __syncthreads();
 }

@@ -51,6 +51,10 @@ struct DecodeParams {
     float k_inv_scale, v_inv_scale;  // E4M3: float(1/scale) applied when quantizing new rows
     float out_scale;               // multiplies the normalised output (E4M3: the V scale; else 1)
     int32_t grid;                  // stream kernel: CTAs of the launch (bounds the merge's reads)
+    int32_t inline_merge;          // stream kernel: the last piece of a cut sequence merges it
+    uint32_t epoch;                // call number (counters of earlier calls read as zero)
+    unsigned long long* merge_cnt; // stream kernel: [Hkv/8][B] counters of counted pieces / groups
+    unsigned long long* group_cnt; // stream kernel: [grid][2] counters of a group's counted pieces
     int32_t selftest_stall;        // PA_FLAG_SELFTEST_STALL: CTA 0 of the stream kernel idles
     unsigned long long wait_ns;    // limit of every bounded wait in the stream kernel
 };
@@ -67,7 +71,7 @@ struct DecodePlan {
     int32_t split_tokens;          // kSimt / kSplit: tokens per split
     int32_t max_splits;            // kSimt / kSplit: splits per (sequence, kv head) at most
     int32_t grid;                  // kStream: persistent CTAs (partial slots: 2 per CTA)
-    size_t off_desc, off_lse, off_o, off_qrot, bytes;
+    size_t off_desc, off_lse, off_o, off_qrot, off_mcnt, off_gcnt, bytes;
 };
 
 // Paged prefill: sequence b's last cu_q[b+1] - cu_q[b] tokens attend causally to its
@@ -87,6 +91,9 @@ struct PrefillParams {
 };
 cudaError_t launch_prefill(const PrefillParams& p, int max_q_len, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const PrefillParams& p, int max_q_len, cudaStream_t stream);
+// warp-specialized tcgen05 prefill (TMA block sizes only: 8, 16, 32, 64 or multiples of 64)
+cudaError_t launch_prefill_ws(const PrefillParams& p, int max_q_len, cudaStream_t stream);
+bool prefill_ws_supports(int block_size);
 
 constexpr size_t kWorkspaceAlign = 256;
 // Limits of the decode kernels' bounded waits: normal calls, and PA_FLAG_SELFTEST_STALL calls

@@ -1,0 +1,461 @@
+// Paged (chunked) prefill attention on the fifth-generation tensor cores, warp-specialized.
+//
+// The operation is the one of prefill_tc.cu: sequence b holds L = context_lens[b] tokens
+// after this step's append, its last Tq = cu_q[b+1] - cu_q[b] tokens are the queries
+// (positions L-Tq .. L-1), and the query at position p attends to cache tokens 0..p
+// (Nano-vLLM page, section "Prefill vs Decode"; causal mask: Tiny-vLLM summary page,
+// section "고성능 추론을 위한 고급 최적화 기법").
+//
+// One CTA per (128 query rows, kv head, sequence), 6 warps with one job each, handing work
+// to one another through mbarriers only (no CTA-wide barrier inside the loop):
+//   warps 0-3  softmax: thread i owns row i (tensor-memory lane i).  Per 64-key tile t it
+//              reads its row of S_t from tensor memory, masks it causally, and writes the
+//              probabilities P_t (bf16) into shared memory as the K-major A operand.
+//   warp 4     MMA issue (one thread): S_t = Q K_t^T into tensor memory, then, once P_t is
+//              written, O += P_t V_t, accumulated in tensor memory across tiles, and at once
+//              S_{t+1}, so the next scores are ready when the softmax warps come back.
+//   warp 5     TMA: K and V tiles of 64 keys into a two-stage ring, one box of 64 dims x
+//              min(Bs, 64) tokens per block and 64-dim atom, swizzled by the copy engine; a
+//              stage is refilled once the MMAs that read it have completed.
+// Online softmax with O in tensor memory: a row keeps its running max m until a tile raises
+// it by more than 8 (log2 domain); only then is the row's O scaled by 2^(m - m_new) in
+// tensor memory (load, scale, store) and m replaced.  In between, probabilities are
+// 2^(s - m) <= 2^8, which bf16 and the fp32 sums carry without loss of relative precision.
+// When the scores of tile t are committed, every MMA issued before them (the P V of tile
+// t-1 included) has completed, so O and P may be touched then without another wait.
+//
+// Every wait is bounded (2 s, then the timeout status bit).  On a timeout each warp leaves
+// its loop; the MMA thread drains the TMA copies it has not seen land and waits for its own
+// MMAs, and the tensor memory is freed before the CTA exits.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <cstring>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+#include "pa_ptx.cuh"
+#include "pa_umma.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int kWsRows = 128;     // query rows per CTA (tensor-memory lanes)
+constexpr int kWsKeys = 64;      // keys per tile
+constexpr int kWsThreads = 192;  // 4 softmax warps, the MMA warp, the TMA warp
+constexpr int kWsStages = 2;
+constexpr float kRescaleLog2 = 8.f;
+
+template <int D>
+struct WsCfg {
+    static constexpr int kQBytes = kWsRows * D * 2;
+    static constexpr int kKVBytes = kWsKeys * D * 2;       // one K (or V) tile
+    static constexpr int kPBytes = kWsRows * kWsKeys * 2;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kWsStages * kKVBytes;
+    static constexpr int kOffP = kOffV + kWsStages * kKVBytes;
+    static constexpr int kOffBar = kOffP + kPBytes;
+    // barriers: s_full, p_full, o_final, drain, k_full[2], v_full[2], kv_empty[2]; then the
+    // tensor-memory address and the number of tiles the TMA warp requested
+    static constexpr int kSmem = kOffBar + 128;
+    static constexpr int kColS = 0;                         // S: 64 fp32 columns
+    static constexpr int kColO = 64;                        // O: D fp32 columns
+    static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;
+    // two CTAs per SM: each softmax thread keeps its row of S (64 registers) while it scales
+    // its row of O, which three CTAs of six warps (at most 96 registers a thread) would spill
+    static constexpr int kMinBlocks = 2;
+};
+
+template <int ROWS>
+__device__ __forceinline__ uint32_t ws_sw128(int row, int c) {
+    return (uint32_t)((c >> 3) * (ROWS * 128) + row * 128 + ((((c & 7) ^ (row & 7))) << 4));
+}
+
+__device__ __forceinline__ void ws_cp_async16(uint32_t dst, const void* src, bool live) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(live ? 16 : 0)
+                 : "memory");
+}
+
+// 32 columns of this thread's lane of tensor memory, scaled by a and stored back.
+__device__ __forceinline__ void tmem_scale32(uint32_t taddr, float a) {
+    uint32_t r[32];
+    tmem_ld32(taddr, r);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * a);
+    tmem_st32(taddr, r);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
+    prefill_ws_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap vmap) {
+    using C = WsCfg<D>;
+    constexpr int kCh = D / 8;                               // 16-byte chunks per row
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t s_q = s_base + C::kOffQ, s_k = s_base + C::kOffK, s_v = s_base + C::kOffV;
+    const uint32_t s_p = s_base + C::kOffP;
+    const uint32_t bar_s = s_base + C::kOffBar, bar_p = bar_s + 8, bar_of = bar_s + 16,
+                   bar_drain = bar_s + 24, bar_k = bar_s + 32, bar_v = bar_s + 48, bar_e = bar_s + 64;
+    const uint32_t s_tmem = bar_s + 80;
+    volatile int* s_kreq = reinterpret_cast<volatile int*>(smem + C::kOffBar + 84);
+
+    const int b = blockIdx.z, kvh = blockIdx.y;
+    const int G = p.group, Hq = p.num_q_heads, Hkv = p.num_kv_heads, Bs = p.block_size;
+    const int q0 = p.cu_q[b], Tq = p.cu_q[b + 1] - q0;
+    const int L = p.context_lens[b];
+    const int cap = p.max_blocks_per_seq * Bs;
+    if (Tq <= 0) return;
+    if (L < Tq || L > cap) {
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) raise_status(p.status, kStatusBadLength);
+        return;
+    }
+    if (s_base & 1023u) {                                    // the swizzle needs 1024-byte-aligned tiles
+        if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
+        return;
+    }
+    // the last row tiles of a chunk attend to the most keys: they take the first CTAs
+    const int rows = Tq * G, ntile = (rows + kWsRows - 1) / kWsRows;
+    const int tile = ntile - 1 - (int)blockIdx.x;
+    if (tile < 0) return;
+    const int r0 = tile * kWsRows;
+    const int* table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int last_tok = min(rows - 1, r0 + kWsRows - 1) / G;
+    const int kend = L - Tq + last_tok + 1;                  // keys needed: up to the last row's position
+    const int ntiles = (kend + kWsKeys - 1) / kWsKeys;
+    const int pos_first = L - Tq + r0 / G;
+
+    if (warp == 0) {
+        tmem_alloc(s_tmem, C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_s, 1);
+        mbar_init(bar_p, 4);                                 // one arrival per softmax warp
+        mbar_init(bar_of, 1);
+        mbar_init(bar_drain, 1);
+        for (int i = 0; i < kWsStages; ++i) {
+            mbar_init(bar_k + 8 * i, 1);
+            mbar_init(bar_v + 8 * i, 1);
+            mbar_init(bar_e + 8 * i, 1);
+        }
+        *s_kreq = -1;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp < 4) {                                          // Q rows; rows past the chunk are zeros
+        for (int i = tid; i < kWsRows * kCh; i += 128) {
+            const int row = i / kCh, c = i - row * kCh, R = r0 + row;
+            const bool live = R < rows;
+            const int tok = live ? R / G : 0, g = live ? R - tok * G : 0;
+            const uint16_t* src = p.q + (((size_t)(q0 + tok) * Hq + (size_t)kvh * G + g) * D + c * 8);
+            ws_cp_async16(s_q + ws_sw128<kWsRows>(row, c), src, live);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    uint32_t tmem;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(tmem) : "r"(s_tmem) : "memory");
+    bool failed = false;
+    int k_seen = -1, v_seen = -1;                            // MMA thread: last K / V tile seen landed
+
+    if (warp == 5) {
+        // ================================ TMA ================================
+        const int rb = Bs < kWsKeys ? Bs : kWsKeys, nslot = kWsKeys / rb;
+        for (int t = 0; t < ntiles && !failed; ++t) {
+            const int st = t & 1;
+            if (t >= kWsStages) {                            // the MMAs of tile t-2 have completed
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(bar_e + 8 * st, (uint32_t)(((t >> 1) - 1) & 1), p.status);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    failed = true;
+                    break;
+                }
+            }
+            const int kp = t * kWsKeys + lane * rb;
+            bool valid = lane < nslot && kp < L;
+            int id = valid ? __ldg(table + kp / Bs) : 0;
+            if (valid && (id < 0 || id >= p.num_blocks)) {
+                raise_status(p.status, kStatusBadBlock);
+                valid = false;
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, valid);
+            const uint32_t bytes = (uint32_t)(__popc(m) * rb * 128 * (D / 64));
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar_k + 8 * st, bytes);
+                mbar_arrive_expect_tx(bar_v + 8 * st, bytes);
+                *s_kreq = t;
+            }
+            __syncwarp();
+            if (valid) {
+                const int z = id * Hkv + kvh, y = Bs > kWsKeys ? kp % Bs : 0;
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a) {
+                    const uint32_t off = a * (kWsKeys * 128) + lane * rb * 128;
+                    tma_load_3d(s_k + st * C::kKVBytes + off, &kmap, a * 64, y, z, bar_k + 8 * st);
+                    tma_load_3d(s_v + st * C::kKVBytes + off, &vmap, a * 64, y, z, bar_v + 8 * st);
+                }
+            }
+        }
+    } else if (warp == 4) {
+        // ================================ MMA ================================
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = umma_idesc_bf16(kWsRows, kWsKeys, false);
+            constexpr uint32_t kIdescO = umma_idesc_bf16(kWsRows, D, true);
+            auto wait_k = [&](int t) {
+                if (!mbar_wait(bar_k + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status)) return false;
+                k_seen = t;
+                return true;
+            };
+            auto wait_v = [&](int t) {
+                if (!mbar_wait(bar_v + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status)) return false;
+                v_seen = t;
+                return true;
+            };
+            auto issue_s = [&](int t) {                      // S = Q K_t^T over D / 16 K steps
+                const uint32_t kt = s_k + (t & 1) * C::kKVBytes;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t a = umma_desc_sw128(s_q + (ks >> 2) * (kWsRows * 128) + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(kt + (ks >> 2) * (kWsKeys * 128) + (ks & 3) * 32, 16, 1024);
+                    umma_bf16_ss(tmem + C::kColS, a, bd, kIdescS, ks > 0);
+                }
+            };
+            auto issue_o = [&](int t) {                      // O += P V_t over 4 K steps of 16 keys
+                const uint32_t vt = s_v + (t & 1) * C::kKVBytes;
+#pragma unroll
+                for (int kk = 0; kk < kWsKeys / 16; ++kk) {
+                    const uint64_t a = umma_desc_sw128(s_p + kk * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(vt + kk * 16 * 128, kWsKeys * 128, 1024);
+                    umma_bf16_ss(tmem + C::kColO, a, bd, kIdescO, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+            };
+            if (wait_k(0)) {
+                tc_fence_after_sync();
+                issue_s(0);
+                umma_commit(bar_s);
+                for (int t = 0; t < ntiles; ++t) {
+                    if (!mbar_wait(bar_p, (uint32_t)(t & 1), p.status) || !wait_v(t)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    issue_o(t);
+                    umma_commit(bar_e + 8 * (t & 1));        // K_t and V_t are free once these land
+                    if (t + 1 < ntiles) {
+                        if (!wait_k(t + 1)) {
+                            failed = true;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        issue_s(t + 1);
+                        umma_commit(bar_s);
+                    } else {
+                        umma_commit(bar_of);
+                    }
+                }
+            } else {
+                failed = true;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ============================== softmax ==============================
+        const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's 32 lanes
+        const int R = r0 + tid;
+        const int pos = R < rows ? L - Tq + R / G : L - 1;  // padded rows: computed, not written
+        const float sl2 = p.scale_log2;
+        float m_run = -INFINITY, l_run = 0.f;
+        for (int t = 0; t < ntiles; ++t) {
+            if (!warp_wait(bar_s, (uint32_t)(t & 1), p.status)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after_sync();
+            uint32_t sr[64];
+            tmem_ld64(t_lane + C::kColS, sr);
+            const int k0 = t * kWsKeys;
+            float mx = -INFINITY;
+            if (k0 + kWsKeys - 1 > pos_first) {              // a tile on the diagonal: mask
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const float v = k0 + j <= pos ? __uint_as_float(sr[j]) : -INFINITY;
+                    sr[j] = __float_as_uint(v);
+                    mx = fmaxf(mx, v);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(sr[j]));
+            }
+            // key 0 is in every row's range, so the max is finite from the first tile on
+            const float m_new = fmaxf(m_run, mx * sl2);
+            if (t == 0) {
+                m_run = m_new;
+            } else {
+                const bool need = m_new > m_run + kRescaleLog2;
+                if (__any_sync(0xffffffffu, need)) {
+                    // O of tile t-1 is complete (it was issued before S_t): scale this row
+                    const float a = need ? fast_exp2(m_run - m_new) : 1.f;
+#pragma unroll
+                    for (int h = 0; h < D / 32; ++h) tmem_scale32(t_lane + C::kColO + h * 32, a);
+                    if (need) {
+                        l_run *= a;
+                        m_run = m_new;
+                    }
+                }
+            }
+            float rsum = 0.f;
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * j]), sl2, -m_run));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * j + 1]), sl2, -m_run));
+                rsum += p0 + p1;
+                pk[j] = pack_bf16x2(p0, p1);
+            }
+            l_run += rsum;
+            const uint32_t prow = s_p + tid * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + ((c ^ (tid & 7)) << 4)),
+                             "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                             : "memory");
+            if (L - k0 < kWsKeys) {
+                // the last tile: V rows past the sequence (stale pool rows, or never copied)
+                // are zeroed so that P = 0 there cannot meet a NaN pattern; the MMA reads V
+                // only after all four warps' arrivals below, so each warp zeroes its share
+                if (!warp_wait(bar_v + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status)) {
+                    failed = true;
+                    break;
+                }
+                const uint32_t vt = s_v + (t & 1) * C::kKVBytes;
+                for (int i = tid; i < (kWsKeys - (L - k0)) * (D / 8); i += 128) {
+                    const int row = (L - k0) + i / (D / 8), c = i % (D / 8);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vt + ws_sw128<kWsKeys>(row, c)),
+                                 "r"(0u)
+                                 : "memory");
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_p);
+        }
+        if (!failed && warp_wait(bar_of, 0u, p.status)) {
+            tc_fence_after_sync();
+            const int tok = R / G, g = R - tok * G;
+            const float inv = 1.f / l_run;
+            uint16_t* out = p.out + ((size_t)(q0 + tok) * Hq + (size_t)kvh * G + g) * D;
+#pragma unroll
+            for (int h = 0; h < D / 32; ++h) {
+                uint32_t o[32];
+                tmem_ld32(t_lane + C::kColO + h * 32, o);   // warp-wide: padded rows join the load
+                if (R < rows) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
+                        *reinterpret_cast<uint4*>(out + h * 32 + 8 * c) = w;
+                    }
+                }
+            }
+        }
+    }
+    // every role is done issuing: the MMA thread drains what may still be in flight (after a
+    // timed-out wait: copies requested but never seen to land), then its own MMAs
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 4 && lane == 0) {
+        const int req = *s_kreq;
+        for (int t = k_seen + 1; t <= req; ++t) mbar_wait(bar_k + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status);
+        for (int t = v_seen + 1; t <= req; ++t) mbar_wait(bar_v + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status);
+        umma_commit(bar_drain);
+        mbar_wait(bar_drain, 0u, p.status);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn ws_encode_tiled() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            f = reinterpret_cast<EncodeTiledFn>(ptr);
+            fn.store(f, std::memory_order_release);
+        }
+    }
+    return f;
+}
+
+// The pool as a 3-D bf16 tensor [blocks * Hkv][block_size][head_dim]; box = 64 dims x
+// min(block_size, 64) tokens x 1, in 128-byte-swizzled rows.
+bool ws_pool_map(CUtensorMap* map, const void* base, const PrefillParams& p) {
+    EncodeTiledFn fn = ws_encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)p.head_dim, (cuuint64_t)p.block_size,
+                                (cuuint64_t)p.num_blocks * p.num_kv_heads};
+    const cuuint64_t strides[2] = {(cuuint64_t)p.head_dim * 2, (cuuint64_t)p.block_size * p.head_dim * 2};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)(p.block_size < kWsKeys ? p.block_size : kWsKeys), 1u};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_ws(const PrefillParams& p, int max_q_len, cudaStream_t stream) {
+    constexpr size_t smem = WsCfg<D>::kSmem;
+    static std::atomic<uint64_t> attr_set{0};               // one bit per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!(attr_set.load(std::memory_order_acquire) & (1ull << dev))) {
+        const cudaError_t e = cudaFuncSetAttribute(prefill_ws_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(1ull << dev, std::memory_order_acq_rel);
+    }
+    const int tiles = (max_q_len * p.group + kWsRows - 1) / kWsRows;
+    if (tiles <= 0) return cudaSuccess;
+    CUtensorMap km, vm;
+    memset(&km, 0, sizeof km);
+    memset(&vm, 0, sizeof vm);
+    if (!ws_pool_map(&km, p.k_cache, p) || !ws_pool_map(&vm, p.v_cache, p)) return cudaErrorInvalidValue;
+    dim3 grid((unsigned)tiles, (unsigned)p.num_kv_heads, (unsigned)p.num_seqs);
+    prefill_ws_kernel<D><<<grid, kWsThreads, smem, stream>>>(p, km, vm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_ws_supports(int block_size) {
+    // TMA boxes: the block size tiles the 64-key tile (8, 16, 32, 64) or is a multiple of it
+    return block_size % kWsKeys == 0 || (block_size >= 8 && kWsKeys % block_size == 0);
+}
+
+cudaError_t launch_prefill_ws(const PrefillParams& p, int max_q_len, cudaStream_t stream) {
+    if (p.head_dim == 64) return launch_ws<64>(p, max_q_len, stream);
+    if (p.head_dim == 128) return launch_ws<128>(p, max_q_len, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pa

@@ -167,7 +167,8 @@ def test_prefill_rejects_bad_arguments_without_a_gpu():
         fake, fake, fake, fake, fake, fake, n, mq, ctypes.c_float(scale), fake, ws, wsb, ctypes.byref(dd), kernel,
         None)
     assert call(-1, 4, 0.1, d) == -1
-    assert call(2, 4, 0.1, d, kernel=3) == -1            # unknown kernel
+    assert call(2, 4, 0.1, d, kernel=4) == -1            # unknown kernel
+    assert call(2, 4, 0.1, _desc(block_size=24), kernel=pa.PA_PREFILL_TCGEN05_WS) == -2   # off the 64-key tile
     assert call(2, 4, 0.1, d, kernel=-1) == -1
     assert call(0, 4, 0.1, d, kernel=pa.PA_PREFILL_MMA) == 0
     # the binding refuses an unknown kernel name before it touches any buffer

@@ -139,13 +139,81 @@ def test_e4m3_unsupported_combinations(h):
                      torch.from_numpy(b.context_lens).to(h.DEV), 40, b.scale, torch.empty_like(q), ws, desc,
                      opts)
     assert e.value.status == -2
-    b2 = wl.config2()
-    desc2 = h.desc_of(b2)
+    opts = pa.DecodeOptions(kernel=pa.PA_KERNEL_SIMT, kv_dtype=pa.PA_KV_E4M3, k_scale=1.0, v_scale=1.0)
+    b2 = wl.config2()                                    # the CUDA-core kernel reads bf16 pools only
     kc2 = torch.zeros(b2.k_cache.size, dtype=torch.uint8, device=h.DEV)
-    opts = pa.DecodeOptions(kv_dtype=pa.PA_KV_E4M3, k_scale=1.0, v_scale=1.0, rope_theta=10000.0)
     with pytest.raises(pa.PaError) as e:
-        pa.pa_append_decode(h.to_dev(b2.q), h.to_dev(b2.k_new), h.to_dev(b2.v_new), kc2, kc2,
-                            torch.from_numpy(b2.block_tables).to(h.DEV),
-                            torch.from_numpy(b2.context_lens).to(h.DEV), 2048, b2.scale,
-                            torch.empty_like(h.to_dev(b2.q)), ws, desc2, opts)
+        pa.pa_decode(h.to_dev(b2.q), kc2, kc2, torch.from_numpy(b2.block_tables).to(h.DEV),
+                     torch.from_numpy(b2.context_lens).to(h.DEV), 2048, b2.scale,
+                     torch.empty_like(h.to_dev(b2.q)), ws, h.desc_of(b2), opts)
     assert e.value.status == -2
+
+
+def _bf16_neighbours(bits):
+    """The bf16 patterns one unit in the last place below and above each pattern."""
+    x = np.asarray(bits, dtype=np.uint16).astype(np.int32)
+    o = np.where(x & 0x8000, -(x & 0x7FFF), x & 0x7FFF)          # ordered integer line
+    back = lambda v: np.where(v < 0, 0x8000 | (-v), v).astype(np.uint16)
+    return back(o - 1), back(o + 1)
+
+
+def _rope_codes_allowed(gpu_rows, k_new, positions, theta, ks):
+    """Each E4M3 code of a rotated K row must be the code of a bf16 value within RoPE's bar
+    (2^-8 |exact| + 2^-20 (|x_i| + |x_i+D/2|)) of the exact rotation: the rounded value or a
+    neighbour inside the bar.  Returns the fraction of codes that differ from the oracle's."""
+    exact = oracle.rope(k_new, positions, theta)
+    x = (k_new.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    half = x.shape[-1] // 2
+    mag = np.abs(x[..., :half]) + np.abs(x[..., half:])
+    bound = 2.0 ** -8 * np.abs(exact) + 2.0 ** -20 * np.concatenate([mag, mag], axis=-1)
+    r0 = oracle.round_bf16(exact)
+    lo, hi = _bf16_neighbours(r0)
+    widen = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    allowed = gpu_rows == oracle.quantize_e4m3(r0, ks)
+    for c in (lo, hi):
+        allowed |= (np.abs(widen(c) - exact) <= bound) & (gpu_rows == oracle.quantize_e4m3(c, ks))
+    assert allowed.all(), "a rotated K code no bf16 value within the bar quantizes to"
+    return float(np.mean(gpu_rows != oracle.quantize_e4m3(r0, ks)))
+
+
+@pytest.mark.parametrize("cfg,ctas,pdl", [("c2", 0, True), ("c3", 0, False), ("c4", 0, True),
+                                          ("c2", 7, False)])
+def test_rope_append_decode_e4m3(h, cfg, ctas, pdl):
+    """RoPE on E4M3 pools: q and the new K turned at position L-1 and rounded to bf16, the K row
+    quantized from that bf16 row; against oracle.rope_bf16 then oracle.quantize_e4m3."""
+    theta, ks, vs = 500000.0, 5.0 / 448, 5.0 / 448
+    b = wl.CONFIGS[cfg]()
+    (slots, tables, lens), (o_slots, o_tables, o_lens) = h.host_step(b)
+    kq, vq = _pools(b, ks, vs)
+    desc = h.desc_of(b)
+    kc, vc = _u8(kq, h), _u8(vq, h)
+    q = h.to_dev(b.q)
+    out = torch.empty_like(q)
+    max_len = int(lens.max())
+    opts = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR, kv_dtype=pa.PA_KV_E4M3, k_scale=ks, v_scale=vs,
+                            max_ctas=ctas, rope_theta=theta,
+                            flags=pa.PA_FLAG_CHECK | (pa.PA_FLAG_PDL if pdl else 0))
+    ws = torch.zeros(pa.pa_decode_workspace_size(b.batch, max_len, desc, opts), dtype=torch.uint8,
+                     device=h.DEV)
+    pa.pa_append_decode(q, h.to_dev(b.k_new), h.to_dev(b.v_new), kc, vc, torch.from_numpy(tables).to(h.DEV),
+                        torch.from_numpy(lens).to(h.DEV), max_len, b.scale, out, ws, desc, opts)
+    torch.cuda.synchronize()
+    pos = np.maximum(o_lens - 1, 0).astype(np.int32)
+    q_rot = oracle.rope_bf16(b.q, pos, theta)
+    k_rot = oracle.rope_bf16(b.k_new, pos, theta)
+    rk, rv = oracle.append_kv_e4m3(oracle.quantize_e4m3(k_rot, ks), oracle.quantize_e4m3(b.v_new, vs),
+                                   o_slots, kq, vq)
+    got_k, got_v = kc.cpu().numpy(), vc.cpu().numpy()
+    np.testing.assert_array_equal(got_v, rv)
+    # K: every byte outside the new rows identical; the new rows within the rounding bar
+    mask = h.pool_rows(kq.shape, o_slots)
+    np.testing.assert_array_equal(got_k[~mask], rk[~mask])
+    Bs = b.block_size
+    rows = np.stack([got_k[s // Bs, :, s % Bs, :] for s in o_slots])
+    differ = _rope_codes_allowed(rows, b.k_new, pos, theta, ks)
+    assert differ < 0.01
+    ref = oracle.paged_decode_e4m3(q_rot, rk, rv, ks, vs, o_tables, o_lens, b.scale)
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    ok, ex = oracle.within_tolerance(got, ref)
+    assert ok, "decode outside tolerance by %g" % ex
