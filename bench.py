@@ -232,23 +232,49 @@ def run_reference(args, rank):
     if rank != 0:
         return None
     if args.config == "c5":
+        # each step a bounded sample of a C5 step: the model block manager's step, then the
+        # oracle's decode of layer 0 for the whole batch; the rate is scaled to all 16 layers
         t = wl.Trace5()
-        bm = oracle.BlockManagerModel(t.num_blocks, t.block_size, t.batch, t.max_blocks_per_seq,
-                                      t.free_order)
-        for s in range(t.batch):
-            bm.add_seq(s, int(t.initial_lens[s]))
-        bm.append_tokens(list(range(t.batch)))
-        tables = np.array([[bm.table_array(s) for s in range(t.batch)]], dtype=np.int32)
-        lens = np.array([bm.lens], dtype=np.int32)
-        t.steps = 1
-        cb = cpu_baseline_c5(t, tables, lens, max(1.0, args.cpu_seconds))
-        return {"metric": METRIC, "value": cb["value"], "unit": "seq-steps/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / cb["value"],
+        events = list(t.events())
+        kc, vc = t.pool(0)
+        q, _, _ = t.token_inputs(0, 0)
+        st = {}
+
+        def sample(i):
+            if i % t.steps == 0:                     # the trace (re)starts: a fresh manager
+                st["bm"] = oracle.BlockManagerModel(t.num_blocks, t.block_size, t.batch,
+                                                    t.max_blocks_per_seq, t.free_order)
+                for s in range(t.batch):
+                    st["bm"].add_seq(s, int(t.initial_lens[s]))
+            bm = st["bm"]
+            _, retired, admitted = events[i % t.steps]
+            for s in retired:
+                bm.free_seq(s)
+            for s, n in admitted:
+                bm.add_seq(s, n)
+            bm.append_tokens(list(range(t.batch)))
+            tables = np.array([bm.table_array(s) for s in range(t.batch)], dtype=np.int32)
+            oracle.paged_decode(q, kc, vc, tables, np.array(bm.lens, dtype=np.int32), t.scale)
+
+        W, K = args.warmup, args.steps
+        for i in range(W):
+            sample(i)
+        t0 = time.perf_counter()
+        for i in range(W, W + K):
+            sample(i)
+        dt = time.perf_counter() - t0
+        value = t.batch * K / dt / t.layers
+        cb = {"value": value, "unit": "seq-steps/s", "cores": oracle.num_threads(), "kind": "oracle",
+              "sample": "%d trace steps (after %d warm-up steps): the model block manager's step and the "
+                        "oracle decode of layer 0 for all 256 sequences, %.1f s; the rate is scaled to all "
+                        "%d layers" % (K, W, dt, t.layers)}
+        return {"metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": args.gpus,
+                "steps": K, "warmup": W, "ms_per_step": 1e3 * dt / K * t.layers,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "impl": "reference",
                 "config": {"workload": WORKLOAD_TEXT["c5"], "config": "c5", "batch": t.batch},
                 "cpu_baseline": cb,
-                "e2e": {"value": cb["value"], "unit": "seq-steps/s", "h2d_bytes_per_step": 0,
+                "e2e": {"value": value, "unit": "seq-steps/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
     if args.config == "pc":
         # the model of the prefix-caching manager admitting the C3 request mix by token ids
@@ -385,6 +411,57 @@ def _pack(specs, device):
     return h_buf, d_buf, views
 
 
+def run_e2e(E, warm, stream, stage, h_in, h_outs, compute, dist, dev, host_fill=None):
+    """Times E end-to-end steps.  Step i copies its inputs from pinned host memory (h_in, or
+    what host_fill(i) returns) into device staging buffer i % 2 on a copy stream, runs compute(i,
+    bufs) on `stream` once that copy has landed, and copies the step's output (the last entry of
+    bufs) back into pinned h_outs[i % 2] on the copy stream.  A staging buffer is refilled only
+    after the step two back has finished with it.  CUDA events on `stream` bracket the whole,
+    max over ranks."""
+    import torch
+    cs = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def step(i):
+        j = i & 1
+        d_buf, bufs = stage[j]
+        if host_fill is not None:
+            ev_in[j].synchronize()                      # the copy of step i - 2 has left its host buffer
+            src = host_fill(i)
+        else:
+            src = h_in
+        with torch.cuda.stream(cs):
+            cs.wait_event(ev_out[j])                    # step i - 2 is done with these buffers
+            d_buf.copy_(src, non_blocking=True)
+            ev_in[j].record(cs)
+        stream.wait_event(ev_in[j])
+        compute(i, bufs)
+        ev_done[j].record(stream)
+        with torch.cuda.stream(cs):
+            cs.wait_event(ev_done[j])
+            h_outs[j].copy_(bufs[-1], non_blocking=True)
+            ev_out[j].record(cs)
+
+    for i in range(warm):
+        step(i)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    cs.wait_event(e0)                                   # no copy of the timed steps starts earlier
+    for i in range(E):
+        step(warm + i)
+    stream.wait_event(ev_out[(warm + E - 1) & 1])       # the last step's output is on the host
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms, = max_over_ranks([e0.elapsed_time(e1)], dist, dev)
+    return ms
+
+
 def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_steps=None, kv=None,
                with_cpu=True):
     """A decode configuration (c1..c4): one step = pa_append_decode (or the separate calls) of
@@ -464,7 +541,10 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
     pos_d = torch.from_numpy(np.maximum(lens - 1, 0).astype(np.int32)).to(dev)
     q_rot = torch.empty_like(q)
 
-    def call(L, ev=None):
+    resident = (q, k_new, v_new, slots_d, tables_d, lens_d, out)
+
+    def call(L, ev=None, bufs=resident):
+        q, k_new, v_new, slots_d, tables_d, lens_d, out = bufs
         if fused:
             if ev is not None:
                 ev[0].record(stream)
@@ -528,32 +608,22 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
         raise RuntimeError("decode reported %s during timing" % pa.pa_status_string(rc))
     value = world * B * K / (elapsed_ms / 1e3)
 
-    # ---- e2e: the step's inputs up from pinned host memory in one copy, the output back in one
+    # ---- e2e: every step's inputs up from pinned host memory in one copy, its output back in
+    # one, on a copy stream that runs a step ahead of the compute (two device staging buffers)
     e2e = None
     if E > 0:
-        h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
-
-        def e2e_step(i):
-            d_buf.copy_(h_buf, non_blocking=True)
-            call(i % layers)
-            h_out.copy_(out, non_blocking=True)
-
-        for i in range(min(W, 20)):
-            e2e_step(i)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(E):
-            e2e_step(i)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms, = max_over_ranks([e0.elapsed_time(e1)], dist, dev)
+        _, d_buf2, io2 = _pack([("q", b.q), ("k", b.k_new), ("v", b.v_new), ("slots", slots),
+                                ("tables", tables), ("lens", lens)], dev)
+        out2 = torch.empty_like(out)
+        stage = [(d_buf, resident), (d_buf2, tuple(io2[n][1] for n in ("q", "k", "v", "slots", "tables",
+                                                                       "lens")) + (out2,))]
+        h_outs = [torch.empty(out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        e2e_ms = run_e2e(E, min(W, 20), stream, stage, h_buf, h_outs,
+                         lambda i, bufs: call(i % layers, bufs=bufs), dist, dev)
         e2e = {"value": world * B * E / (e2e_ms / 1e3), "unit": "seq-steps/s",
-               "h2d_bytes_per_step": int(h_buf.numel()), "d2h_bytes_per_step": int(h_out.numel() * 2),
-               "copies_per_step": {"h2d": 1, "d2h": 1}, "steps": E}
+               "h2d_bytes_per_step": int(h_buf.numel()), "d2h_bytes_per_step": int(h_outs[0].numel() * 2),
+               "copies_per_step": {"h2d": 1, "d2h": 1}, "steps": E,
+               "overlap": "copies on a second stream, one step ahead of the compute"}
 
     if rank != 0:
         return None
@@ -594,9 +664,10 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
         "kv_read_gbs_step": kv_bytes * K / (elapsed_ms / 1e3) / 1e9,
         "e2e": e2e,
         # per step: the append (its own kernel unless the stream kernel fuses it), the decode
-        # kernel and (when any sequence can be cut) the merge kernel
+        # kernel and (split kernels, when a sequence can be cut) the merge kernel; the stream
+        # kernel merges cut sequences itself
         "gpu_launches": K * ((0 if (fused and kernel_name == "tensor") else 1) + 1 +
-                             (1 if (kernel_name == "tensor" or plan.max_splits > 1) else 0)),
+                             (1 if (kernel_name != "tensor" and plan.max_splits > 1) else 0)),
         "clocks": clk,
     }
     if with_cpu and not args.no_cpu_baseline and world == 1:
@@ -761,39 +832,37 @@ def run_c5(args, rank, world, dist):
         raise RuntimeError("decode reported %s during timing" % pa.pa_status_string(rc))
 
     # e2e: the host block manager replays the trace inside the timed region.  Per step one copy
-    # up (table rows, lengths, every layer's q/k/v) and one copy down (every layer's output),
-    # through two pinned staging buffers so that the host prepares step i+1 while step i runs.
-    E = min(args.e2e_steps, S)
-    stage = []
+    # up (table rows, lengths, every layer's q/k/v) and one copy down (every layer's output), on
+    # a copy stream a step ahead of the compute; the host fills one of two pinned staging
+    # buffers while the other's step runs.
+    warm = min(args.warmup, 20)
+    E = max(1, min(args.e2e_steps, S - warm))
+    hosts, stage, mx_of = [], [], [0, 0]
     for _ in range(2):
         hb, db, v2 = _pack([("tables", tables[0]), ("lens", lens[0])] +
                            [(n % l, a) for l in range(NL) for n, a in zip(("q%d", "k%d", "v%d"), tok[l])], dev)
-        stage.append((hb, db, v2, torch.cuda.Event()))
+        o = torch.empty_like(outs_all)
+        hosts.append((hb, v2))
+        stage.append((db, (v2, o)))
     h_outs = [torch.empty(outs_all.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for step, bm in replay():
-        if step >= E:
-            break
-        hb, db, v2, done = stage[step & 1]
-        done.synchronize()                       # the copy that last read this staging buffer is over
+    trace = replay()
+
+    def host_fill(i):
+        step, bm = next(trace)                   # retire, admit, append: the host manager's step
+        hb, v2 = hosts[i & 1]
         v2["tables"][0][...] = bm.block_tables()
         v2["lens"][0][...] = bm.context_lens()
-        mx = int(v2["lens"][0].max())
-        db.copy_(hb, non_blocking=True)
+        mx_of[i & 1] = int(v2["lens"][0].max())
+        return hb
+
+    def compute(i, bufs):
+        v2, o = bufs
         for layer in range(NL):
             pa.pa_append_decode(v2["q%d" % layer][1], v2["k%d" % layer][1], v2["v%d" % layer][1],
-                                kcs[layer], vcs[layer], v2["tables"][1], v2["lens"][1], mx, t.scale,
-                                outs[layer], ws, desc, opts, stream=stream)
-        h_outs[step & 1].copy_(outs_all, non_blocking=True)
-        done.record(stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms, = max_over_ranks([e2e_ms], dist, dev)
+                                kcs[layer], vcs[layer], v2["tables"][1], v2["lens"][1], mx_of[i & 1], t.scale,
+                                o[layer], ws, desc, opts, stream=stream)
+
+    e2e_ms = run_e2e(E, warm, stream, stage, None, h_outs, compute, dist, dev, host_fill=host_fill)
     if rank != 0:
         return None
     peak, peak_kind = measured_peaks()
@@ -819,11 +888,12 @@ def run_c5(args, rank, world, dist):
                      "avg_launch_ms": float(call_ms.mean()),
                      "launch_timing": "timed region / calls" if pdl else "CUDA events around each call"},
         "e2e": {"value": world * B * E / (e2e_ms / 1e3), "unit": "seq-steps/s",
-                "h2d_bytes_per_step": int(stage[0][0].numel()),
+                "h2d_bytes_per_step": int(hosts[0][0].numel()),
                 "d2h_bytes_per_step": int(h_outs[0].numel() * 2),
                 "copies_per_step": {"h2d": 1, "d2h": 1}, "steps": E,
-                "includes": "host block manager (retire, admit, append) per step"},
-        "gpu_launches": K * NL * 2,
+                "includes": "host block manager (retire, admit, append) per step",
+                "overlap": "copies on a second stream, one step ahead of the compute"},
+        "gpu_launches": K * NL * (1 if kernel_name == "tensor" else 2),   # one fused call per layer
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:
