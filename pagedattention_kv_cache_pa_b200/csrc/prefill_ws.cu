@@ -78,6 +78,18 @@ __device__ __forceinline__ void ws_cp_async16(uint32_t dst, const void* src, boo
                  : "memory");
 }
 
+// 2^x on the FMA pipe, for x <= 8: x = n + f with n = floor(x), 2^f from a cubic fitted to
+// it on [0, 1) (relative error below 9e-5, under the bf16 rounding the probabilities get), and
+// n added to the exponent field.  0 below 2^-126.  Some of each row's exponentials take this
+// path so that they do not all queue on the special-function unit.
+__device__ __forceinline__ float exp2_fma(float x) {
+    const float xc = fmaxf(x, -126.f);
+    const float n = floorf(xc), f = xc - n;
+    const float p = fmaf(fmaf(fmaf(0.0770652f, f, 0.227647f), f, 0.69511634f), f, 1.f);
+    const float r = __int_as_float(__float_as_int(p) + ((int)n << 23));
+    return x < -126.f ? 0.f : r;
+}
+
 // 32 columns of this thread's lane of tensor memory, scaled by a and stored back.
 __device__ __forceinline__ void tmem_scale32(uint32_t taddr, float a) {
     uint32_t r[32];
@@ -87,7 +99,7 @@ __device__ __forceinline__ void tmem_scale32(uint32_t taddr, float a) {
     tmem_st32(taddr, r);
 }
 
-template <int D>
+template <int D, int kPolyPairs>
 __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
     prefill_ws_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap) {
@@ -313,8 +325,10 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
             uint32_t pk[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * j]), sl2, -m_run));
-                const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * j + 1]), sl2, -m_run));
+                const float x0 = fmaf(__uint_as_float(sr[2 * j]), sl2, -m_run);
+                const float x1 = fmaf(__uint_as_float(sr[2 * j + 1]), sl2, -m_run);
+                const float p0 = j < kPolyPairs ? exp2_fma(x0) : fast_exp2(x0);
+                const float p1 = j < kPolyPairs ? exp2_fma(x1) : fast_exp2(x1);
                 rsum += p0 + p1;
                 pk[j] = pack_bf16x2(p0, p1);
             }
@@ -422,15 +436,18 @@ bool ws_pool_map(CUtensorMap* map, const void* base, const PrefillParams& p) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+// Pairs of each row's 64 exponentials per tile computed on the FMA pipe (exp2_fma).
+constexpr int kWsPolyPairs = 0;
+
+template <int D, int kPoly = kWsPolyPairs>
 cudaError_t launch_ws(const PrefillParams& p, int max_q_len, cudaStream_t stream) {
     constexpr size_t smem = WsCfg<D>::kSmem;
     static std::atomic<uint64_t> attr_set{0};               // one bit per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!(attr_set.load(std::memory_order_acquire) & (1ull << dev))) {
-        const cudaError_t e = cudaFuncSetAttribute(prefill_ws_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)smem);
+        const cudaError_t e = cudaFuncSetAttribute(prefill_ws_kernel<D, kPoly>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_set.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
@@ -441,7 +458,7 @@ cudaError_t launch_ws(const PrefillParams& p, int max_q_len, cudaStream_t stream
     memset(&vm, 0, sizeof vm);
     if (!ws_pool_map(&km, p.k_cache, p) || !ws_pool_map(&vm, p.v_cache, p)) return cudaErrorInvalidValue;
     dim3 grid((unsigned)tiles, (unsigned)p.num_kv_heads, (unsigned)p.num_seqs);
-    prefill_ws_kernel<D><<<grid, kWsThreads, smem, stream>>>(p, km, vm);
+    prefill_ws_kernel<D, kPoly><<<grid, kWsThreads, smem, stream>>>(p, km, vm);
     return cudaGetLastError();
 }
 
