@@ -96,6 +96,10 @@ def parse_args(argv=None):
     ap.add_argument("--rope", type=float, default=0.0,
                     help="RoPE frequency base for the fused call (q and the new K turned at position "
                          "L-1); 0 = no rotation")
+    ap.add_argument("--graphs", choices=["on", "off"], default="on",
+                    help="time the device-resident steps as replays of CUDA graphs captured from "
+                         "the same library calls (host launch cost out of the timed region); "
+                         "needs --pdl on")
     ap.add_argument("--pdl", choices=["on", "off"], default="on",
                     help="PA_FLAG_PDL: the tensor kernel plans its work while the previous kernel "
                          "runs; tables and lengths are written once before the timed region, as "
@@ -411,6 +415,18 @@ def _pack(specs, device):
     return h_buf, d_buf, views
 
 
+def capture_graph(fn, dev):
+    """A CUDA graph of the library calls fn() makes (captured on a side stream; the calls take
+    the current stream, which is the capture stream inside the capture)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def run_e2e(E, warm, stream, stage, h_in, h_outs, compute, dist, dev, host_fill=None):
     """Times E end-to-end steps.  Step i copies its inputs from pinned host memory (h_in, or
     what host_fill(i) returns) into device staging buffer i % 2 on a copy stream, runs compute(i,
@@ -545,6 +561,7 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
 
     def call(L, ev=None, bufs=resident):
         q, k_new, v_new, slots_d, tables_d, lens_d, out = bufs
+        stream = torch.cuda.current_stream(dev)        # the capture stream while capturing
         if fused:
             if ev is not None:
                 ev[0].record(stream)
@@ -577,8 +594,26 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
         raise RuntimeError("decode reported %s" % pa.pa_status_string(rc))
 
     settle(lambda i: call(i % layers))
+    graphs = args.graphs == "on" and pdl
+    if graphs:
+        # one graph of `layers` calls (one per pool, back to back as the loop below issues them)
+        # and one of the remainder: K calls = K // layers full replays + the remainder
+        full = capture_graph(lambda: [call(L) for L in range(layers)], dev)
+        rem = capture_graph(lambda: [call(L) for L in range(K % layers)], dev) if K % layers else None
+        launch_desc = "CUDA graphs of the library calls: %d calls per replay" % layers
+
+        def timed_steps(n):
+            for _ in range(n // layers):
+                full.replay()
+            if n % layers:
+                (rem if n % layers == K % layers else
+                 capture_graph(lambda: [call(L) for L in range(n % layers)], dev)).replay()
+    else:
+        launch_desc = "direct calls"
     for i in range(W):
         call(i % layers)
+    if graphs:
+        timed_steps(W)
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -588,8 +623,11 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
     torch.cuda.synchronize()
     clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
     t_start.record(stream)
-    for i in range(K):
-        call(i % layers, None if pdl else ev_dec[i])
+    if graphs:
+        timed_steps(K)
+    else:
+        for i in range(K):
+            call(i % layers, None if pdl else ev_dec[i])
     t_end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -647,7 +685,7 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
                    "split_tokens": args.split_tokens or "auto", "max_splits": plan.max_splits,
                    "call": "pa_append_decode" if fused else
                            ("pa_rope_append_kv + pa_decode" if args.rope > 0 else "pa_append_kv + pa_decode"),
-                   "pdl": pdl, "rope_theta": args.rope, "kv_dtype": kv,
+                   "pdl": pdl, "launch": launch_desc, "rope_theta": args.rope, "kv_dtype": kv,
                    "l2": "inputs larger than L2: %d rotating layer pools of %.0f MB" % (layers, pool_bytes / 1e6),
                    "parallelism": "replicas x%d" % world},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -781,7 +819,7 @@ def run_c5(args, rank, world, dist):
         pa.pa_append_decode(qs[layer], ks[layer], vs[layer], kcs[layer], vcs[layer],
                             tables_d[s] if tb is None else tb, lens_d[s] if ln is None else ln,
                             step_max[s] if mx is None else mx, t.scale, outs[layer], ws, desc, opts,
-                            stream=stream)
+                            stream=torch.cuda.current_stream(dev))
 
     def trace_step(i):
         for layer in range(NL):
@@ -794,6 +832,14 @@ def run_c5(args, rank, world, dist):
         raise RuntimeError("decode reported %s" % pa.pa_status_string(rc))
     K, W = args.steps, args.warmup
     settle(trace_step)
+    graphs = args.graphs == "on" and pdl
+    if graphs:
+        # one graph per trace step: its 16 layer calls, with that step's tables and lengths
+        step_graphs = [capture_graph(lambda s=s: [call(s, layer) for layer in range(NL)], dev) for s in range(S)]
+        trace_step = lambda i: step_graphs[i % S].replay()       # noqa: E731
+        launch_desc = "CUDA graphs of the library calls: one per trace step (16 calls)"
+    else:
+        launch_desc = "direct calls"
     for i in range(W):
         trace_step(i)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -805,6 +851,9 @@ def run_c5(args, rank, world, dist):
     clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
     t0e.record(stream)
     for i in range(K):
+        if graphs:
+            trace_step(i)
+            continue
         s = i % S
         for layer in range(NL):
             if not pdl:
@@ -875,7 +924,7 @@ def run_c5(args, rank, world, dist):
                    "trace_steps": S, "step": "one decode step of all 16 layers (trace replayed as needed)",
                    "num_blocks": N, "mean_context": float(lens.mean()),
                    "decode_kernel": kernel_name, "ctas": plan.ctas, "call": "pa_append_decode per layer",
-                   "pdl": pdl, "rope_theta": args.rope,
+                   "pdl": pdl, "launch": launch_desc, "rope_theta": args.rope,
                    "l2": "inputs larger than L2: 16 layer pools of %.0f MB" % (2 * kcs[0].numel() * 2 / 1e6),
                    "parallelism": "replicas x%d" % world},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",

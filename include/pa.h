@@ -206,10 +206,11 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * workspace: caller-owned device buffer of at least
  * pa_decode_workspace_size(...) bytes, 256-byte aligned, ZERO-FILLED BEFORE
  * ITS FIRST USE.  The kernels leave their work counters at zero when they
- * complete, and the merge counters of the whole-group tensor kernel carry the
- * call's number (so a workspace left by a call that gave up on a wait serves
- * the next call as it is); the buffer can be reused by later calls without
- * clearing.  Calls that may overlap on the GPU need separate workspaces.
+ * complete, and the merge counters of the whole-group tensor kernel carry a
+ * launch number kept in the workspace (so a workspace left by a call that gave
+ * up on a wait, or replayed in a captured graph, serves the next launch as it
+ * is); the buffer can be reused by later calls without clearing.  Calls that
+ * may overlap on the GPU need separate workspaces.
  *
  * Built shapes: head_dim 64 or 128; block_size 8, 16, 32, 64, 128 or 256;
  * Hq / Hkv <= 16.  Others return PA_ERR_UNSUPPORTED.  The tensor-core

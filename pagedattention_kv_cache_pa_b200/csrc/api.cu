@@ -46,15 +46,6 @@ int32_t env_split_tokens() {
     return v;
 }
 
-// Call numbers for the stream kernel's merge counters: never 0 (a zero-filled workspace holds
-// counters of call 0), distinct for 2^32 - 1 calls in a row.
-uint32_t next_epoch() {
-    static std::atomic<uint32_t> n{0};
-    uint32_t e = n.fetch_add(1, std::memory_order_relaxed) + 1;
-    if (e == 0) e = n.fetch_add(1, std::memory_order_relaxed) + 1;
-    return e;
-}
-
 int32_t env_kernel() {
     static int32_t v = [] {
         const char* s = getenv("PA_DECODE_KERNEL");
@@ -94,7 +85,8 @@ int num_sms_current_device(int* out) {
 //    ceil(max_context_len / C) per (sequence, kv head).  Automatic C: enough
 //    work items for about 32 per SM if every sequence were max_context_len
 //    long, never below 128 tokens.
-// Workspace: [0, 256) status word and work counters; (kStream) one piece
+// Workspace: [0, 256) status word, work counters, the stream kernel's launch number and
+// finished-CTA count (words 0-4); (kStream) one piece
 // descriptor per (kv group, sequence); partial log-sum-exps; partial outputs.
 int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc& d,
                      const pa_decode_options* opt, DecodePlan* plan) {
@@ -388,7 +380,8 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     DecodeParams p;
     p.grid = plan.grid;
     p.inline_merge = plan.kernel == DecodeKernel::kStream ? 1 : 0;
-    p.epoch = next_epoch();
+    p.epoch = reinterpret_cast<uint32_t*>(ws) + 3;
+    p.stream_done = reinterpret_cast<int32_t*>(ws) + 4;
     p.merge_cnt = reinterpret_cast<unsigned long long*>(ws + plan.off_mcnt);
     p.group_cnt = reinterpret_cast<unsigned long long*>(ws + plan.off_gcnt);
     p.selftest_stall = stall ? 1 : 0;

@@ -153,8 +153,10 @@ __device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 x, float inv_scale) {
 // merged in two levels: the pieces are counted per group of kMergeFan on a counter of the
 // group's first piece; the CTA completing a group merges it into that first piece's rows and
 // counts the group on the sequence's counter, and the CTA completing that merges the groups.
-// Counters hold (call number << 32 | count): a counter left by an earlier call (one that gave
-// up on a wait, say) reads as zero, so they never need clearing.
+// Counters hold (launch number << 32 | count): a counter left by an earlier launch (one that
+// gave up on a wait, say) reads as zero, so they never need clearing.  The launch number lives
+// in the workspace; the last CTA of a launch to finish advances it, so every launch, and every
+// replay of a captured graph, counts under a number of its own.
 constexpr int32_t kMergeFan = 16;
 
 __device__ __forceinline__ int32_t counter_add(unsigned long long* c, uint32_t epoch, int32_t* status) {
@@ -170,76 +172,97 @@ __device__ __forceinline__ int32_t counter_add(unsigned long long* c, uint32_t e
     return -1;
 }
 
-// Merges pieces k = k0, k0 + step, ... < k1 of one sequence for the 8 kv heads of group gi:
-// into out (bf16) when lead < 0, else into the partial rows of piece `lead` (fp32 + lse).
+// Merges pieces k = k0, k0 + step, ... < k1 (at most kMergeInputs of them) of one sequence for
+// the 8 kv heads of group gi: into out (bf16) when lead < 0, else into the partial rows of piece
+// `lead` (fp32 state + lse).  Three phases, so that every load of a phase is independent of the
+// others: (1) one thread per query head loads the pieces' lse values into shared memory, (2)
+// turns them into normalised weights 2^(lse_k - M) / W, (3) every thread accumulates its float4
+// columns over the pieces with those weights.  `scratch` is the CTA's stage memory, idle once
+// its slice is streamed.
+constexpr int32_t kMergeInputs = 32;
+
 template <int D>
 __device__ void merge_pieces(const DecodeParams& p, int32_t b, int32_t gi, int32_t i_first, int32_t fslot,
-                             int32_t k0, int32_t k1, int32_t step, int32_t lead, float* s_lse) {
-    const int32_t G = p.group, Hkv = p.num_kv_heads;
+                             int32_t k0, int32_t k1, int32_t step, int32_t lead, float* scratch) {
+    const int32_t G = p.group, Hkv = p.num_kv_heads, HG = 8 * G;
     constexpr int kCols = D / 4;
-    const int32_t units = 8 * G * kCols;
+    const int32_t np = (k1 - k0 + step - 1) / step;
+    float* s_w = scratch;                       // [np][HG] weights
+    float* s_lse = scratch + kMergeInputs * 128; // [HG] the merged lse (group merges)
     auto row_of = [&](int32_t k) -> size_t {
         const int32_t cta = i_first + k, slot = k == 0 ? fslot : 0;
         return ((size_t)cta * 2 + slot) * Hkv;
     };
+    for (int32_t t = threadIdx.x; t < HG; t += blockDim.x) {
+        const int32_t kvh = gi * 8 + t / G, h = t % G;
+        float m = -INFINITY;
+#pragma unroll 4
+        for (int32_t i = 0; i < np; ++i) {
+            const float lse = __ldcg(p.part_lse + (row_of(k0 + i * step) + kvh) * G + h);
+            s_w[i * HG + t] = lse;
+            m = fmaxf(m, lse);
+        }
+        float W = 0.f;
+        for (int32_t i = 0; i < np; ++i) W += fast_exp2(s_w[i * HG + t] - m);
+        const float inv = 1.f / W;
+        for (int32_t i = 0; i < np; ++i) s_w[i * HG + t] = fast_exp2(s_w[i * HG + t] - m) * inv;
+        s_lse[t] = m + __log2f(W);
+    }
+    __syncthreads();
+    const int32_t units = HG * kCols;
     for (int32_t u = threadIdx.x; u < units; u += blockDim.x) {
-        const int32_t kvl = u / (G * kCols), rem = u - kvl * (G * kCols);
-        const int32_t h = rem / kCols, c4 = rem - h * kCols;
-        const int32_t kvh = gi * 8 + kvl;
-        float m = -INFINITY, W = 0.f;
+        const int32_t t = u / kCols, c4 = u - t * kCols;
+        const int32_t kvh = gi * 8 + t / G, h = t % G;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-        for (int32_t k = k0; k < k1; k += step) {
-            const size_t r = (row_of(k) + kvh) * G + h;
-            const float lse = __ldcg(p.part_lse + r);
+        for (int32_t i = 0; i < np; ++i) {
+            const size_t r = (row_of(k0 + i * step) + kvh) * G + h;
             const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + r * D) + c4);
-            const float mn = fmaxf(m, lse);
-            const float sc = fast_exp2(m - mn), w = fast_exp2(lse - mn);
-            W = W * sc + w;
-            acc.x = acc.x * sc + w * o.x;
-            acc.y = acc.y * sc + w * o.y;
-            acc.z = acc.z * sc + w * o.z;
-            acc.w = acc.w * sc + w * o.w;
-            m = mn;
+            const float w = s_w[i * HG + t];
+            acc.x = fmaf(w, o.x, acc.x);
+            acc.y = fmaf(w, o.y, acc.y);
+            acc.z = fmaf(w, o.z, acc.z);
+            acc.w = fmaf(w, o.w, acc.w);
         }
-        const float inv = 1.f / W;
         if (lead < 0) {
             uint2 packed;
-            packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-            packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+            packed.x = pack_bf16x2(acc.x, acc.y);
+            packed.y = pack_bf16x2(acc.z, acc.w);
             reinterpret_cast<uint2*>(p.out + ((size_t)b * p.num_q_heads + (size_t)kvh * G + h) * D)[c4] = packed;
         } else {
-            // the group's state replaces its first piece's (each thread wrote back only what it
-            // read itself; the lse, read by every column, is written after the barrier below)
+            // the group's state replaces its first piece's (each thread writes back only the
+            // columns it read itself)
             const size_t r = (row_of(lead) + kvh) * G + h;
-            reinterpret_cast<float4*>(p.part_o + r * D)[c4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-            if (c4 == 0) s_lse[kvl * G + h] = m + __log2f(W);
+            reinterpret_cast<float4*>(p.part_o + r * D)[c4] = acc;
         }
     }
     if (lead >= 0) {
-        __syncthreads();
-        for (int32_t i = threadIdx.x; i < 8 * G; i += blockDim.x)
-            p.part_lse[(row_of(lead) + gi * 8 + i / G) * G + i % G] = s_lse[i];
+        for (int32_t t = threadIdx.x; t < HG; t += blockDim.x)
+            p.part_lse[(row_of(lead) + gi * 8 + t / G) * G + t % G] = s_lse[t];
     }
+    __syncthreads();                            // scratch free again
 }
 
 // The CTA's share of the merging, after its own pieces are written (called by every thread).
 template <int D>
-__device__ void merge_tail(const DecodeParams& p, const int4* s_cut, const int32_t* s_cut_fslot, bool failed) {
+__device__ void merge_tail(const DecodeParams& p, const int4* s_cut, const int32_t* s_cut_fslot, bool failed,
+                           float* scratch) {
     __shared__ int32_t s_todo[2], s_final;
-    __shared__ float s_lse[8 * 16];
+    __shared__ uint32_t s_epoch;
     if (threadIdx.x == 0) {
+        // advanced only after every CTA of this launch has finished: one value for all of them
+        s_epoch = *reinterpret_cast<volatile uint32_t*>(p.epoch);
         for (int s = 0; s < 2; ++s) {
             const int4 c = s_cut[s];
             int32_t todo = 0;
             if (!failed && c.z > 1) {
                 const int32_t n = c.z, i_first = c.w, k = (int32_t)blockIdx.x - i_first;
                 if (n <= kMergeFan) {
-                    todo = counter_add(p.merge_cnt + (size_t)c.y * p.num_seqs + c.x, p.epoch, p.status) == n ? 1 : 0;
+                    todo = counter_add(p.merge_cnt + (size_t)c.y * p.num_seqs + c.x, s_epoch, p.status) == n ? 1 : 0;
                 } else {
                     const int32_t lead = k / kMergeFan * kMergeFan, size = min(kMergeFan, n - lead);
                     const int32_t cta = i_first + lead, slot = lead == 0 ? s_cut_fslot[s] : 0;
-                    todo = counter_add(p.group_cnt + (size_t)cta * 2 + slot, p.epoch, p.status) == size ? 2 : 0;
+                    todo = counter_add(p.group_cnt + (size_t)cta * 2 + slot, s_epoch, p.status) == size ? 2 : 0;
                 }
             }
             s_todo[s] = todo;
@@ -253,20 +276,20 @@ __device__ void merge_tail(const DecodeParams& p, const int4* s_cut, const int32
         const int32_t n = c.z, i_first = c.w, fslot = s_cut_fslot[s];
         __threadfence();   // the other pieces' states, counted before this CTA's, are visible
         if (todo == 1) {
-            merge_pieces<D>(p, c.x, c.y, i_first, fslot, 0, n, 1, -1, s_lse);
+            merge_pieces<D>(p, c.x, c.y, i_first, fslot, 0, n, 1, -1, scratch);
             continue;
         }
         const int32_t k = (int32_t)blockIdx.x - i_first, lead = k / kMergeFan * kMergeFan;
-        merge_pieces<D>(p, c.x, c.y, i_first, fslot, lead, min(n, lead + kMergeFan), 1, lead, s_lse);
+        merge_pieces<D>(p, c.x, c.y, i_first, fslot, lead, min(n, lead + kMergeFan), 1, lead, scratch);
         __threadfence();
         __syncthreads();
         if (threadIdx.x == 0)
-            s_final = counter_add(p.merge_cnt + (size_t)c.y * p.num_seqs + c.x, p.epoch, p.status) ==
+            s_final = counter_add(p.merge_cnt + (size_t)c.y * p.num_seqs + c.x, s_epoch, p.status) ==
                       (n + kMergeFan - 1) / kMergeFan;
         __syncthreads();
         if (s_final) {
             __threadfence();
-            merge_pieces<D>(p, c.x, c.y, i_first, fslot, 0, n, kMergeFan, -1, s_lse);
+            merge_pieces<D>(p, c.x, c.y, i_first, fslot, 0, n, kMergeFan, -1, scratch);
         }
         __syncthreads();
     }
@@ -866,7 +889,15 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     if (p.inline_merge) {
         __threadfence();   // this CTA's partial states, before its pieces are counted
         __syncthreads();
-        merge_tail<D>(p, s_cut, s_cut_fslot, s_failed != 0);
+        // every stage has been consumed: the stage memory is scratch for the merges
+        merge_tail<D>(p, s_cut, s_cut_fslot, s_failed != 0, reinterpret_cast<float*>(smem_gen));
+        if (threadIdx.x == 0) {   // the last CTA to finish gives the next launch a new number
+            __threadfence();
+            if (atomicAdd(p.stream_done, 1) == (int32_t)gridDim.x - 1) {
+                *reinterpret_cast<volatile int32_t*>(p.stream_done) = 0;
+                atomicAdd(p.epoch, 1u);
+            }
+        }
     }
     __syncthreads();
 }
@@ -1008,6 +1039,9 @@ int stream_kernel_grid(const pa_cache_desc& d, int max_ctas, bool fp8) {
     if (occ <= 0) return 0;
     int grid = sms * occ;
     if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
+    // a sequence has at most `grid` pieces, merged in groups of kMergeFan: the final merge of
+    // the groups takes at most kMergeInputs inputs
+    if (grid > kMergeFan * kMergeInputs) grid = kMergeFan * kMergeInputs;
     return grid;
 }
 

@@ -52,7 +52,10 @@ struct DecodeParams {
     float out_scale;               // multiplies the normalised output (E4M3: the V scale; else 1)
     int32_t grid;                  // stream kernel: CTAs of the launch (bounds the merge's reads)
     int32_t inline_merge;          // stream kernel: the last piece of a cut sequence merges it
-    uint32_t epoch;                // call number (counters of earlier calls read as zero)
+    uint32_t* epoch;               // stream kernel: launch number (workspace word 3); the last CTA
+                                   //   to finish advances it, so counters of earlier launches,
+                                   //   graph replays included, read as zero
+    int32_t* stream_done;          // stream kernel: CTAs finished (workspace word 4, self-resetting)
     unsigned long long* merge_cnt; // stream kernel: [Hkv/8][B] counters of counted pieces / groups
     unsigned long long* group_cnt; // stream kernel: [grid][2] counters of a group's counted pieces
     int32_t selftest_stall;        // PA_FLAG_SELFTEST_STALL: CTA 0 of the stream kernel idles

@@ -11,18 +11,19 @@
 //   warps 0-3  softmax: thread i owns row i (tensor-memory lane i).  Per 64-key tile t it
 //              reads its row of S_t from tensor memory, masks it causally, and writes the
 //              probabilities P_t (bf16) into shared memory as the K-major A operand.
-//   warp 4     MMA issue (one thread): S_t = Q K_t^T into tensor memory, then, once P_t is
-//              written, O += P_t V_t, accumulated in tensor memory across tiles, and at once
-//              S_{t+1}, so the next scores are ready when the softmax warps come back.
-//   warp 5     TMA: K and V tiles of 64 keys into a two-stage ring, one box of 64 dims x
+//   warp 4     MMA issue (one thread): S_t = Q K_t^T into one of two score buffers in tensor
+//              memory two tiles ahead, and, once P_t is written, O += P_t V_t, accumulated in
+//              tensor memory across tiles.  The scores of the next tile are ready before the
+//              softmax warps finish this one, so no MMA latency sits between two tiles.
+//   warp 5     TMA: K and V tiles of 64 keys into a ring of stages, one box of 64 dims x
 //              min(Bs, 64) tokens per block and 64-dim atom, swizzled by the copy engine; a
 //              stage is refilled once the MMAs that read it have completed.
 // Online softmax with O in tensor memory: a row keeps its running max m until a tile raises
 // it by more than 8 (log2 domain); only then is the row's O scaled by 2^(m - m_new) in
-// tensor memory (load, scale, store) and m replaced.  In between, probabilities are
-// 2^(s - m) <= 2^8, which bf16 and the fp32 sums carry without loss of relative precision.
-// When the scores of tile t are committed, every MMA issued before them (the P V of tile
-// t-1 included) has completed, so O and P may be touched then without another wait.
+// tensor memory (load, scale, store), after the P V of the previous tile has completed, and m
+// replaced.  In between, probabilities are 2^(s - m) <= 2^8, which bf16 and the fp32 sums
+// carry without loss of relative precision.  P has two buffers: P_t is written once the P V
+// of tile t-2, which read the same buffer, has completed.
 //
 // Every wait is bounded (2 s, then the timeout status bit).  On a timeout each warp leaves
 // its loop; the MMA thread drains the TMA copies it has not seen land and waits for its own
@@ -44,28 +45,30 @@ namespace {
 constexpr int kWsRows = 128;     // query rows per CTA (tensor-memory lanes)
 constexpr int kWsKeys = 64;      // keys per tile
 constexpr int kWsThreads = 192;  // 4 softmax warps, the MMA warp, the TMA warp
-constexpr int kWsStages = 2;
 constexpr float kRescaleLog2 = 8.f;
 
 template <int D>
 struct WsCfg {
+    static constexpr int kStages = D == 64 ? 3 : 2;         // K/V ring
     static constexpr int kQBytes = kWsRows * D * 2;
     static constexpr int kKVBytes = kWsKeys * D * 2;       // one K (or V) tile
     static constexpr int kPBytes = kWsRows * kWsKeys * 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
-    static constexpr int kOffV = kOffK + kWsStages * kKVBytes;
-    static constexpr int kOffP = kOffV + kWsStages * kKVBytes;
-    static constexpr int kOffBar = kOffP + kPBytes;
-    // barriers: s_full, p_full, o_final, drain, k_full[2], v_full[2], kv_empty[2]; then the
-    // tensor-memory address and the number of tiles the TMA warp requested
-    static constexpr int kSmem = kOffBar + 128;
-    static constexpr int kColS = 0;                         // S: 64 fp32 columns
-    static constexpr int kColO = 64;                        // O: D fp32 columns
-    static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;
-    // two CTAs per SM: each softmax thread keeps its row of S (64 registers) while it scales
-    // its row of O, which three CTAs of six warps (at most 96 registers a thread) would spill
-    static constexpr int kMinBlocks = 2;
+    static constexpr int kOffV = kOffK + kStages * kKVBytes;
+    static constexpr int kOffP = kOffV + kStages * kKVBytes;   // 2 buffers
+    static constexpr int kOffBar = kOffP + 2 * kPBytes;
+    // barriers (8 bytes each): s_full[2], p_full, o_done[2], drain, k_full[S], v_full[S],
+    // kv_empty[S]; then the tensor-memory address and the last tile the TMA warp requested
+    static constexpr int kBars = 6 + 3 * kStages;
+    static constexpr int kSmem = kOffBar + kBars * 8 + 16;
+    static constexpr int kColS = 0;                         // S: two buffers of 64 fp32 columns
+    static constexpr int kColO = 128;                       // O: D fp32 columns
+    static constexpr uint32_t kTmemCols = 256;
+    // D = 64: two CTAs per SM (each softmax thread keeps its row of S in 64 registers while it
+    // scales its row of O, which three CTAs of six warps would spill); D = 128: one (its
+    // shared memory)
+    static constexpr int kMinBlocks = D == 64 ? 2 : 1;
 };
 
 template <int ROWS>
@@ -109,10 +112,11 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
     const uint32_t s_base = smem_u32(smem);
     const uint32_t s_q = s_base + C::kOffQ, s_k = s_base + C::kOffK, s_v = s_base + C::kOffV;
     const uint32_t s_p = s_base + C::kOffP;
-    const uint32_t bar_s = s_base + C::kOffBar, bar_p = bar_s + 8, bar_of = bar_s + 16,
-                   bar_drain = bar_s + 24, bar_k = bar_s + 32, bar_v = bar_s + 48, bar_e = bar_s + 64;
-    const uint32_t s_tmem = bar_s + 80;
-    volatile int* s_kreq = reinterpret_cast<volatile int*>(smem + C::kOffBar + 84);
+    constexpr int ST = C::kStages;
+    const uint32_t bar_s = s_base + C::kOffBar, bar_p = bar_s + 16, bar_o = bar_s + 24,
+                   bar_drain = bar_s + 40, bar_k = bar_s + 48, bar_v = bar_k + 8 * ST, bar_e = bar_v + 8 * ST;
+    const uint32_t s_tmem = bar_s + C::kBars * 8;
+    volatile int* s_kreq = reinterpret_cast<volatile int*>(smem + C::kOffBar + C::kBars * 8 + 4);
 
     const int b = blockIdx.z, kvh = blockIdx.y;
     const int G = p.group, Hq = p.num_q_heads, Hkv = p.num_kv_heads, Bs = p.block_size;
@@ -146,10 +150,12 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
     }
     if (tid == 0) {
         mbar_init(bar_s, 1);
+        mbar_init(bar_s + 8, 1);
         mbar_init(bar_p, 4);                                 // one arrival per softmax warp
-        mbar_init(bar_of, 1);
+        mbar_init(bar_o, 1);
+        mbar_init(bar_o + 8, 1);
         mbar_init(bar_drain, 1);
-        for (int i = 0; i < kWsStages; ++i) {
+        for (int i = 0; i < ST; ++i) {
             mbar_init(bar_k + 8 * i, 1);
             mbar_init(bar_v + 8 * i, 1);
             mbar_init(bar_e + 8 * i, 1);
@@ -180,10 +186,10 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
         // ================================ TMA ================================
         const int rb = Bs < kWsKeys ? Bs : kWsKeys, nslot = kWsKeys / rb;
         for (int t = 0; t < ntiles && !failed; ++t) {
-            const int st = t & 1;
-            if (t >= kWsStages) {                            // the MMAs of tile t-2 have completed
+            const int st = t % ST;
+            if (t >= ST) {                                   // the MMAs of tile t - ST have completed
                 bool ok = true;
-                if (lane == 0) ok = mbar_wait(bar_e + 8 * st, (uint32_t)(((t >> 1) - 1) & 1), p.status);
+                if (lane == 0) ok = mbar_wait(bar_e + 8 * st, (uint32_t)((t / ST - 1) & 1), p.status);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     failed = true;
                     break;
@@ -220,60 +226,62 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
             constexpr uint32_t kIdescS = umma_idesc_bf16(kWsRows, kWsKeys, false);
             constexpr uint32_t kIdescO = umma_idesc_bf16(kWsRows, D, true);
             auto wait_k = [&](int t) {
-                if (!mbar_wait(bar_k + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status)) return false;
+                if (!mbar_wait(bar_k + 8 * (t % ST), (uint32_t)((t / ST) & 1), p.status)) return false;
                 k_seen = t;
                 return true;
             };
             auto wait_v = [&](int t) {
-                if (!mbar_wait(bar_v + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status)) return false;
+                if (!mbar_wait(bar_v + 8 * (t % ST), (uint32_t)((t / ST) & 1), p.status)) return false;
                 v_seen = t;
                 return true;
             };
-            auto issue_s = [&](int t) {                      // S = Q K_t^T over D / 16 K steps
-                const uint32_t kt = s_k + (t & 1) * C::kKVBytes;
+            auto issue_s = [&](int t) {                      // S buffer t & 1 = Q K_t^T over D / 16 K steps
+                const uint32_t kt = s_k + (t % ST) * C::kKVBytes;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint64_t a = umma_desc_sw128(s_q + (ks >> 2) * (kWsRows * 128) + (ks & 3) * 32, 16, 1024);
                     const uint64_t bd = umma_desc_sw128(kt + (ks >> 2) * (kWsKeys * 128) + (ks & 3) * 32, 16, 1024);
-                    umma_bf16_ss(tmem + C::kColS, a, bd, kIdescS, ks > 0);
+                    umma_bf16_ss(tmem + C::kColS + (t & 1) * 64, a, bd, kIdescS, ks > 0);
                 }
+                umma_commit(bar_s + 8 * (t & 1));
             };
-            auto issue_o = [&](int t) {                      // O += P V_t over 4 K steps of 16 keys
-                const uint32_t vt = s_v + (t & 1) * C::kKVBytes;
+            auto issue_o = [&](int t) {                      // O += P_t V_t over 4 K steps of 16 keys
+                const uint32_t vt = s_v + (t % ST) * C::kKVBytes, pt = s_p + (t & 1) * C::kPBytes;
 #pragma unroll
                 for (int kk = 0; kk < kWsKeys / 16; ++kk) {
-                    const uint64_t a = umma_desc_sw128(s_p + kk * 32, 16, 1024);
+                    const uint64_t a = umma_desc_sw128(pt + kk * 32, 16, 1024);
                     const uint64_t bd = umma_desc_sw128(vt + kk * 16 * 128, kWsKeys * 128, 1024);
                     umma_bf16_ss(tmem + C::kColO, a, bd, kIdescO, (t > 0 || kk > 0) ? 1u : 0u);
                 }
+                umma_commit(bar_e + 8 * (t % ST));           // K_t and V_t are free once these land
+                umma_commit(bar_o + 8 * (t & 1));
             };
-            if (wait_k(0)) {
+            // scores run two tiles ahead of P V: S_0 and S_1 first, then per tile P_t V_t and S_{t+2}
+            bool ok = wait_k(0);
+            if (ok) {
                 tc_fence_after_sync();
                 issue_s(0);
-                umma_commit(bar_s);
-                for (int t = 0; t < ntiles; ++t) {
-                    if (!mbar_wait(bar_p, (uint32_t)(t & 1), p.status) || !wait_v(t)) {
-                        failed = true;
+            }
+            if (ok && ntiles > 1) {
+                ok = wait_k(1);
+                if (ok) issue_s(1);
+            }
+            for (int t = 0; t < ntiles && ok; ++t) {
+                if (!mbar_wait(bar_p, (uint32_t)(t & 1), p.status) || !wait_v(t)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                issue_o(t);
+                if (t + 2 < ntiles) {
+                    if (!wait_k(t + 2)) {
+                        ok = false;
                         break;
                     }
-                    tc_fence_after_sync();
-                    issue_o(t);
-                    umma_commit(bar_e + 8 * (t & 1));        // K_t and V_t are free once these land
-                    if (t + 1 < ntiles) {
-                        if (!wait_k(t + 1)) {
-                            failed = true;
-                            break;
-                        }
-                        tc_fence_after_sync();
-                        issue_s(t + 1);
-                        umma_commit(bar_s);
-                    } else {
-                        umma_commit(bar_of);
-                    }
+                    issue_s(t + 2);
                 }
-            } else {
-                failed = true;
             }
+            if (!ok) failed = true;
         }
         __syncwarp();
     } else {
@@ -283,14 +291,18 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
         const int pos = R < rows ? L - Tq + R / G : L - 1;  // padded rows: computed, not written
         const float sl2 = p.scale_log2;
         float m_run = -INFINITY, l_run = 0.f;
+        // P V of tile t: its barrier (buffer t & 1) completes once per use
+        auto wait_o = [&](int t) {
+            return warp_wait(bar_o + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status);
+        };
         for (int t = 0; t < ntiles; ++t) {
-            if (!warp_wait(bar_s, (uint32_t)(t & 1), p.status)) {
+            if (!warp_wait(bar_s + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status)) {
                 failed = true;
                 break;
             }
             tc_fence_after_sync();
             uint32_t sr[64];
-            tmem_ld64(t_lane + C::kColS, sr);
+            tmem_ld64(t_lane + C::kColS + (t & 1) * 64, sr);
             const int k0 = t * kWsKeys;
             float mx = -INFINITY;
             if (k0 + kWsKeys - 1 > pos_first) {              // a tile on the diagonal: mask
@@ -311,7 +323,12 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
             } else {
                 const bool need = m_new > m_run + kRescaleLog2;
                 if (__any_sync(0xffffffffu, need)) {
-                    // O of tile t-1 is complete (it was issued before S_t): scale this row
+                    // once O holds tile t-1 in full, scale this row
+                    if (!wait_o(t - 1)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
                     const float a = need ? fast_exp2(m_run - m_new) : 1.f;
 #pragma unroll
                     for (int h = 0; h < D / 32; ++h) tmem_scale32(t_lane + C::kColO + h * 32, a);
@@ -333,7 +350,11 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
                 pk[j] = pack_bf16x2(p0, p1);
             }
             l_run += rsum;
-            const uint32_t prow = s_p + tid * 128;
+            if (t >= 2 && !wait_o(t - 2)) {                 // the P V that read this P buffer is done
+                failed = true;
+                break;
+            }
+            const uint32_t prow = s_p + (t & 1) * C::kPBytes + tid * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + ((c ^ (tid & 7)) << 4)),
@@ -343,11 +364,11 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
                 // the last tile: V rows past the sequence (stale pool rows, or never copied)
                 // are zeroed so that P = 0 there cannot meet a NaN pattern; the MMA reads V
                 // only after all four warps' arrivals below, so each warp zeroes its share
-                if (!warp_wait(bar_v + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status)) {
+                if (!warp_wait(bar_v + 8 * (t % ST), (uint32_t)((t / ST) & 1), p.status)) {
                     failed = true;
                     break;
                 }
-                const uint32_t vt = s_v + (t & 1) * C::kKVBytes;
+                const uint32_t vt = s_v + (t % ST) * C::kKVBytes;
                 for (int i = tid; i < (kWsKeys - (L - k0)) * (D / 8); i += 128) {
                     const int row = (L - k0) + i / (D / 8), c = i % (D / 8);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vt + ws_sw128<kWsKeys>(row, c)),
@@ -360,7 +381,7 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_p);
         }
-        if (!failed && warp_wait(bar_of, 0u, p.status)) {
+        if (!failed && wait_o(ntiles - 1)) {
             tc_fence_after_sync();
             const int tok = R / G, g = R - tok * G;
             const float inv = 1.f / l_run;
@@ -389,8 +410,8 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
     __syncthreads();
     if (warp == 4 && lane == 0) {
         const int req = *s_kreq;
-        for (int t = k_seen + 1; t <= req; ++t) mbar_wait(bar_k + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status);
-        for (int t = v_seen + 1; t <= req; ++t) mbar_wait(bar_v + 8 * (t & 1), (uint32_t)((t >> 1) & 1), p.status);
+        for (int t = k_seen + 1; t <= req; ++t) mbar_wait(bar_k + 8 * (t % ST), (uint32_t)((t / ST) & 1), p.status);
+        for (int t = v_seen + 1; t <= req; ++t) mbar_wait(bar_v + 8 * (t % ST), (uint32_t)((t / ST) & 1), p.status);
         umma_commit(bar_drain);
         mbar_wait(bar_drain, 0u, p.status);
     }

@@ -71,13 +71,14 @@ def test_c4_planted_stream_kernel(h, c4_stream, fused):
 
 
 def test_c4_planted_stream_kernel_odd_grid(h):
-    # a grid that is no multiple of the SM count: slices start mid-block everywhere
+    # a grid that is no multiple of the SM count (max_ctas caps the resident grid): slices
+    # start mid-block everywhere and every sequence is cut into more, longer pieces
     b = wl.config4()
     max_len = int(b.context_lens.max()) + 1
-    opts = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR, max_ctas=211)
+    opts = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR, max_ctas=97)
     pb, info = _planted(h, b, opts, max_len)
-    assert info.ctas == 211
-    _check(h.run_step(pb, kernel=pa.PA_KERNEL_TENSOR, max_ctas=211))
+    assert info.ctas == 97
+    _check(h.run_step(pb, kernel=pa.PA_KERNEL_TENSOR, max_ctas=97))
 
 
 @pytest.mark.parametrize("kernel", [pa.PA_KERNEL_TENSOR_SPLIT, pa.PA_KERNEL_SIMT], ids=["split", "simt"])
