@@ -198,19 +198,15 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * with K_j, V_j the rows of kv head h / (Hq/Hkv).  fp32 accumulation, online
  * softmax, the result rounded to nearest-even bf16.  A sequence with
  * context_lens[b] == 0 outputs zeros.  Long contexts are split across CTAs:
- * each piece leaves an fp32 partial state in the workspace, and the pieces are
- * merged (log-sum-exp) into out: by the CTA that finishes a sequence's last
- * piece, inside the same launch, for the whole-group tensor kernel; by a
- * second kernel, launched by the same call on the same stream, for the others.
+ * each piece leaves an fp32 partial state in the workspace, and a second
+ * kernel, launched by the same call on the same stream, merges them
+ * (log-sum-exp) into out.
  *
  * workspace: caller-owned device buffer of at least
  * pa_decode_workspace_size(...) bytes, 256-byte aligned, ZERO-FILLED BEFORE
  * ITS FIRST USE.  The kernels leave their work counters at zero when they
- * complete, and the merge counters of the whole-group tensor kernel carry a
- * launch number kept in the workspace (so a workspace left by a call that gave
- * up on a wait, or replayed in a captured graph, serves the next launch as it
- * is); the buffer can be reused by later calls without clearing.  Calls that
- * may overlap on the GPU need separate workspaces.
+ * complete, so the buffer can be reused by later calls without clearing;
+ * calls that may overlap on the GPU need separate workspaces.
  *
  * Built shapes: head_dim 64 or 128; block_size 8, 16, 32, 64, 128 or 256;
  * Hq / Hkv <= 16.  Others return PA_ERR_UNSUPPORTED.  The tensor-core
@@ -238,8 +234,7 @@ PA_API size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t max_context_
  * workspace are touched after the wait.  Set the flag only when context_lens
  * and block_tables were complete before the previous kernel on `stream`
  * started (host-written metadata, as in a serving step's layer loop).  The
- * library's own kernels (append, merge, the decode itself) let such a launch
- * start early.
+ * library's own kernels (append, merge) let such a launch start early.
  */
 PA_API int pa_decode(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf16* v_cache,
               const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,

@@ -85,8 +85,7 @@ int num_sms_current_device(int* out) {
 //    ceil(max_context_len / C) per (sequence, kv head).  Automatic C: enough
 //    work items for about 32 per SM if every sequence were max_context_len
 //    long, never below 128 tokens.
-// Workspace: [0, 256) status word, work counters, the stream kernel's launch number and
-// finished-CTA count (words 0-4); (kStream) one piece
+// Workspace: [0, 256) status word and work counters; (kStream) one piece
 // descriptor per (kv group, sequence); partial log-sum-exps; partial outputs.
 int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_desc& d,
                      const pa_decode_options* opt, DecodePlan* plan) {
@@ -99,7 +98,6 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
     plan->off_desc = kWorkspaceAlign;
     plan->off_lse = plan->off_desc;
     plan->off_qrot = 0;
-    plan->off_mcnt = plan->off_gcnt = 0;
     plan->grid = 0;
     plan->split_tokens = 0;
     plan->max_splits = 1;
@@ -114,9 +112,7 @@ int make_decode_plan(int32_t num_seqs, int32_t max_context_len, const pa_cache_d
         plan->off_lse = plan->off_desc + up((size_t)(d.num_kv_heads / 8) * num_seqs * 16);
         const size_t rows = (size_t)plan->grid * 2 * d.num_kv_heads * G;
         plan->off_o = plan->off_lse + up(rows * sizeof(float));
-        plan->off_mcnt = plan->off_o + up(rows * (size_t)d.head_dim * sizeof(float));
-        plan->off_gcnt = plan->off_mcnt + up((size_t)(d.num_kv_heads / 8) * num_seqs * sizeof(uint64_t));
-        plan->bytes = plan->off_gcnt + up((size_t)plan->grid * 2 * sizeof(uint64_t));
+        plan->bytes = plan->off_o + up(rows * (size_t)d.head_dim * sizeof(float));
         return PA_OK;
     }
     if (kernel == PA_KERNEL_TENSOR || kernel == PA_KERNEL_TENSOR_SPLIT) {
@@ -379,11 +375,6 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
     char* ws = static_cast<char*>(workspace);
     DecodeParams p;
     p.grid = plan.grid;
-    p.inline_merge = plan.kernel == DecodeKernel::kStream ? 1 : 0;
-    p.epoch = reinterpret_cast<uint32_t*>(ws) + 3;
-    p.stream_done = reinterpret_cast<int32_t*>(ws) + 4;
-    p.merge_cnt = reinterpret_cast<unsigned long long*>(ws + plan.off_mcnt);
-    p.group_cnt = reinterpret_cast<unsigned long long*>(ws + plan.off_gcnt);
     p.selftest_stall = stall ? 1 : 0;
     p.wait_ns = stall ? kSelftestWaitNs : kDecodeWaitNs;
     p.q = q;
@@ -440,10 +431,8 @@ static int decode_call(const pa_bf16* q, const pa_bf16* k_new, const pa_bf16* v_
         case DecodeKernel::kSplit: e = launch_decode_tensor(p, st); break;
         default: e = launch_decode_simt(p, st); break;
     }
-    // second pass: merge the pieces of every sequence that was cut (the stream kernel merges
-    // its own)
-    if (e == cudaSuccess && ((plan.kernel == DecodeKernel::kStream && !p.inline_merge) ||
-                             (plan.kernel != DecodeKernel::kStream && plan.max_splits > 1)))
+    // second pass: merge the pieces of every sequence that was cut
+    if (e == cudaSuccess && (plan.kernel == DecodeKernel::kStream || plan.max_splits > 1))
         e = launch_merge(p, plan.kernel == DecodeKernel::kStream,
                          plan.kernel != DecodeKernel::kSimt, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;

@@ -17,8 +17,7 @@
 // host-side stand-in), so on the first call on each device, with that device
 // current, its address is looked up once with cudaGetSymbolAddress and cached.
 // Calls share the array and it keeps the previous call's contents; the words
-// that must start at zero (the status word and the work counters) are cleared
-// by a cudaMemsetAsync on the call's stream.
+// that must start at zero are cleared by a cudaMemsetAsync on the call's stream.
 // The address belongs to the device's primary context (the runtime API's
 // context); a caller that makes another driver-API context current on the same
 // device must not call this entry point from it.
@@ -75,10 +74,8 @@ extern "C" int pa_decode_noalloc(const pa_bf16* q, const pa_bf16* k_cache, const
     void* scratch = nullptr;
     const int rc = scratch_address(&scratch);
     if (rc != PA_OK) return rc;
-    // status word and work counters (words 0-2) must start at zero; the launch number of the
-    // merge counters (word 3) must not go back, and the rest is written before it is read
-    if (cudaMemsetAsync(scratch, 0, 3 * sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
-        return PA_ERR_CUDA;
+    // status word and work counters must start at zero; the rest is written before it is read
+    if (cudaMemsetAsync(scratch, 0, 256, (cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
     return pa_decode_ex(q, k_cache, v_cache, block_tables, context_lens, num_seqs, max_context_len,
                         scale, out, scratch, kNoAllocScratchBytes, desc, options, stream);
 }

@@ -144,157 +144,6 @@ __device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 x, float inv_scale) {
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-// ---- merging the pieces of cut sequences, inside the decode kernel ----------------------
-// A sequence cut across CTAs i_first .. i_first + n - 1 leaves one normalised partial state per
-// piece: piece 0 in partial slot `fslot` of CTA i_first, piece k >= 1 in slot 0 of CTA
-// i_first + k (rows of part_o / part_lse).  Each CTA, once its pieces are written, counts them
-// on the sequence's counter; the CTA whose count completes it merges all pieces (log-sum-exp,
-// the same arithmetic as merge.cu) into out.  A sequence of more than kMergeFan pieces is
-// merged in two levels: the pieces are counted per group of kMergeFan on a counter of the
-// group's first piece; the CTA completing a group merges it into that first piece's rows and
-// counts the group on the sequence's counter, and the CTA completing that merges the groups.
-// Counters hold (launch number << 32 | count): a counter left by an earlier launch (one that
-// gave up on a wait, say) reads as zero, so they never need clearing.  The launch number lives
-// in the workspace; the last CTA of a launch to finish advances it, so every launch, and every
-// replay of a captured graph, counts under a number of its own.
-constexpr int32_t kMergeFan = 16;
-
-__device__ __forceinline__ int32_t counter_add(unsigned long long* c, uint32_t epoch, int32_t* status) {
-    unsigned long long old = __ldcg(c);
-    for (int it = 0; it < (1 << 20); ++it) {
-        const unsigned long long nw =
-            (uint32_t)(old >> 32) == epoch ? old + 1 : (((unsigned long long)epoch << 32) | 1ull);
-        const unsigned long long prev = atomicCAS(c, old, nw);
-        if (prev == old) return (int32_t)(uint32_t)nw;
-        old = prev;
-    }
-    raise_status(status, kStatusTimeout);
-    return -1;
-}
-
-// Merges pieces k = k0, k0 + step, ... < k1 (at most kMergeInputs of them) of one sequence for
-// the 8 kv heads of group gi: into out (bf16) when lead < 0, else into the partial rows of piece
-// `lead` (fp32 state + lse).  Three phases, so that every load of a phase is independent of the
-// others: (1) one thread per query head loads the pieces' lse values into shared memory, (2)
-// turns them into normalised weights 2^(lse_k - M) / W, (3) every thread accumulates its float4
-// columns over the pieces with those weights.  `scratch` is the CTA's stage memory, idle once
-// its slice is streamed.
-constexpr int32_t kMergeInputs = 32;
-
-template <int D>
-__device__ void merge_pieces(const DecodeParams& p, int32_t b, int32_t gi, int32_t i_first, int32_t fslot,
-                             int32_t k0, int32_t k1, int32_t step, int32_t lead, float* scratch) {
-    const int32_t G = p.group, Hkv = p.num_kv_heads, HG = 8 * G;
-    constexpr int kCols = D / 4;
-    const int32_t np = (k1 - k0 + step - 1) / step;
-    float* s_w = scratch;                       // [np][HG] weights
-    float* s_lse = scratch + kMergeInputs * 128; // [HG] the merged lse (group merges)
-    auto row_of = [&](int32_t k) -> size_t {
-        const int32_t cta = i_first + k, slot = k == 0 ? fslot : 0;
-        return ((size_t)cta * 2 + slot) * Hkv;
-    };
-    for (int32_t t = threadIdx.x; t < HG; t += blockDim.x) {
-        const int32_t kvh = gi * 8 + t / G, h = t % G;
-        float m = -INFINITY;
-#pragma unroll 4
-        for (int32_t i = 0; i < np; ++i) {
-            const float lse = __ldcg(p.part_lse + (row_of(k0 + i * step) + kvh) * G + h);
-            s_w[i * HG + t] = lse;
-            m = fmaxf(m, lse);
-        }
-        float W = 0.f;
-        for (int32_t i = 0; i < np; ++i) W += fast_exp2(s_w[i * HG + t] - m);
-        const float inv = 1.f / W;
-        for (int32_t i = 0; i < np; ++i) s_w[i * HG + t] = fast_exp2(s_w[i * HG + t] - m) * inv;
-        s_lse[t] = m + __log2f(W);
-    }
-    __syncthreads();
-    const int32_t units = HG * kCols;
-    for (int32_t u = threadIdx.x; u < units; u += blockDim.x) {
-        const int32_t t = u / kCols, c4 = u - t * kCols;
-        const int32_t kvh = gi * 8 + t / G, h = t % G;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int32_t i = 0; i < np; ++i) {
-            const size_t r = (row_of(k0 + i * step) + kvh) * G + h;
-            const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + r * D) + c4);
-            const float w = s_w[i * HG + t];
-            acc.x = fmaf(w, o.x, acc.x);
-            acc.y = fmaf(w, o.y, acc.y);
-            acc.z = fmaf(w, o.z, acc.z);
-            acc.w = fmaf(w, o.w, acc.w);
-        }
-        if (lead < 0) {
-            uint2 packed;
-            packed.x = pack_bf16x2(acc.x, acc.y);
-            packed.y = pack_bf16x2(acc.z, acc.w);
-            reinterpret_cast<uint2*>(p.out + ((size_t)b * p.num_q_heads + (size_t)kvh * G + h) * D)[c4] = packed;
-        } else {
-            // the group's state replaces its first piece's (each thread writes back only the
-            // columns it read itself)
-            const size_t r = (row_of(lead) + kvh) * G + h;
-            reinterpret_cast<float4*>(p.part_o + r * D)[c4] = acc;
-        }
-    }
-    if (lead >= 0) {
-        for (int32_t t = threadIdx.x; t < HG; t += blockDim.x)
-            p.part_lse[(row_of(lead) + gi * 8 + t / G) * G + t % G] = s_lse[t];
-    }
-    __syncthreads();                            // scratch free again
-}
-
-// The CTA's share of the merging, after its own pieces are written (called by every thread).
-template <int D>
-__device__ void merge_tail(const DecodeParams& p, const int4* s_cut, const int32_t* s_cut_fslot, bool failed,
-                           float* scratch) {
-    __shared__ int32_t s_todo[2], s_final;
-    __shared__ uint32_t s_epoch;
-    if (threadIdx.x == 0) {
-        // advanced only after every CTA of this launch has finished: one value for all of them
-        s_epoch = *reinterpret_cast<volatile uint32_t*>(p.epoch);
-        for (int s = 0; s < 2; ++s) {
-            const int4 c = s_cut[s];
-            int32_t todo = 0;
-            if (!failed && c.z > 1) {
-                const int32_t n = c.z, i_first = c.w, k = (int32_t)blockIdx.x - i_first;
-                if (n <= kMergeFan) {
-                    todo = counter_add(p.merge_cnt + (size_t)c.y * p.num_seqs + c.x, s_epoch, p.status) == n ? 1 : 0;
-                } else {
-                    const int32_t lead = k / kMergeFan * kMergeFan, size = min(kMergeFan, n - lead);
-                    const int32_t cta = i_first + lead, slot = lead == 0 ? s_cut_fslot[s] : 0;
-                    todo = counter_add(p.group_cnt + (size_t)cta * 2 + slot, s_epoch, p.status) == size ? 2 : 0;
-                }
-            }
-            s_todo[s] = todo;
-        }
-    }
-    __syncthreads();
-    for (int s = 0; s < 2; ++s) {
-        const int32_t todo = s_todo[s];
-        if (todo == 0) continue;
-        const int4 c = s_cut[s];
-        const int32_t n = c.z, i_first = c.w, fslot = s_cut_fslot[s];
-        __threadfence();   // the other pieces' states, counted before this CTA's, are visible
-        if (todo == 1) {
-            merge_pieces<D>(p, c.x, c.y, i_first, fslot, 0, n, 1, -1, scratch);
-            continue;
-        }
-        const int32_t k = (int32_t)blockIdx.x - i_first, lead = k / kMergeFan * kMergeFan;
-        merge_pieces<D>(p, c.x, c.y, i_first, fslot, lead, min(n, lead + kMergeFan), 1, lead, scratch);
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0)
-            s_final = counter_add(p.merge_cnt + (size_t)c.y * p.num_seqs + c.x, s_epoch, p.status) ==
-                      (n + kMergeFan - 1) / kMergeFan;
-        __syncthreads();
-        if (s_final) {
-            __threadfence();
-            merge_pieces<D>(p, c.x, c.y, i_first, fslot, 0, n, kMergeFan, -1, scratch);
-        }
-        __syncthreads();
-    }
-}
-
 template <int D, int NT, bool F8>
 __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     decode_stream_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
@@ -307,9 +156,6 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     __shared__ __align__(8) uint64_t qfull_bar[kQSlots];
     __shared__ __align__(8) uint64_t qempty_bar[kQSlots];
     __shared__ double s_rope_inv[64];   // RoPE inverse frequencies of the D/2 pairs
-    __shared__ int4 s_cut[2];            // per partial slot: {sequence, kv group, pieces, first CTA}
-    __shared__ int32_t s_cut_fslot[2];   //   and the partial slot the sequence's first CTA used
-    __shared__ int32_t s_failed;         // a wait of this CTA gave up: it merges nothing
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t G = p.group;
@@ -333,8 +179,6 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             mbar_init(smem_u32(&qfull_bar[s]), 1);
             mbar_init(smem_u32(&qempty_bar[s]), kGroup);
         }
-        s_cut[0] = s_cut[1] = make_int4(0, 0, 0, 0);
-        s_failed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (p.rope_theta > 0.f)
@@ -344,7 +188,6 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     if (warp == kGroup && p.selftest_stall && blockIdx.x == 0) {
         // failure-handling self-test: this CTA's producer issues no copy and signals nothing,
         // so its consumers' first waits run out with no copy in flight
-        if (lane == 0) s_failed = 1;
     } else if (warp == kGroup) {
         // ================================ producer ================================
         const int32_t B = p.num_seqs, Bs = p.block_size;
@@ -448,11 +291,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     seg_slot = P < lo ? 0 : 1;
                     seg_ifirst = i_first;
                     seg_fslot = P < (int64_t)i_first * S / Gc ? 0 : 1;
-                    if (lane == 0 && seg_nsplit > 1) {   // a cut sequence: this CTA holds one piece
-                        s_cut[seg_slot] = make_int4(b, gi, seg_nsplit, i_first);
-                        s_cut_fslot[seg_slot] = seg_fslot;
-                    }
-                    if (!p.inline_merge && P >= lo && lane == 0)   // the merge kernel's descriptor
+                    if (P >= lo && lane == 0)   // this CTA holds the sequence's first slab
                         reinterpret_cast<int4*>(p.seq_desc)[(size_t)gi * B + b] =
                             make_int4(seg_nsplit, i_first, seg_fslot, 0);
                     if (s != lo) {
@@ -461,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     }
                     if (L > 0) {
                         int qs;
-                        if (!acquire(qempty_bar, qk, kQSlots, qs)) { alive = false; s_failed = 1; break; }
+                        if (!acquire(qempty_bar, qk, kQSlots, qs)) { alive = false; break; }
                         seg_q = qs;
                         if (lane == 0) {
                             const uint32_t bar = smem_u32(&qfull_bar[qs]);
@@ -474,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     }
                 }
                 int st;
-                if (!acquire(empty_bar, gtile, C::kStages, st)) { alive = false; s_failed = 1; break; }
+                if (!acquire(empty_bar, gtile, C::kStages, st)) { alive = false; break; }
                 const int32_t t0 = j * kSlab;
                 const int32_t valid = L == 0 ? 0 : min(kSlab, L - t0);
                 const uint32_t fbar = smem_u32(&full_bar[st]);
@@ -629,10 +468,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
         const int row_b = stage_row(warp, rr + ((mi >> 1) << 3), tb);    // V: tokens rr (+8)
         for (uint32_t gtile = 0;; ++gtile) {
             const int st = gtile % C::kStages;
-            if (!warp_wait(smem_u32(&full_bar[st]), (gtile / C::kStages) & 1, p.status, p.wait_ns)) {
-                s_failed = 1;
-                break;
-            }
+            if (!warp_wait(smem_u32(&full_bar[st]), (gtile / C::kStages) & 1, p.status, p.wait_ns)) break;
             const Hdr hd = s_hdr[st];
             if (hd.flags & kEnd) break;
             const int32_t kvh = hd.kvh0 + warp;
@@ -644,10 +480,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             }
             if (hd.flags & kFirst) {
                 const int qs = qk % kQSlots;
-                if (!warp_wait(smem_u32(&qfull_bar[qs]), (qk / kQSlots) & 1, p.status, p.wait_ns)) {
-                    s_failed = 1;
-                    break;
-                }
+                if (!warp_wait(smem_u32(&qfull_bar[qs]), (qk / kQSlots) & 1, p.status, p.wait_ns)) break;
                 uint16_t* qsm = reinterpret_cast<uint16_t*>(
                     smem_gen + (q_base - smem_base) + qs * (size_t)(kGroup * G * D * 2)) + (size_t)warp * G * D;
                 if (p.rope_theta > 0.f) {
@@ -886,19 +719,6 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 }
         }
     }
-    if (p.inline_merge) {
-        __threadfence();   // this CTA's partial states, before its pieces are counted
-        __syncthreads();
-        // every stage has been consumed: the stage memory is scratch for the merges
-        merge_tail<D>(p, s_cut, s_cut_fslot, s_failed != 0, reinterpret_cast<float*>(smem_gen));
-        if (threadIdx.x == 0) {   // the last CTA to finish gives the next launch a new number
-            __threadfence();
-            if (atomicAdd(p.stream_done, 1) == (int32_t)gridDim.x - 1) {
-                *reinterpret_cast<volatile int32_t*>(p.stream_done) = 0;
-                atomicAdd(p.epoch, 1u);
-            }
-        }
-    }
     __syncthreads();
 }
 
@@ -1039,9 +859,6 @@ int stream_kernel_grid(const pa_cache_desc& d, int max_ctas, bool fp8) {
     if (occ <= 0) return 0;
     int grid = sms * occ;
     if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
-    // a sequence has at most `grid` pieces, merged in groups of kMergeFan: the final merge of
-    // the groups takes at most kMergeInputs inputs
-    if (grid > kMergeFan * kMergeInputs) grid = kMergeFan * kMergeInputs;
     return grid;
 }
 

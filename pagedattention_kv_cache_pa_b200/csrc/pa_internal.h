@@ -51,13 +51,7 @@ struct DecodeParams {
     float k_inv_scale, v_inv_scale;  // E4M3: float(1/scale) applied when quantizing new rows
     float out_scale;               // multiplies the normalised output (E4M3: the V scale; else 1)
     int32_t grid;                  // stream kernel: CTAs of the launch (bounds the merge's reads)
-    int32_t inline_merge;          // stream kernel: the last piece of a cut sequence merges it
-    uint32_t* epoch;               // stream kernel: launch number (workspace word 3); the last CTA
-                                   //   to finish advances it, so counters of earlier launches,
-                                   //   graph replays included, read as zero
-    int32_t* stream_done;          // stream kernel: CTAs finished (workspace word 4, self-resetting)
-    unsigned long long* merge_cnt; // stream kernel: [Hkv/8][B] counters of counted pieces / groups
-    unsigned long long* group_cnt; // stream kernel: [grid][2] counters of a group's counted pieces
+
     int32_t selftest_stall;        // PA_FLAG_SELFTEST_STALL: CTA 0 of the stream kernel idles
     unsigned long long wait_ns;    // limit of every bounded wait in the stream kernel
 };
@@ -74,7 +68,7 @@ struct DecodePlan {
     int32_t split_tokens;          // kSimt / kSplit: tokens per split
     int32_t max_splits;            // kSimt / kSplit: splits per (sequence, kv head) at most
     int32_t grid;                  // kStream: persistent CTAs (partial slots: 2 per CTA)
-    size_t off_desc, off_lse, off_o, off_qrot, off_mcnt, off_gcnt, bytes;
+    size_t off_desc, off_lse, off_o, off_qrot, bytes;
 };
 
 // Paged prefill: sequence b's last cu_q[b+1] - cu_q[b] tokens attend causally to its

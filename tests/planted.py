@@ -17,8 +17,8 @@ query head's attention is pinned to a few planted keys instead:
 The planted positions are chosen from the decode kernel's own partition of the work: the
 first, middle and last 16-token slab of every CTA slice of the stream-partitioned kernel, and
 both sides of every split edge for the split kernels.  Every piece a cut sequence leaves for the
-merge holds the first or the last slab of its slice, so every piece (and every group of pieces
-the merge combines) carries planted keys.  The stream partition below restates the kernel's slicing
+merge holds the first or the last slab of its slice, so every piece (and every piece group of
+the merge) carries planted keys.  The stream partition below restates the kernel's slicing
 rule: the work is the concatenation, over groups of 8 kv heads and sequences, of 16-token slabs
 (an empty sequence counts one), cut into `grid` equal slices [i S / grid, (i + 1) S / grid).
 
