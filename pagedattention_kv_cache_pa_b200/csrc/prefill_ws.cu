@@ -304,18 +304,21 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
             uint32_t sr[64];
             tmem_ld64(t_lane + C::kColS + (t & 1) * 64, sr);
             const int k0 = t * kWsKeys;
-            float mx = -INFINITY;
+            // the row max over four independent chains (a single chain of 64 dependent maxima
+            // would sit on the tile's critical path)
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             if (k0 + kWsKeys - 1 > pos_first) {              // a tile on the diagonal: mask
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     const float v = k0 + j <= pos ? __uint_as_float(sr[j]) : -INFINITY;
                     sr[j] = __float_as_uint(v);
-                    mx = fmaxf(mx, v);
+                    mq[j & 3] = fmaxf(mq[j & 3], v);
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(sr[j]));
+                for (int j = 0; j < 64; ++j) mq[j & 3] = fmaxf(mq[j & 3], __uint_as_float(sr[j]));
             }
+            const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
             // key 0 is in every row's range, so the max is finite from the first tile on
             const float m_new = fmaxf(m_run, mx * sl2);
             if (t == 0) {
@@ -338,7 +341,7 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
                     }
                 }
             }
-            float rsum = 0.f;
+            float rs[4] = {0.f, 0.f, 0.f, 0.f};            // four independent partial sums
             uint32_t pk[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -346,10 +349,10 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
                 const float x1 = fmaf(__uint_as_float(sr[2 * j + 1]), sl2, -m_run);
                 const float p0 = j < kPolyPairs ? exp2_fma(x0) : fast_exp2(x0);
                 const float p1 = j < kPolyPairs ? exp2_fma(x1) : fast_exp2(x1);
-                rsum += p0 + p1;
+                rs[j & 3] += p0 + p1;
                 pk[j] = pack_bf16x2(p0, p1);
             }
-            l_run += rsum;
+            l_run += (rs[0] + rs[1]) + (rs[2] + rs[3]);
             if (t >= 2 && !wait_o(t - 2)) {                 // the P V that read this P buffer is done
                 failed = true;
                 break;
