@@ -81,8 +81,8 @@ def parse_args(argv=None):
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "split"], default="auto")
     ap.add_argument("--max-ctas", type=int, default=0)
     ap.add_argument("--prefill-kernel", choices=["auto", "tcgen05", "tcgen05_ws", "mma"], default="auto",
-                    help="pf: tcgen05 (tensor-memory accumulators), tcgen05_ws (one job per warp, O in "
-                         "tensor memory) or warp-level mma.sync")
+                    help="pf: tcgen05_ws (one job per warp, O in tensor memory; auto), tcgen05 "
+                         "(tensor-memory accumulators, one thread issues) or warp-level mma.sync")
     ap.add_argument("--path", choices=["fused", "separate"], default="fused",
                     help="fused: pa_append_decode; separate: pa_append_kv then pa_decode")
     ap.add_argument("--split-tokens", type=int, default=0)
@@ -1164,7 +1164,7 @@ def run_pf(args, rank, world, dist):
     if rank != 0:
         return None
     flops = prefill_flops(lens, q_lens, Hq, D)
-    pk = "tcgen05" if args.prefill_kernel == "auto" else args.prefill_kernel
+    pk = "tcgen05_ws" if args.prefill_kernel == "auto" else args.prefill_kernel   # auto at Bs = 16
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))

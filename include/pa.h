@@ -288,9 +288,11 @@ PA_API int pa_append_decode(const pa_bf16* q, const pa_bf16* k, const pa_bf16* v
  * aligned, its status word as for pa_decode (a block id outside the pool, or
  * L < Tq or L past the table: the sequence's rows are left unwritten and
  * pa_decode_status reports it).  head_dim 64 or 128.
- * kernel: PA_PREFILL_AUTO (= PA_PREFILL_TCGEN05), PA_PREFILL_TCGEN05 (128-row
- * tiles on the fifth-generation tensor cores, accumulators in tensor memory) or
- * PA_PREFILL_MMA (64-row tiles on warp-level mma.sync); both compute the same
+ * kernel: PA_PREFILL_AUTO (PA_PREFILL_TCGEN05_WS where it serves the block
+ * size, else PA_PREFILL_TCGEN05), PA_PREFILL_TCGEN05 (128-row tiles on the
+ * fifth-generation tensor cores, accumulators in tensor memory),
+ * PA_PREFILL_TCGEN05_WS (the same tiles with one job per warp) or
+ * PA_PREFILL_MMA (64-row tiles on warp-level mma.sync); all compute the same
  * operation, with fp32 accumulation in a different order.
  * Errors: PA_ERR_INVALID (also an unknown kernel), PA_ERR_UNSUPPORTED,
  * PA_ERR_WORKSPACE, PA_ERR_CUDA.

@@ -265,7 +265,8 @@ def pa_prefill(q, k_cache, v_cache, block_tables, cu_seqlens_q, context_lens, ma
                out, workspace, desc: CacheDesc, stream=None, kernel: str = "auto") -> None:
     """Causal attention of each sequence's last Tq tokens over its paged cache.
 
-    kernel: "auto" (= "tcgen05"), "tcgen05" or "mma" (the warp-level mma.sync kernel)."""
+    kernel: "auto" ("tcgen05_ws" where it serves the block size, else "tcgen05"), "tcgen05",
+    "tcgen05_ws" or "mma" (the warp-level mma.sync kernel)."""
     n = int(context_lens.shape[0])
     if kernel not in _PREFILL_KERNELS:
         raise ValueError("pa_prefill: kernel must be one of %s" % sorted(_PREFILL_KERNELS))

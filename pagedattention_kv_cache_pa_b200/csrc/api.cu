@@ -270,6 +270,9 @@ extern "C" int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf1
     p.max_blocks_per_seq = desc->max_blocks_per_seq;
     p.scale_log2 = scale * 1.4426950408889634f;
     const cudaStream_t st = (cudaStream_t)stream;
+    // automatic: the warp-specialized kernel where its TMA boxes tile the block size
+    if (kernel == PA_PREFILL_AUTO)
+        kernel = prefill_ws_supports(desc->block_size) ? PA_PREFILL_TCGEN05_WS : PA_PREFILL_TCGEN05;
     const cudaError_t e = kernel == PA_PREFILL_MMA          ? launch_prefill(p, max_q_len, st)
                           : kernel == PA_PREFILL_TCGEN05_WS ? launch_prefill_ws(p, max_q_len, st)
                                                             : launch_prefill_tc(p, max_q_len, st);

@@ -6,9 +6,9 @@
 //   M = max_s lse_s,  w_s = 2^(lse_s - M),  out = sum_s w_s o_s / sum_s w_s,
 // rounded once to bf16.  The pieces are spread over a CTA's threads and
 // folded with a running max, so a merge costs one round of L2 reads (after the
-// piece descriptor): for the stream-partitioned decode, one CTA per (sequence,
-// kv head) holding the kv head's G query heads; for the split kernels, one CTA
-// per (sequence, kv head, query head).  The kernels run as programmatic
+// piece descriptor): one CTA per (sequence, kv head, query head), or, for a
+// stream-partitioned decode of a large batch, one CTA per (sequence, kv head)
+// holding the kv head's G query heads.  The kernels run as programmatic
 // dependent launches: their CTAs may start while the decode kernel drains and
 // wait (griddepcontrol.wait) for the decode grid to complete before reading.
 #include <cuda_runtime.h>
@@ -19,13 +19,15 @@
 namespace pa {
 namespace {
 
-// Split kernels: one CTA of PG * D/4 threads per (sequence, kv head, query head): PG groups over
+// One CTA of PG * D/4 threads per (sequence, kv head, query head): PG groups over
 // the pieces (piece k goes to group k % PG) times D/4 float4 columns of the head
 // dimension.  Each thread folds its pieces into a running (max, weight, sum)
 // state as their lse and output arrive (independent loads), and the groups'
 // states are merged the same way through shared memory.  Long contexts cut a
 // sequence into many pieces: 16 groups keep each thread's chain short there.
-template <int D, int PG>
+// kStream: the stream partition's pieces (read from the sequence's descriptor);
+// else the split kernels' fixed splits.
+template <int D, bool kStream, int PG>
 __global__ void __launch_bounds__(PG * D / 4) merge_kernel(const DecodeParams p) {
     constexpr int kCols = D / 4;
     constexpr int kPieceGroups = PG;
@@ -36,12 +38,27 @@ __global__ void __launch_bounds__(PG * D / 4) merge_kernel(const DecodeParams p)
     const int32_t b = blockIdx.x, kvh = blockIdx.y, h = blockIdx.z;
     const int32_t G = p.group, Hkv = p.num_kv_heads;
     const int tid = threadIdx.x;
-    const int32_t L = clipped_length(p, b);
-    const int32_t nsplit = (L + p.split_tokens - 1) / p.split_tokens;
-    if (nsplit <= 1) return;
-    // piece 0: first_row; piece k >= 1: row0 + (k-1) * row_step
-    const size_t first_row = (((size_t)b * Hkv + kvh) * p.max_splits) * G + h;
-    const size_t row0 = first_row + G, row_step = (size_t)G;
+    int32_t nsplit;
+    size_t first_row, row0, row_step;   // piece 0: first_row; piece k >= 1: row0 + (k-1) * row_step
+    if (kStream) {
+        const int4 dsc = reinterpret_cast<const int4*>(p.seq_desc)[(size_t)(kvh / 8) * p.num_seqs + b];
+        nsplit = dsc.x;
+        if (nsplit <= 1) return;
+        // a descriptor this launch's decode did not write (it gave up on a timed-out wait)
+        // may be left from an earlier call: read nothing outside this launch's partial rows
+        if (dsc.y < 0 || dsc.z < 0 || dsc.z > 1 || (int64_t)dsc.y + nsplit > p.grid) return;
+        // CTA i_first + k wrote slot 0 for k > 0; the first CTA used slot dsc.z
+        first_row = (((size_t)dsc.y * 2 + dsc.z) * Hkv + kvh) * G + h;
+        row0 = (((size_t)(dsc.y + 1) * 2) * Hkv + kvh) * G + h;
+        row_step = (size_t)2 * Hkv * G;
+    } else {
+        const int32_t L = clipped_length(p, b);
+        nsplit = (L + p.split_tokens - 1) / p.split_tokens;
+        if (nsplit <= 1) return;
+        first_row = (((size_t)b * Hkv + kvh) * p.max_splits) * G + h;
+        row0 = first_row + G;
+        row_step = (size_t)G;
+    }
     const int kg = tid / kCols, col = tid - kg * kCols;
     float m = -INFINITY, W = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -89,11 +106,10 @@ __global__ void __launch_bounds__(PG * D / 4) merge_kernel(const DecodeParams p)
     }
 }
 
-// The stream kernel's pieces: one CTA per (sequence, kv head) with all G query heads of the
-// kv head in it, PG groups of G * D/4 threads (piece k to group k % PG).  A sequence the decode
-// did not cut costs its CTA one descriptor read.  PG is chosen at launch so that the grid fills
-// about one wave of the GPU: a batch of many short sequences (few pieces each) gets small CTAs,
-// a few long contexts (many pieces) get up to 1024 threads each.
+// The stream kernel's pieces of a large batch: one CTA per (sequence, kv head) with all G
+// query heads of the kv head in it, PG groups of G * D/4 threads (piece k to group k % PG).  A
+// sequence the decode did not cut costs its CTA one descriptor read, instead of G CTAs' worth.
+// PG is chosen at launch so that the grid fills about one wave of the GPU.
 template <int D>
 __global__ void __launch_bounds__(1024) merge_stream_kernel(const DecodeParams p, int PG) {
     constexpr int kCols = D / 4;
@@ -177,7 +193,7 @@ cudaError_t launch_ms(const DecodeParams& p, bool pdl, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, merge_stream_kernel<D>, p, PG);
 }
 
-template <int D, int PG>
+template <int D, bool kStream, int PG>
 cudaError_t launch_m(const DecodeParams& p, bool pdl, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.num_seqs, (unsigned)p.num_kv_heads, (unsigned)p.group);
@@ -188,22 +204,36 @@ cudaError_t launch_m(const DecodeParams& p, bool pdl, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, merge_kernel<D, PG>, p);
+    return cudaLaunchKernelEx(&cfg, merge_kernel<D, kStream, PG>, p);
 }
 
-template <int D>
+template <int D, bool kStream>
 cudaError_t launch_mg(const DecodeParams& p, bool pdl, cudaStream_t stream) {
     // contexts of 8K tokens and more are cut into many pieces per sequence
-    return p.max_context_len >= 8192 ? launch_m<D, 16>(p, pdl, stream) : launch_m<D, 4>(p, pdl, stream);
+    return p.max_context_len >= 8192 ? launch_m<D, kStream, 16>(p, pdl, stream)
+                                     : launch_m<D, kStream, 4>(p, pdl, stream);
+}
+
+// Stream partition: one CTA per query head while that grid stays within about two waves of
+// small CTAs (C2: 2048, C3: 1024, C4: 256 CTAs); beyond it (C5: 8192, mostly sequences that
+// were not cut) one CTA per kv head.  Measured per call: C5 88.0 -> 83.8 us with the
+// per-kv-head CTAs, while C2, C3 and C4 were 1.4 to 7 us faster with the per-head ones.
+template <int D>
+cudaError_t launch_stream_merge(const DecodeParams& p, bool pdl, cudaStream_t stream) {
+    int sms = 0;
+    if (num_sms_current_device(&sms) != PA_OK) return cudaErrorInvalidDevice;
+    const int64_t per_head_ctas = (int64_t)p.num_seqs * p.num_kv_heads * p.group;
+    if (per_head_ctas <= (int64_t)sms * 16) return launch_mg<D, true>(p, pdl, stream);
+    return launch_ms<D>(p, pdl, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const DecodeParams& p, bool stream_layout, bool pdl, cudaStream_t stream) {
     if (p.head_dim == 64)
-        return stream_layout ? launch_ms<64>(p, pdl, stream) : launch_mg<64>(p, pdl, stream);
+        return stream_layout ? launch_stream_merge<64>(p, pdl, stream) : launch_mg<64, false>(p, pdl, stream);
     if (p.head_dim == 128)
-        return stream_layout ? launch_ms<128>(p, pdl, stream) : launch_mg<128>(p, pdl, stream);
+        return stream_layout ? launch_stream_merge<128>(p, pdl, stream) : launch_mg<128, false>(p, pdl, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -1,7 +1,7 @@
 """Paged (chunked) prefill through the C ABI against the fp64 oracle (needs a B200).
 
-Both kernels (tcgen05 with tensor-memory accumulators, and warp-level mma.sync), each
-within 1e-2 + 1e-2 * |oracle|; cases: whole prompts (Tq = L), chunks after a cached
+The automatic choice and the single-issuer kernels (tcgen05 with tensor-memory accumulators,
+warp-level mma.sync), each within 1e-2 + 1e-2 * |oracle|; cases: whole prompts (Tq = L), chunks after a cached
 prefix (Tq < L), one-token chunks, lengths off the 64-key and 64/128-row tiles, GQA
 groups 1..16, head dims 64 and 128, block sizes 8..256; errors reported through the
 status word without a fault.
@@ -25,7 +25,7 @@ def h():
     return gpu_harness
 
 
-KERNELS = ["tcgen05", "mma"]
+KERNELS = ["auto", "tcgen05", "mma"]   # auto: the warp-specialized kernel where it serves the block size
 
 
 def _run(h, seed, lens, q_lens, kernel="auto", mutate=None, **kw):

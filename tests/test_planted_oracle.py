@@ -94,12 +94,12 @@ def test_dropping_one_slab_leaves_the_tolerance(c4, which):
     assert excess > 0.1
 
 
-# The merge kernel folds piece k of a sequence into piece group k % PG; PG is chosen at launch
-# to fill one wave of the GPU: 4 for C4 on a B200 (32 CTAs of 1024 threads).
-C4_MERGE_GROUPS = 4
+# The merge kernel folds piece k of a sequence into piece group k % PG: for C4 (contexts of 8K
+# tokens and more, 256 CTAs of one query head each) PG = 16.
+C4_MERGE_GROUPS = 16
 
 
-@pytest.mark.parametrize("group", range(C4_MERGE_GROUPS))
+@pytest.mark.parametrize("group", [0, 9, 15])
 def test_dropping_one_merge_piece_group_leaves_the_tolerance(c4, group):
     d = c4
     seq = 3            # the longest context: cut into about 60 pieces
