@@ -180,15 +180,24 @@ def profiled_traffic(config, kernel_name):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons sampled during the timed region.
+
+    NVML is polled from a thread every few milliseconds (read-only queries), so that even a
+    timed region of a few tens of milliseconds gets samples; the constructor returns once
+    the first sample is in.  Without NVML, `nvidia-smi -lms 100` is the fallback."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, device_index, enabled=True):
+    def __init__(self, device_index, enabled=True, interval_s=0.004):
         self.proc = None
+        self.thread = None
         self.device_index = device_index
+        self.samples = []                       # (sm_mhz, sm_max_mhz, reasons)
         if not enabled:
+            return
+        if self._start_nvml(interval_s):
             return
         try:
             self.proc = subprocess.Popen(
@@ -198,7 +207,63 @@ class ClockSampler:
         except (OSError, ValueError):
             self.proc = None
 
+    def _start_nvml(self, interval_s):
+        try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            handle = None
+            try:                                # the CUDA device's own GPU, by UUID
+                uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+                handle = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                handle = nv.nvmlDeviceGetHandleByIndex(self.device_index)
+            smax = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+            bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+        except Exception:
+            return False
+        self._stop_flag = threading.Event()
+        first = threading.Event()
+
+        def poll():
+            while True:
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                    self.samples.append((float(sm), float(smax),
+                                         {n for n, b in zip(self.NAMES, bits) if r & b}))
+                except Exception:
+                    pass
+                first.set()
+                if self._stop_flag.wait(interval_s):
+                    return
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+        first.wait(2.0)
+        self._nv = nv
+        return True
+
+    def _summary(self):
+        if not self.samples:
+            return None
+        reasons = set()
+        for _, _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(s for s, _, _ in self.samples),
+                "sm_max_mhz": max(m for _, m, _ in self.samples),
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
     def stop(self):
+        if self.thread is not None:
+            self._stop_flag.set()
+            self.thread.join(5.0)
+            try:
+                self._nv.nvmlShutdown()
+            except Exception:
+                pass
+            return self._summary()
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -207,25 +272,17 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            r = [x.strip() for x in r]
+        for r in out.strip().splitlines():
+            r = [x.strip() for x in r.split(",")]
             if len(r) < 9:
                 continue
             try:
-                sm.append(float(r[1]))
-                smax.append(float(r[2]))
+                sm, smax = float(r[1]), float(r[2])
             except ValueError:
                 continue
-            for name, val in zip(names, r[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+            self.samples.append((sm, smax, {n for n, v in zip(self.NAMES, r[5:9])
+                                            if v.lower().startswith("active")}))
+        return self._summary()
 
 
 # ---------------------------------------------------------------------------------------------
