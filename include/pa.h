@@ -286,8 +286,8 @@ PA_API int pa_append_decode(const pa_bf16* q, const pa_bf16* k, const pa_bf16* v
  * cu_seqlens_q: [num_seqs + 1] int32 device array (0 first, non-decreasing);
  * max_q_len >= every Tq (sizes the grid).  workspace: >= 256 bytes, 256-byte
  * aligned, its status word as for pa_decode (a block id outside the pool, or
- * L < Tq or L past the table: the sequence's rows are left unwritten and
- * pa_decode_status reports it).  head_dim 64 or 128.
+ * L < Tq, L past the table or Tq > max_q_len: the sequence's rows are left
+ * unwritten and pa_decode_status reports it).  head_dim 64 or 128.
  * kernel: PA_PREFILL_AUTO (PA_PREFILL_TCGEN05_WS where it serves the block
  * size, else PA_PREFILL_TCGEN05), PA_PREFILL_TCGEN05 (128-row tiles on the
  * fifth-generation tensor cores, accumulators in tensor memory),

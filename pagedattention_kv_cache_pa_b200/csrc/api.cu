@@ -268,6 +268,7 @@ extern "C" int pa_prefill(const pa_bf16* q, const pa_bf16* k_cache, const pa_bf1
     p.head_dim = desc->head_dim;
     p.group = desc->num_q_heads / desc->num_kv_heads;
     p.max_blocks_per_seq = desc->max_blocks_per_seq;
+    p.max_q_len = max_q_len;
     p.scale_log2 = scale * 1.4426950408889634f;
     const cudaStream_t st = (cudaStream_t)stream;
     // automatic: the warp-specialized kernel where its TMA boxes tile the block size

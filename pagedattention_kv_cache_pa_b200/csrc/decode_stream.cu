@@ -68,17 +68,20 @@ struct SCfg {
     }
 };
 
-enum : int32_t { kFirst = 1, kLast = 2, kEmpty = 4, kEnd = 8 };
+// kNew: the segment that starts at this stage holds the sequence's newest token (fused append)
+enum : int32_t { kFirst = 1, kLast = 2, kEmpty = 4, kEnd = 8, kNew = 16 };
 
 // Slabs an early-launched CTA prefetches into L2 before it waits for the previous kernel.
 constexpr int32_t kPrefetchSlabs = 2;
 
 struct Hdr {
     int32_t b, kvh0, t0, valid;   // sequence, first kv head of the group, stage tokens [t0, t0+valid)
-    int32_t flags, qslot;         // kFirst / kLast / kEmpty / kEnd; q ring slot of the segment
+    int32_t flags, qslot;         // kFirst / kLast / kEmpty / kEnd / kNew; q ring slot of the segment
     int32_t nsplit, slot;         // CTAs sharing the sequence; this CTA's partial slot (0/1)
     int32_t i_first, first_slot;  // first CTA of the sequence and the slot it used
-    int32_t rope_pos, pad1;       // RoPE: position of the sequence's newest token (L-1)
+    int32_t rope_pos;             // position of the sequence's newest token (L-1)
+    int32_t new_blk;              // fused append, on the stage holding that token: its physical
+                                  // block (-1: none, or an id outside the pool)
 };
 
 // Row of (kv head hl, token t) inside a stage half-tile filled by boxes of tb tokens x 8 heads.
@@ -129,19 +132,11 @@ template <bool F8>
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
     if constexpr (F8) return pack_f16x2(lo, hi); else return pack_bf16x2(lo, hi);
 }
-// Eight bf16 -> eight E4M3 codes of value * inv_scale (float product, nearest even, saturating).
+// Two floats -> two E4M3 codes (nearest even, saturating), the first in the low byte.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
-}
-__device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 x, float inv_scale) {
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    uint32_t c[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        c[i] = f32x2_to_e4m3x2(__fmul_rn(bf16_lo(w[i]), inv_scale), __fmul_rn(bf16_hi(w[i]), inv_scale));
-    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
 template <int D, int NT, bool F8>
@@ -260,6 +255,27 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             // the first table window, fetched while a prerequisite grid may still run
             int32_t win_base = (j * kSlab) / Bs, win_entry = -1;
             if (win_base + lane < p.max_blocks_per_seq) win_entry = __ldg(table + win_base + lane);
+            // Loads issued ahead so that no copy waits on one: the window after the current one
+            // (nx_win2), and, once a slice reaches the next sequence of the stream, that
+            // sequence's length and first window (nx_len, nx_win)
+            int32_t nx_len = 0, nx_win = -1, nx_win2 = -1;
+            bool have_win2 = false;
+            auto prefetch_win2 = [&]() {
+                have_win2 = (int64_t)(win_base + 32) * Bs < L;      // the sequence goes past it
+                const int32_t idx = win_base + 32 + lane;
+                if (have_win2) nx_win2 = idx < p.max_blocks_per_seq ? __ldg(table + idx) : -1;
+            };
+            auto refill = [&](int32_t lbk) {                         // warp-uniform
+                if (have_win2 && lbk == win_base + 32) {
+                    win_entry = nx_win2;
+                } else {
+                    const int32_t idx = lbk + lane;
+                    win_entry = idx < p.max_blocks_per_seq ? __ldg(table + idx) : -1;
+                }
+                win_base = lbk;
+                prefetch_win2();
+            };
+            prefetch_win2();
             if (p.early) {
                 // launched early: pull the first slabs of the slice (inside the first sequence
                 // and the fetched table window) into L2 while the previous kernel finishes
@@ -285,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             for (int64_t s = lo; s < hi && alive; ++s) {
                 const bool first = (s == lo) || (j == 0);
                 const bool last = (s == hi - 1) || (j == nb - 1);
+                bool seg_new = false;
                 if (first) {
                     const int32_t i_first = cta_of(P, S, Gc), i_last = cta_of(P + nb - 1, S, Gc);
                     seg_nsplit = i_last - i_first + 1;
@@ -294,10 +311,21 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     if (P >= lo && lane == 0)   // this CTA holds the sequence's first slab
                         reinterpret_cast<int4*>(p.seq_desc)[(size_t)gi * B + b] =
                             make_int4(seg_nsplit, i_first, seg_fslot, 0);
-                    if (s != lo) {
+                    if (s != lo) {                   // a new sequence: its window is in hand
                         table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
-                        win_base = -1;
+                        win_base = 0;
+                        win_entry = nx_win;
+                        prefetch_win2();
                     }
+                    if (s + (nb - j) < hi) {         // the slice reaches the next sequence
+                        const int32_t bn = b + 1 == B ? 0 : b + 1;
+                        nx_len = __ldg(p.context_lens + bn);
+                        nx_win = lane < p.max_blocks_per_seq
+                                     ? __ldg(p.block_tables + (size_t)bn * p.max_blocks_per_seq + lane)
+                                     : -1;
+                    }
+                    // fused append: this segment holds the sequence's newest token
+                    seg_new = p.k_new != nullptr && L > 0 && s + (nb - 1 - j) < hi;
                     if (L > 0) {
                         int qs;
                         if (!acquire(qempty_bar, qk, kQSlots, qs)) { alive = false; break; }
@@ -317,83 +345,21 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 const int32_t t0 = j * kSlab;
                 const int32_t valid = L == 0 ? 0 : min(kSlab, L - t0);
                 const uint32_t fbar = smem_u32(&full_bar[st]);
+                // fused append: the stage that holds the newest token (position L-1) carries its
+                // physical block; the consumer warps write the new K/V rows to the pool and into
+                // the staged tile, so no copy waits on those writes
+                int32_t new_blk = -1;
+                if (valid > 0 && p.k_new != nullptr && j == nb - 1) {
+                    const int32_t lbn = (L - 1) / Bs, lb0 = t0 / Bs;
+                    if (win_base < 0 || lbn >= win_base + 32) refill(lb0);
+                    const int32_t blk = __shfl_sync(0xffffffffu, win_entry, lbn - win_base);
+                    new_blk = blk >= 0 && blk < p.num_blocks ? blk : -1;
+                }
                 if (lane == 0) {
                     s_hdr[st] = Hdr{b, gi * kGroup, t0, valid,
-                                    (first ? kFirst : 0) | (last ? kLast : 0) | (L == 0 ? kEmpty : 0),
-                                    seg_q, seg_nsplit, seg_slot, seg_ifirst, seg_fslot, L - 1, 0};
-                }
-                if (valid > 0 && p.k_new != nullptr && j == nb - 1) {
-                    // fused append: this slab holds the sequence's newest token (position L-1);
-                    // write its K/V rows for the group's 8 kv heads before the slab is loaded
-                    // (K turned by RoPE at that position when the call asks for it)
-                    const int32_t pos = L - 1, lbn = pos / Bs;
-                    const int32_t blk = __ldg(table + lbn);
-                    if (blk >= 0 && blk < p.num_blocks) {
-                        constexpr int kChunks = D / 8;                    // 16-byte chunks per row
-                        // the caches are the caller's writable buffers (pa_append_decode)
-                        uint16_t* kc = const_cast<uint16_t*>(p.k_cache);
-                        uint16_t* vc = const_cast<uint16_t*>(p.v_cache);
-                        const size_t row0 = ((size_t)blk * Hkv + gi * kGroup) * Bs + (pos - lbn * Bs);
-                        const size_t src0 = ((size_t)b * Hkv + gi * kGroup) * D;
-                        if constexpr (F8) {
-                            // E4M3 pools: the new rows quantized with the caches' scales (K first
-                            // turned by RoPE and rounded to bf16 when the call asks for it)
-                            uint8_t* kq = reinterpret_cast<uint8_t*>(kc);
-                            uint8_t* vq = reinterpret_cast<uint8_t*>(vc);
-                            if (p.rope_theta > 0.f) {
-                                constexpr int kHalfChunks = D / 16;
-                                for (int i = lane; i < kGroup * kHalfChunks; i += 32) {
-                                    const int hh = i / kHalfChunks, cc = i - hh * kHalfChunks;
-                                    float cs[8], sn[8];
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) rope_cos_sin(pos, s_rope_inv[cc * 8 + e], &cs[e], &sn[e]);
-                                    const uint16_t* src = p.k_new + src0 + (size_t)hh * D + cc * 8;
-                                    uint4 x1 = __ldg(reinterpret_cast<const uint4*>(src));
-                                    uint4 x2 = __ldg(reinterpret_cast<const uint4*>(src + D / 2));
-                                    rope_rotate8(x1, x2, cs, sn);
-                                    uint8_t* dst = kq + (row0 + (size_t)hh * Bs) * D + cc * 8;
-                                    *reinterpret_cast<uint2*>(dst) = bf16x8_to_e4m3x8(x1, p.k_inv_scale);
-                                    *reinterpret_cast<uint2*>(dst + D / 2) = bf16x8_to_e4m3x8(x2, p.k_inv_scale);
-                                }
-                            }
-                            for (int i = lane; i < kGroup * kChunks; i += 32) {
-                                const int hh = i / kChunks, cc = i - hh * kChunks;
-                                const size_t dst = (row0 + (size_t)hh * Bs) * D + cc * 8;
-                                const size_t src = src0 + (size_t)hh * D + cc * 8;
-                                if (p.rope_theta <= 0.f)
-                                    *reinterpret_cast<uint2*>(kq + dst) = bf16x8_to_e4m3x8(
-                                        __ldg(reinterpret_cast<const uint4*>(p.k_new + src)), p.k_inv_scale);
-                                *reinterpret_cast<uint2*>(vq + dst) = bf16x8_to_e4m3x8(
-                                    __ldg(reinterpret_cast<const uint4*>(p.v_new + src)), p.v_inv_scale);
-                            }
-                        } else if (p.rope_theta > 0.f) {
-                            constexpr int kHalfChunks = D / 16;
-                            for (int i = lane; i < kGroup * kHalfChunks; i += 32) {
-                                const int hh = i / kHalfChunks, cc = i - hh * kHalfChunks;
-                                float cs[8], sn[8];
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) rope_cos_sin(pos, s_rope_inv[cc * 8 + e], &cs[e], &sn[e]);
-                                const uint16_t* src = p.k_new + src0 + (size_t)hh * D + cc * 8;
-                                uint4 x1 = __ldg(reinterpret_cast<const uint4*>(src));
-                                uint4 x2 = __ldg(reinterpret_cast<const uint4*>(src + D / 2));
-                                rope_rotate8(x1, x2, cs, sn);
-                                uint16_t* dst = kc + (row0 + (size_t)hh * Bs) * D + cc * 8;
-                                *reinterpret_cast<uint4*>(dst) = x1;
-                                *reinterpret_cast<uint4*>(dst + D / 2) = x2;
-                            }
-                        }
-                        for (int i = lane; i < kGroup * kChunks && !F8; i += 32) {
-                            const int hh = i / kChunks, cc = i - hh * kChunks;
-                            const size_t dst = (row0 + (size_t)hh * Bs) * D + cc * 8;
-                            const size_t src = src0 + (size_t)hh * D + cc * 8;
-                            if (p.rope_theta <= 0.f)
-                                reinterpret_cast<uint4*>(kc + dst)[0] = __ldg(reinterpret_cast<const uint4*>(p.k_new + src));
-                            reinterpret_cast<uint4*>(vc + dst)[0] = __ldg(reinterpret_cast<const uint4*>(p.v_new + src));
-                        }
-                    }
-                    // order these generic-proxy writes before the TMA reads of the slab
-                    asm volatile("fence.proxy.async.global;" ::: "memory");
-                    __syncwarp();
+                                    (first ? kFirst : 0) | (last ? kLast : 0) | (L == 0 ? kEmpty : 0) |
+                                        (seg_new ? kNew : 0),
+                                    seg_q, seg_nsplit, seg_slot, seg_ifirst, seg_fslot, L - 1, new_blk};
                 }
                 if (valid > 0) {
                     const int32_t nbox = (valid + tb - 1) / tb;
@@ -404,11 +370,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     for (int32_t x = 0; x < nbox; ++x) {
                         const int32_t tok = t0 + x * tb;
                         const int32_t lbk = tok / Bs;
-                        if (win_base < 0 || lbk >= win_base + 32) {      // warp-uniform refill
-                            win_base = lbk;
-                            const int32_t idx = win_base + lane;
-                            win_entry = idx < p.max_blocks_per_seq ? __ldg(table + idx) : -1;
-                        }
+                        if (win_base < 0 || lbk >= win_base + 32) refill(lbk);
                         const int32_t blk = __shfl_sync(0xffffffffu, win_entry, lbk - win_base);
                         if (lane == 0) {
                             int32_t z;
@@ -440,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                         ++gi;
                     }
                     if (s + 1 < hi) {
-                        L = clipped_length(p, b);
+                        L = clip_length(p, nx_len);
                         nb = L == 0 ? 1 : (L + kSlab - 1) / kSlab;
                     }
                 }
@@ -463,6 +425,10 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
         float m_run[NT][2], l_run[NT][2];
         float o_acc[NT][C::kMTiles][4];
         uint32_t qk = 0;
+        // fused append: this warp's kv head's new K and V rows, lane i < D/4 holding dims
+        // 2i, 2i+1 and D/2 + 2i, D/2 + 2i + 1 (the RoPE pairs of those dims), read when the
+        // segment starts and written when the stage holding the token arrives
+        uint32_t nk[2] = {0u, 0u}, nv[2] = {0u, 0u};
         // rows of this warp's 16 tokens: lane-provided ldmatrix row addresses
         const int row_a = stage_row(warp, rr + ((mi & 1) << 3), tb);     // K: tokens rr (+8)
         const int row_b = stage_row(warp, rr + ((mi >> 1) << 3), tb);    // V: tokens rr (+8)
@@ -525,10 +491,78 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&qempty_bar[qs]));
                 ++qk;
+                if (hd.flags & kNew) {
+                    const int i = lane < D / 4 ? lane : 0;
+                    const size_t row = ((size_t)hd.b * Hkv + kvh) * D / 2;
+                    const uint32_t* kn = reinterpret_cast<const uint32_t*>(p.k_new) + row;
+                    const uint32_t* vn = reinterpret_cast<const uint32_t*>(p.v_new) + row;
+                    nk[0] = __ldg(kn + i);
+                    nk[1] = __ldg(kn + D / 4 + i);
+                    nv[0] = __ldg(vn + i);
+                    nv[1] = __ldg(vn + D / 4 + i);
+                }
             }
             const int valid = hd.valid;
             uint32_t k_tile = smem_base + st * C::kStageBytes;
             uint32_t v_tile = k_tile + C::kTileBytes;
+            if (hd.new_blk >= 0 && hd.rope_pos >= hd.t0 && hd.rope_pos < hd.t0 + valid) {
+                // fused append: the stage holds the sequence's newest token.  Its K (turned by
+                // RoPE at that position when the call asks for it) and V rows go to the pool and
+                // over the staged copy, which may predate them.
+                if (lane < D / 4) {
+                    const int32_t pos = hd.rope_pos, Bs = p.block_size, t = pos - hd.t0;
+                    const int row = stage_row(warp, t, tb);
+                    const size_t grow = ((size_t)hd.new_blk * Hkv + kvh) * Bs + (pos - (pos / Bs) * Bs);
+                    uint32_t ka = nk[0], kb = nk[1];
+                    if (p.rope_theta > 0.f) {
+                        float c0, s0, c1, s1;
+                        rope_cos_sin(pos, s_rope_inv[2 * lane], &c0, &s0);
+                        rope_cos_sin(pos, s_rope_inv[2 * lane + 1], &c1, &s1);
+                        const float a0 = bf16_lo(ka), a1 = bf16_hi(ka), b0 = bf16_lo(kb), b1 = bf16_hi(kb);
+                        ka = pack_bf16x2(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
+                        kb = pack_bf16x2(a0 * s0 + b0 * c0, a1 * s1 + b1 * c1);
+                    }
+                    const int d0 = 2 * lane, d1 = D / 2 + 2 * lane;
+                    if constexpr (F8) {
+                        const float ks = p.k_inv_scale, vs = p.v_inv_scale;
+                        const uint32_t q0 = f32x2_to_e4m3x2(__fmul_rn(bf16_lo(ka), ks), __fmul_rn(bf16_hi(ka), ks));
+                        const uint32_t q1 = f32x2_to_e4m3x2(__fmul_rn(bf16_lo(kb), ks), __fmul_rn(bf16_hi(kb), ks));
+                        const uint32_t w0 = f32x2_to_e4m3x2(__fmul_rn(bf16_lo(nv[0]), vs), __fmul_rn(bf16_hi(nv[0]), vs));
+                        const uint32_t w1 = f32x2_to_e4m3x2(__fmul_rn(bf16_lo(nv[1]), vs), __fmul_rn(bf16_hi(nv[1]), vs));
+                        // the caches are the caller's writable buffers (pa_append_decode)
+                        uint8_t* kq = reinterpret_cast<uint8_t*>(const_cast<uint16_t*>(p.k_cache)) + grow * D;
+                        uint8_t* vq = reinterpret_cast<uint8_t*>(const_cast<uint16_t*>(p.v_cache)) + grow * D;
+                        *reinterpret_cast<uint16_t*>(kq + d0) = (uint16_t)q0;
+                        *reinterpret_cast<uint16_t*>(kq + d1) = (uint16_t)q1;
+                        *reinterpret_cast<uint16_t*>(vq + d0) = (uint16_t)w0;
+                        *reinterpret_cast<uint16_t*>(vq + d1) = (uint16_t)w1;
+                        uint8_t* kt = smem_gen + (k_tile - smem_base);
+                        uint8_t* vt = smem_gen + (k_tile + C::kTileBytesIn - smem_base);
+                        *reinterpret_cast<uint16_t*>(kt + f8_off<D>(row, d0 / 16) + d0 % 16) = (uint16_t)q0;
+                        *reinterpret_cast<uint16_t*>(kt + f8_off<D>(row, d1 / 16) + d1 % 16) = (uint16_t)q1;
+                        *reinterpret_cast<uint16_t*>(vt + f8_off<D>(row, d0 / 16) + d0 % 16) = (uint16_t)w0;
+                        *reinterpret_cast<uint16_t*>(vt + f8_off<D>(row, d1 / 16) + d1 % 16) = (uint16_t)w1;
+                    } else {
+                        uint32_t* kc = reinterpret_cast<uint32_t*>(const_cast<uint16_t*>(p.k_cache)) + grow * D / 2;
+                        uint32_t* vc = reinterpret_cast<uint32_t*>(const_cast<uint16_t*>(p.v_cache)) + grow * D / 2;
+                        kc[lane] = ka;
+                        kc[D / 4 + lane] = kb;
+                        vc[lane] = nv[0];
+                        vc[D / 4 + lane] = nv[1];
+                        auto at = [&](uint32_t tile, int d) {   // byte address of dim d in the row
+                            const int ch = d / 8;
+                            return swz(tile + (ch >> 3) * C::kHalfBytes, row, ch) + (uint32_t)((d % 8) * 2);
+                        };
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(at(k_tile, d0)), "r"(ka) : "memory");
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(at(k_tile, d1)), "r"(kb) : "memory");
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(at(v_tile, d0)), "r"(nv[0]) : "memory");
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(at(v_tile, d1)), "r"(nv[1]) : "memory");
+                    }
+                }
+                // generic writes to a stage the copy engine refills later: order them first
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+            }
             if constexpr (F8) {
                 if (valid < kSlab) {
                     // tokens past the sequence: zero their V bytes (0-probability rows add nothing)

@@ -47,9 +47,9 @@ __device__ __forceinline__ void raise_status(int32_t* status, int32_t bit) {
     if (status) atomicOr(status, bit);
 }
 
-// Context length of sequence b after clipping to what the grid and the table cover.
-__device__ __forceinline__ int32_t clipped_length(const DecodeParams& p, int32_t b) {
-    int32_t L = p.context_lens[b];
+// A context length as the decode uses it: negative or past what the table (and the call's
+// max_context_len) can hold is reported and clipped.
+__device__ __forceinline__ int32_t clip_length(const DecodeParams& p, int32_t L) {
     const int32_t table_cap = p.max_blocks_per_seq * p.block_size;
     const int32_t cap = p.max_context_len < table_cap ? p.max_context_len : table_cap;
     if (L < 0 || L > cap) {
@@ -57,6 +57,11 @@ __device__ __forceinline__ int32_t clipped_length(const DecodeParams& p, int32_t
         L = L < 0 ? 0 : cap;
     }
     return L;
+}
+
+// Context length of sequence b after clipping to what the grid and the table cover.
+__device__ __forceinline__ int32_t clipped_length(const DecodeParams& p, int32_t b) {
+    return clip_length(p, p.context_lens[b]);
 }
 
 // RoPE: pair i (of D/2) at position pos turns by a = pos * theta^(-2i/D).  The

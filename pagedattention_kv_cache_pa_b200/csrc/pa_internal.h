@@ -84,6 +84,7 @@ struct PrefillParams {
     int32_t* status;
     int32_t num_seqs, num_blocks, block_size, num_kv_heads, num_q_heads, head_dim, group;
     int32_t max_blocks_per_seq;
+    int32_t max_q_len;             // the caller's bound on every sequence's query count
     float scale_log2;
 };
 cudaError_t launch_prefill(const PrefillParams& p, int max_q_len, cudaStream_t stream);

@@ -39,6 +39,19 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t tmem_d, uint64_t adesc, ui
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]; issued by one thread.  A (M = 128 rows x 16 elements per
+// instruction) sits in tensor memory K-major: lane m = row m, each 32-bit column two
+// consecutive elements of the row, the lower index in the low half.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // One arrival on the mbarrier once every tcgen05 operation this thread issued so far
 // has completed (their shared-memory reads and tensor-memory writes included).
 __device__ __forceinline__ void umma_commit(uint32_t bar) {

@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(kThreadsPf) prefill_kernel(const PrefillParams
     const int L = p.context_lens[b];
     const int cap = p.max_blocks_per_seq * Bs;
     if (Tq <= 0) return;
-    if (L < Tq || L > cap) {                             // fewer tokens than queries, or past the table
+    if (L < Tq || L > cap || Tq > p.max_q_len) {         // fewer tokens than queries, past the table,
+                                                         // or more queries than the grid holds
         if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) raise_status(p.status, kStatusBadLength);
         return;
     }

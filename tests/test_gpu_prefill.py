@@ -122,3 +122,29 @@ def test_prefill_reports_bad_lengths_and_blocks(h, kernel):
     pa.pa_prefill(q, kc, vc, torch.from_numpy(bad).to(h.DEV), cu, lens, 5, b.scale, out, ws, desc, kernel=kernel)
     torch.cuda.synchronize()
     assert pa.pa_decode_status(ws) == -7
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_many_sequences_mixed_lengths(h, kernel):
+    # more than 32 sequences (the work-item search walks them 32 at a time), with empty
+    # chunks, single tokens, whole prompts and chunks after long caches mixed
+    rng = np.random.default_rng(7400)
+    q_lens = [int(x) for x in rng.choice([0, 1, 3, 64, 129, 300], size=70)]
+    lens = [t + int(rng.choice([0, 5, 200, 900])) for t in q_lens]
+    lens = [max(L, 1) for L in lens]
+    _run(h, 7401, lens, q_lens, kernel=kernel, num_q_heads=16, num_kv_heads=4, head_dim=64, block_size=16)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_reports_more_queries_than_max_q_len(h, kernel):
+    b = wl.small_batch(7500, [40, 30], num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16)
+    desc = h.desc_of(b)
+    q = torch.zeros((30, 4, 64), dtype=torch.bfloat16, device=h.DEV)
+    out = torch.zeros_like(q)
+    ws = torch.zeros(256, dtype=torch.uint8, device=h.DEV)
+    cu = torch.tensor([0, 10, 30], dtype=torch.int32, device=h.DEV)       # second: 20 queries
+    lens = torch.tensor([40, 30], dtype=torch.int32, device=h.DEV)
+    pa.pa_prefill(q, h.to_dev(b.k_cache), h.to_dev(b.v_cache), torch.from_numpy(b.block_tables).to(h.DEV), cu,
+                  lens, 10, b.scale, out, ws, desc, kernel=kernel)
+    torch.cuda.synchronize()
+    assert pa.pa_decode_status(ws) == -8
