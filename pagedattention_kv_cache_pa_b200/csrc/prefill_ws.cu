@@ -6,11 +6,13 @@
 // (Nano-vLLM page, section "Prefill vs Decode"; causal mask: Tiny-vLLM summary page,
 // section "고성능 추론을 위한 고급 최적화 기법").
 //
-// One CTA per (128 query rows, kv head, sequence), 6 warps with one job each, handing work
-// to one another through mbarriers only (no CTA-wide barrier inside the loop):
+// One CTA per (128 query rows, kv head, sequence), started row tile by row tile from the end
+// of every chunk, so the CTAs with the most keys run first.  6 warps with one job each hand
+// work to one another through mbarriers only (no CTA-wide barrier inside the loop):
 //   warps 0-3  softmax: thread i owns row i (tensor-memory lane i).  Per 64-key tile t it
 //              reads its row of S_t from tensor memory, masks it causally, and writes the
-//              probabilities P_t (bf16) into shared memory as the K-major A operand.
+//              probabilities P_t (bf16, two to a 32-bit column) back to tensor memory, where
+//              the P V MMA takes them as its A operand (no shared-memory round trip).
 //   warp 4     MMA issue (one thread): S_t = Q K_t^T into one of two score buffers in tensor
 //              memory two tiles ahead, and, once P_t is written, O += P_t V_t, accumulated in
 //              tensor memory across tiles.  The scores of the next tile are ready before the
@@ -22,8 +24,10 @@
 // it by more than 8 (log2 domain); only then is the row's O scaled by 2^(m - m_new) in
 // tensor memory (load, scale, store), after the P V of the previous tile has completed, and m
 // replaced.  In between, probabilities are 2^(s - m) <= 2^8, which bf16 and the fp32 sums
-// carry without loss of relative precision.  P has two buffers: P_t is written once the P V
-// of tile t-2, which read the same buffer, has completed.
+// carry without loss of relative precision.  P has two tensor-memory buffers: P_t is written
+// once the P V of tile t-2, which read the same buffer, has completed.
+// Tensor memory per CTA: S 2 x 64 columns, O D columns, P 2 x 32 columns (256 columns at
+// D = 64, two CTAs per SM; 512 at D = 128, one CTA per SM).
 //
 // Every wait is bounded (2 s, then the timeout status bit).  On a timeout each warp leaves
 // its loop; the MMA thread drains the TMA copies it has not seen land and waits for its own
@@ -49,26 +53,30 @@ constexpr float kRescaleLog2 = 8.f;
 
 template <int D>
 struct WsCfg {
-    static constexpr int kStages = D == 64 ? 3 : 2;         // K/V ring
+    // K/V ring.  The depth also bounds residency, so that no CTA's tensor-memory allocation
+    // waits for a neighbour's: D = 64 needs 80 KB (three CTAs would not fit in 228 KB, and two
+    // allocate 2 x 256 columns), D = 128 needs 128 KB (one CTA, 512 columns)
+    static constexpr int kStages = D == 64 ? 4 : 3;
     static constexpr int kQBytes = kWsRows * D * 2;
     static constexpr int kKVBytes = kWsKeys * D * 2;       // one K (or V) tile
-    static constexpr int kPBytes = kWsRows * kWsKeys * 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
-    static constexpr int kOffP = kOffV + kStages * kKVBytes;   // 2 buffers
-    static constexpr int kOffBar = kOffP + 2 * kPBytes;
+    static constexpr int kOffBar = kOffV + kStages * kKVBytes;
     // barriers (8 bytes each): s_full[2], p_full, o_done[2], drain, k_full[S], v_full[S],
     // kv_empty[S]; then the tensor-memory address and the last tile the TMA warp requested
     static constexpr int kBars = 6 + 3 * kStages;
     static constexpr int kSmem = kOffBar + kBars * 8 + 16;
     static constexpr int kColS = 0;                         // S: two buffers of 64 fp32 columns
     static constexpr int kColO = 128;                       // O: D fp32 columns
-    static constexpr uint32_t kTmemCols = 256;
+    static constexpr int kColP = kColO + D;                 // P: two buffers of 64 bf16 (32 columns)
+    static constexpr uint32_t kTmemCols = D == 64 ? 256 : 512;
     // D = 64: two CTAs per SM (each softmax thread keeps its row of S in 64 registers while it
-    // scales its row of O, which three CTAs of six warps would spill); D = 128: one (its
-    // shared memory)
+    // scales its row of O, which three CTAs of six warps would spill); D = 128: one
     static constexpr int kMinBlocks = D == 64 ? 2 : 1;
+    static_assert(kMinBlocks * (kSmem + 1024) <= 228 * 1024 && (kMinBlocks + 1) * (kSmem + 1024) > 228 * 1024,
+                  "shared memory must hold exactly kMinBlocks CTAs per SM");
+    static_assert(kMinBlocks * kTmemCols <= 512, "tensor memory of the resident CTAs");
 };
 
 template <int ROWS>
@@ -81,16 +89,30 @@ __device__ __forceinline__ void ws_cp_async16(uint32_t dst, const void* src, boo
                  : "memory");
 }
 
-// 2^x on the FMA pipe, for x <= 8: x = n + f with n = floor(x), 2^f from a cubic fitted to
-// it on [0, 1) (relative error below 9e-5, under the bf16 rounding the probabilities get), and
-// n added to the exponent field.  0 below 2^-126.  Some of each row's exponentials take this
-// path so that they do not all queue on the special-function unit.
-__device__ __forceinline__ float exp2_fma(float x) {
-    const float xc = fmaxf(x, -126.f);
-    const float n = floorf(xc), f = xc - n;
-    const float p = fmaf(fmaf(fmaf(0.0770652f, f, 0.227647f), f, 0.69511634f), f, 1.f);
-    const float r = __int_as_float(__float_as_int(p) + ((int)n << 23));
-    return x < -126.f ? 0.f : r;
+// Row arithmetic two lanes at a time: three-input maximum and packed fp32 pairs (one
+// instruction for two FMAs or two adds).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
 // 32 columns of this thread's lane of tensor memory, scaled by a and stored back.
@@ -102,7 +124,7 @@ __device__ __forceinline__ void tmem_scale32(uint32_t taddr, float a) {
     tmem_st32(taddr, r);
 }
 
-template <int D, int kPolyPairs>
+template <int D>
 __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
     prefill_ws_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap) {
@@ -111,31 +133,34 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t s_base = smem_u32(smem);
     const uint32_t s_q = s_base + C::kOffQ, s_k = s_base + C::kOffK, s_v = s_base + C::kOffV;
-    const uint32_t s_p = s_base + C::kOffP;
     constexpr int ST = C::kStages;
     const uint32_t bar_s = s_base + C::kOffBar, bar_p = bar_s + 16, bar_o = bar_s + 24,
                    bar_drain = bar_s + 40, bar_k = bar_s + 48, bar_v = bar_k + 8 * ST, bar_e = bar_v + 8 * ST;
     const uint32_t s_tmem = bar_s + C::kBars * 8;
     volatile int* s_kreq = reinterpret_cast<volatile int*>(smem + C::kOffBar + C::kBars * 8 + 4);
 
-    const int b = blockIdx.z, kvh = blockIdx.y;
-    const int G = p.group, Hq = p.num_q_heads, Hkv = p.num_kv_heads, Bs = p.block_size;
+    // CTA (x, y): sequence b = x / Hkv, kv head x % Hkv, the y-th row tile from the end of the
+    // chunk (the last row tiles attend to the most keys; the hardware starts the CTAs with x
+    // fastest, so every sequence's longest tiles run first)
+    const int Hkv = p.num_kv_heads;
+    const int b = (int)(blockIdx.x / (unsigned)Hkv), kvh = (int)(blockIdx.x - (unsigned)b * Hkv);
+    const int G = p.group, Hq = p.num_q_heads, Bs = p.block_size;
     const int q0 = p.cu_q[b], Tq = p.cu_q[b + 1] - q0;
     const int L = p.context_lens[b];
-    const int cap = p.max_blocks_per_seq * Bs;
     if (Tq <= 0) return;
-    if (L < Tq || L > cap) {
-        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) raise_status(p.status, kStatusBadLength);
+    if (L < Tq || L > p.max_blocks_per_seq * Bs || Tq > p.max_q_len) {
+        // fewer tokens than queries, past the table, or more queries than the grid holds
+        if (threadIdx.x == 0 && blockIdx.y == 0 && kvh == 0) raise_status(p.status, kStatusBadLength);
         return;
     }
     if (s_base & 1023u) {                                    // the swizzle needs 1024-byte-aligned tiles
         if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
         return;
     }
-    // the last row tiles of a chunk attend to the most keys: they take the first CTAs
-    const int rows = Tq * G, ntile = (rows + kWsRows - 1) / kWsRows;
-    const int tile = ntile - 1 - (int)blockIdx.x;
+    const int ntile = (Tq * G + kWsRows - 1) / kWsRows;
+    const int tile = ntile - 1 - (int)blockIdx.y;
     if (tile < 0) return;
+    const int rows = Tq * G;
     const int r0 = tile * kWsRows;
     const int* table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -185,6 +210,9 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
     if (warp == 5) {
         // ================================ TMA ================================
         const int rb = Bs < kWsKeys ? Bs : kWsKeys, nslot = kWsKeys / rb;
+        // K tile t into K stage t % ST once S_{t-ST} has completed; V tile t into its stage once
+        // P_{t-ST} V_{t-ST} has.  K runs two tiles ahead of V, in the order the MMA thread
+        // takes them (P_t V_t, then S_{t+2}).
         for (int t = 0; t < ntiles && !failed; ++t) {
             const int st = t % ST;
             if (t >= ST) {                                   // the MMAs of tile t - ST have completed
@@ -246,12 +274,12 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
                 umma_commit(bar_s + 8 * (t & 1));
             };
             auto issue_o = [&](int t) {                      // O += P_t V_t over 4 K steps of 16 keys
-                const uint32_t vt = s_v + (t % ST) * C::kKVBytes, pt = s_p + (t & 1) * C::kPBytes;
+                const uint32_t vt = s_v + (t % ST) * C::kKVBytes;
+                const uint32_t pt = tmem + C::kColP + (t & 1) * (kWsKeys / 2);   // P_t in tensor memory
 #pragma unroll
                 for (int kk = 0; kk < kWsKeys / 16; ++kk) {
-                    const uint64_t a = umma_desc_sw128(pt + kk * 32, 16, 1024);
                     const uint64_t bd = umma_desc_sw128(vt + kk * 16 * 128, kWsKeys * 128, 1024);
-                    umma_bf16_ss(tmem + C::kColO, a, bd, kIdescO, (t > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(tmem + C::kColO, pt + kk * 8, bd, kIdescO, (t > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(bar_e + 8 * (t % ST));           // K_t and V_t are free once these land
                 umma_commit(bar_o + 8 * (t & 1));
@@ -304,21 +332,18 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
             uint32_t sr[64];
             tmem_ld64(t_lane + C::kColS + (t & 1) * 64, sr);
             const int k0 = t * kWsKeys;
-            // the row max over four independent chains (a single chain of 64 dependent maxima
-            // would sit on the tile's critical path)
-            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             if (k0 + kWsKeys - 1 > pos_first) {              // a tile on the diagonal: mask
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const float v = k0 + j <= pos ? __uint_as_float(sr[j]) : -INFINITY;
-                    sr[j] = __float_as_uint(v);
-                    mq[j & 3] = fmaxf(mq[j & 3], v);
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 64; ++j) mq[j & 3] = fmaxf(mq[j & 3], __uint_as_float(sr[j]));
+                for (int j = 0; j < 64; ++j)
+                    if (k0 + j > pos) sr[j] = __float_as_uint(-INFINITY);
             }
-            const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            // the row max over four independent chains of three-input maxima (a single chain
+            // of dependent maxima would sit on the tile's critical path)
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int j = 0; j < 64; j += 2)
+                mq[(j >> 1) & 3] = fmax3(mq[(j >> 1) & 3], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+            const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
             // key 0 is in every row's range, so the max is finite from the first tile on
             const float m_new = fmaxf(m_run, mx * sl2);
             if (t == 0) {
@@ -341,28 +366,28 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
                     }
                 }
             }
-            float rs[4] = {0.f, 0.f, 0.f, 0.f};            // four independent partial sums
+            // p = 2^(s sl2 - m) for two keys per packed FMA; the row sum in two independent
+            // packed partial sums
+            const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(-m_run, -m_run);
+            uint64_t rs2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
             uint32_t pk[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float x0 = fmaf(__uint_as_float(sr[2 * j]), sl2, -m_run);
-                const float x1 = fmaf(__uint_as_float(sr[2 * j + 1]), sl2, -m_run);
-                const float p0 = j < kPolyPairs ? exp2_fma(x0) : fast_exp2(x0);
-                const float p1 = j < kPolyPairs ? exp2_fma(x1) : fast_exp2(x1);
-                rs[j & 3] += p0 + p1;
+                float x0, x1;
+                f2_split(f2_fma(f2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])), sc2, nm2), x0, x1);
+                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                rs2[j & 1] = f2_add(rs2[j & 1], f2(p0, p1));
                 pk[j] = pack_bf16x2(p0, p1);
             }
-            l_run += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+            float r0a, r0b, r1a, r1b;
+            f2_split(rs2[0], r0a, r0b);
+            f2_split(rs2[1], r1a, r1b);
+            l_run += (r0a + r1a) + (r0b + r1b);
             if (t >= 2 && !wait_o(t - 2)) {                 // the P V that read this P buffer is done
                 failed = true;
                 break;
             }
-            const uint32_t prow = s_p + (t & 1) * C::kPBytes + tid * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + ((c ^ (tid & 7)) << 4)),
-                             "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                             : "memory");
+            tmem_st32(t_lane + C::kColP + (t & 1) * (kWsKeys / 2), pk);   // P_t: this row's 64 bf16
             if (L - k0 < kWsKeys) {
                 // the last tile: V rows past the sequence (stale pool rows, or never copied)
                 // are zeroed so that P = 0 there cannot meet a NaN pattern; the MMA reads V
@@ -378,8 +403,8 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
                                  "r"(0u)
                                  : "memory");
                 }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_p);
@@ -460,17 +485,14 @@ bool ws_pool_map(CUtensorMap* map, const void* base, const PrefillParams& p) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Pairs of each row's 64 exponentials per tile computed on the FMA pipe (exp2_fma).
-constexpr int kWsPolyPairs = 0;
-
-template <int D, int kPoly = kWsPolyPairs>
+template <int D>
 cudaError_t launch_ws(const PrefillParams& p, int max_q_len, cudaStream_t stream) {
     constexpr size_t smem = WsCfg<D>::kSmem;
     static std::atomic<uint64_t> attr_set{0};               // one bit per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!(attr_set.load(std::memory_order_acquire) & (1ull << dev))) {
-        const cudaError_t e = cudaFuncSetAttribute(prefill_ws_kernel<D, kPoly>,
+        const cudaError_t e = cudaFuncSetAttribute(prefill_ws_kernel<D>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_set.fetch_or(1ull << dev, std::memory_order_acq_rel);
@@ -481,8 +503,9 @@ cudaError_t launch_ws(const PrefillParams& p, int max_q_len, cudaStream_t stream
     memset(&km, 0, sizeof km);
     memset(&vm, 0, sizeof vm);
     if (!ws_pool_map(&km, p.k_cache, p) || !ws_pool_map(&vm, p.v_cache, p)) return cudaErrorInvalidValue;
-    dim3 grid((unsigned)tiles, (unsigned)p.num_kv_heads, (unsigned)p.num_seqs);
-    prefill_ws_kernel<D, kPoly><<<grid, kWsThreads, smem, stream>>>(p, km, vm);
+    if ((int64_t)p.num_seqs * p.num_kv_heads > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)(p.num_seqs * p.num_kv_heads), (unsigned)tiles, 1u);
+    prefill_ws_kernel<D><<<grid, kWsThreads, smem, stream>>>(p, km, vm);
     return cudaGetLastError();
 }
 
