@@ -71,6 +71,11 @@ struct SCfg {
 // kNew: the segment that starts at this stage holds the sequence's newest token (fused append)
 enum : int32_t { kFirst = 1, kLast = 2, kEmpty = 4, kEnd = 8, kNew = 16 };
 
+// Lazy running max: a slab rescales O only when a score passes the running max by more than
+// this (log2 domain); probabilities up to 2^8 keep bf16 / f16 P and the fp32 sums exact in
+// relative terms.
+constexpr float kLazyLog2 = 8.f;
+
 // Slabs an early-launched CTA prefetches into L2 before it waits for the previous kernel.
 constexpr int32_t kPrefetchSlabs = 2;
 
@@ -276,6 +281,18 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 prefetch_win2();
             };
             prefetch_win2();
+            int q_next = -1;                                 // q ring slot already requested
+            auto issue_q = [&](int32_t bq, int32_t gq, int& slot) -> bool {
+                if (!acquire(qempty_bar, qk, kQSlots, slot)) return false;
+                if (lane == 0) {
+                    const uint32_t bar = smem_u32(&qfull_bar[slot]);
+                    mbar_arrive_expect_tx(bar, q_slot_bytes);
+                    bulk_load(q_base + slot * q_slot_bytes,
+                              p.q + ((size_t)bq * p.num_q_heads + (size_t)gq * kGroup * G) * D, q_slot_bytes, bar);
+                }
+                ++qk;
+                return true;
+            };
             if (p.early) {
                 // launched early: pull the first slabs of the slice (inside the first sequence
                 // and the fetched table window) into L2 while the previous kernel finishes
@@ -326,18 +343,22 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     }
                     // fused append: this segment holds the sequence's newest token
                     seg_new = p.k_new != nullptr && L > 0 && s + (nb - 1 - j) < hi;
-                    if (L > 0) {
-                        int qs;
-                        if (!acquire(qempty_bar, qk, kQSlots, qs)) { alive = false; break; }
-                        seg_q = qs;
-                        if (lane == 0) {
-                            const uint32_t bar = smem_u32(&qfull_bar[qs]);
-                            mbar_arrive_expect_tx(bar, q_slot_bytes);
-                            bulk_load(q_base + qs * q_slot_bytes,
-                                      p.q + ((size_t)b * p.num_q_heads + (size_t)gi * kGroup * G) * D,
-                                      q_slot_bytes, bar);
+                    // q of every segment (empty sequences' too): requested at the previous
+                    // sequence's start when the slice ran on into this one, else now; then the
+                    // next sequence's q, if the slice reaches it
+                    if (q_next >= 0) {
+                        seg_q = q_next;
+                        q_next = -1;
+                    } else if (!issue_q(b, gi, seg_q)) {
+                        alive = false;
+                        break;
+                    }
+                    if (s + (nb - j) < hi) {
+                        const bool wrap = b + 1 == B;
+                        if (!issue_q(wrap ? 0 : b + 1, wrap ? gi + 1 : gi, q_next)) {
+                            alive = false;
+                            break;
                         }
-                        ++qk;
                     }
                 }
                 int st;
@@ -441,6 +462,13 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             if (hd.flags & kEmpty) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+                if (hd.flags & kFirst) {                     // its q slot, unread
+                    const int qs = qk % kQSlots;
+                    if (!warp_wait(smem_u32(&qfull_bar[qs]), (qk / kQSlots) & 1, p.status, p.wait_ns)) break;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&qempty_bar[qs]));
+                    ++qk;
+                }
                 store_zero_group(p, hd.b, kvh, lane, 32);
                 continue;
             }
@@ -622,34 +650,53 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             }
             // ---- online softmax over the 16 rows (tokens) per head column ----
             const bool v_lo = r < valid, v_hi = (r + 8) < valid;
+            // The running max m is kept lazily: while every score of the slab stays within
+            // 2^kLazyLog2 of its head's m (log2 domain), the slab is weighted by 2^(s - m) as m
+            // stands, with no cross-lane maximum and no rescale of O.  Otherwise (always on a
+            // segment's first slab, where m = -inf) m moves to the maximum over the slab.
+            float sv[NT][4], mx[NT][2];
+            bool need = false;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                sv[nt][0] = v_lo ? sacc[nt][0] * sl2 : -INFINITY;
+                sv[nt][1] = v_lo ? sacc[nt][1] * sl2 : -INFINITY;
+                sv[nt][2] = v_hi ? sacc[nt][2] * sl2 : -INFINITY;
+                sv[nt][3] = v_hi ? sacc[nt][3] * sl2 : -INFINITY;
+                mx[nt][0] = fmaxf(sv[nt][0], sv[nt][2]);
+                mx[nt][1] = fmaxf(sv[nt][1], sv[nt][3]);
+                need |= mx[nt][0] > m_run[nt][0] + kLazyLog2 || mx[nt][1] > m_run[nt][1] + kLazyLog2;
+            }
+            if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float mx0 = mx[nt][0], mx1 = mx[nt][1];
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                    }
+                    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+                    const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
+                    m_run[nt][0] = mn0;
+                    m_run[nt][1] = mn1;
+                    l_run[nt][0] *= al0;
+                    l_run[nt][1] *= al1;
+#pragma unroll
+                    for (int mt = 0; mt < C::kMTiles; ++mt) {
+                        o_acc[nt][mt][0] *= al0;
+                        o_acc[nt][mt][1] *= al1;
+                        o_acc[nt][mt][2] *= al0;
+                        o_acc[nt][mt][3] *= al1;
+                    }
+                }
+            }
             uint32_t pb[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const float s0 = v_lo ? sacc[nt][0] * sl2 : -INFINITY;
-                const float s1 = v_lo ? sacc[nt][1] * sl2 : -INFINITY;
-                const float s2 = v_hi ? sacc[nt][2] * sl2 : -INFINITY;
-                const float s3 = v_hi ? sacc[nt][3] * sl2 : -INFINITY;
-                float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-                }
-                const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-                const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
-                m_run[nt][0] = mn0;
-                m_run[nt][1] = mn1;
-                const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
-                const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
-                l_run[nt][0] = l_run[nt][0] * al0 + (p0 + p2);
-                l_run[nt][1] = l_run[nt][1] * al1 + (p1 + p3);
-#pragma unroll
-                for (int mt = 0; mt < C::kMTiles; ++mt) {
-                    o_acc[nt][mt][0] *= al0;
-                    o_acc[nt][mt][1] *= al1;
-                    o_acc[nt][mt][2] *= al0;
-                    o_acc[nt][mt][3] *= al1;
-                }
+                const float p0 = fast_exp2(sv[nt][0] - m_run[nt][0]), p1 = fast_exp2(sv[nt][1] - m_run[nt][1]);
+                const float p2 = fast_exp2(sv[nt][2] - m_run[nt][0]), p3 = fast_exp2(sv[nt][3] - m_run[nt][1]);
+                l_run[nt][0] += p0 + p2;
+                l_run[nt][1] += p1 + p3;
                 pb[nt][0] = movmatrix_trans(pack_p<F8>(p0, p1));   // tokens 0-7
                 pb[nt][1] = movmatrix_trans(pack_p<F8>(p2, p3));   // tokens 8-15
             }
