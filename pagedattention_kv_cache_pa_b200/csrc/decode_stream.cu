@@ -108,11 +108,12 @@ __device__ __forceinline__ int32_t cta_of(int64_t s, int64_t S, int64_t G) {
     return (int32_t)(((s + 1) * G - 1) / S);
 }
 
-// Two E4M3 codes (the low 16 bits) -> two f16 (exact: every E4M3 value is an f16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes) {
-    uint32_t h2;
-    asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e4m3x2 %0, c; }" : "=r"(h2) : "r"(codes & 0xFFFFu));
-    return h2;
+// Four E4M3 codes -> two f16 pairs (exact: every E4M3 value is an f16 value): codes 0,1 (low
+// half-word) and codes 2,3 (high half-word), one conversion per half-word register.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %2; cvt.rn.f16x2.e4m3x2 %0, l; cvt.rn.f16x2.e4m3x2 %1, h; }"
+        : "=r"(lo), "=r"(hi)
+        : "r"(codes));
 }
 // Byte offset of (row, 16-byte chunk) in an E4M3 tile as TMA writes it: 64-byte rows (D=64)
 // under the 64B swizzle (chunk ^= (row >> 1) & 3), 128-byte rows (D=128) under the 128B one.
@@ -631,8 +632,9 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     ldmatrix_x4(k_tile + f8_off<D>(row_a, ks + (mi >> 1)), w);
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
-                        const uint32_t a[4] = {e4m3x2_to_f16x2(w[2 * h2]), e4m3x2_to_f16x2(w[2 * h2 + 1]),
-                                               e4m3x2_to_f16x2(w[2 * h2] >> 16), e4m3x2_to_f16x2(w[2 * h2 + 1] >> 16)};
+                        uint32_t a[4];
+                        e4m3x4_to_f16x2x2(w[2 * h2], a[0], a[2]);
+                        e4m3x4_to_f16x2x2(w[2 * h2 + 1], a[1], a[3]);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt)
                             mma_16816<F8>(sacc[nt], a, qf[nt][ks + h2][0], qf[nt][ks + h2][1]);
@@ -710,14 +712,10 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 for (int j = 0; j < D / 32; ++j) {
                     uint32_t w[4];
                     ldmatrix_x4_trans(f8v + f8_off<D>(row_b, 2 * j + (mi & 1)), w);
-                    const uint32_t ae[4] = {e4m3x2_to_f16x2(__byte_perm(w[0], 0u, 0x20u)),
-                                            e4m3x2_to_f16x2(__byte_perm(w[1], 0u, 0x20u)),
-                                            e4m3x2_to_f16x2(__byte_perm(w[2], 0u, 0x20u)),
-                                            e4m3x2_to_f16x2(__byte_perm(w[3], 0u, 0x20u))};
-                    const uint32_t ao[4] = {e4m3x2_to_f16x2(__byte_perm(w[0], 0u, 0x31u)),
-                                            e4m3x2_to_f16x2(__byte_perm(w[1], 0u, 0x31u)),
-                                            e4m3x2_to_f16x2(__byte_perm(w[2], 0u, 0x31u)),
-                                            e4m3x2_to_f16x2(__byte_perm(w[3], 0u, 0x31u))};
+                    uint32_t ae[4], ao[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)   // bytes 0, 2 (even dims) low, 1, 3 (odd dims) high
+                        e4m3x4_to_f16x2x2(__byte_perm(w[i], 0u, 0x3120u), ae[i], ao[i]);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
                         mma_16816<F8>(o_acc[nt][2 * j], ae, pb[nt][0], pb[nt][1]);
