@@ -328,10 +328,11 @@ PA_API int32_t pa_decode_max_splits(int32_t num_seqs, int32_t max_context_len, c
  *  kernel:       PA_KERNEL_TENSOR for the stream-partitioned whole-group kernel (Hkv a
  *                multiple of 8), PA_KERNEL_TENSOR_SPLIT or PA_KERNEL_SIMT for the split ones.
  *  ctas:         stream kernel: CTAs of its persistent grid.  The work is the concatenation,
- *                over groups of 8 kv heads and then sequences, of 16-token slabs (an empty
- *                sequence counts one); CTA i of G = min(ctas, slabs S) takes slabs
- *                [i S / G, (i + 1) S / G).  0 for the split kernels.
- *  split_tokens: split kernels: tokens per split (split k covers [k C, (k + 1) C)); else 0.
+ *                over groups of 8 kv heads and then sequences, of slabs of split_tokens
+ *                tokens (an empty sequence counts one); CTA i of G = min(ctas, slabs S) takes
+ *                slabs [i S / G, (i + 1) S / G).  0 for the split kernels.
+ *  split_tokens: split kernels: tokens per split (split k covers [k C, (k + 1) C)); stream
+ *                kernel: tokens per slab (32 for E4M3 pools with head_dim 64, else 16).
  *  max_splits:   split kernels: splits per (sequence, kv head) at most; else 1.
  * Returns PA_OK, or the error the decode call itself would return for these arguments.
  */

@@ -339,7 +339,9 @@ extern "C" int pa_decode_describe(int32_t num_seqs, int32_t max_context_len, con
                   : plan.kernel == DecodeKernel::kSplit ? PA_KERNEL_TENSOR_SPLIT
                                                         : PA_KERNEL_SIMT;
     out->ctas = plan.kernel == DecodeKernel::kStream ? plan.grid : 0;
-    out->split_tokens = plan.kernel == DecodeKernel::kStream ? 0 : plan.split_tokens;
+    out->split_tokens = plan.kernel == DecodeKernel::kStream
+                            ? stream_slab_tokens(options && options->kv_dtype == PA_KV_E4M3, desc->head_dim)
+                            : plan.split_tokens;
     out->max_splits = plan.max_splits;
     return PA_OK;
 }

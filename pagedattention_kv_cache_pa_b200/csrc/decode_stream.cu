@@ -40,13 +40,17 @@ namespace {
 
 constexpr int kGroup = 8;                    // kv heads per CTA = consumer warps
 constexpr int kThreads = (kGroup + 1) * 32;
-constexpr int kSlab = 16;                    // tokens per stage
+constexpr int kSlab = 16;                    // tokens per stage (bf16 pools, E4M3 at D=128)
 constexpr int kRowBytes = 128;               // 64 bf16 of head dim, one swizzled row
 constexpr int kQSlots = 2;
 
 template <int D, int NT, bool F8 = false>
 struct SCfg {
     static constexpr int kHalves = D / 64;
+    // tokens per stage: E4M3 stages at D=64 hold 32 (the 16 KB of a bf16 stage), so that the
+    // per-stage waits, votes and releases are spread over twice the tokens
+    static constexpr int kSlab = (F8 && D == 64) ? 32 : ::pa::kSlab;
+    static constexpr int kMT = kSlab / 16;                           // 16-token M tiles per stage
     static constexpr int kHalfBytes = kGroup * kSlab * kRowBytes;   // 16 KB
     static constexpr int kTileBytes = kHalves * kHalfBytes;         // bf16 K (or V) of a stage
     // as loaded: bf16 in 128-byte swizzled rows (one box per 64 dims), or E4M3 in plain D-byte rows
@@ -57,7 +61,7 @@ struct SCfg {
     // E4M3 stages carry half the bytes: more of them keep as many bytes in flight, except at
     // D=128, G<=8, where two CTAs of two stages per SM beat one of five (a CTA retires TMA
     // requests at a bounded rate, so more CTAs issue more of them)
-    static constexpr int kStages = F8 ? (D == 64 ? (NT == 1 ? 6 : 4) : (NT == 1 ? 2 : 4))
+    static constexpr int kStages = F8 ? (D == 64 ? (NT == 1 ? 3 : 2) : (NT == 1 ? 2 : 4))
                                       : ((D == 128 && NT == 2) ? 2 : 3);
     static constexpr int kKSteps = D / 16;
     static constexpr int kMTiles = D / 16;
@@ -98,9 +102,10 @@ __device__ __forceinline__ uint32_t swz(uint32_t half_tile, int row, int chunk) 
     return half_tile + row * kRowBytes + (((chunk & 7) ^ (row & 7)) << 4);
 }
 
+template <int SL>
 __device__ __forceinline__ int32_t nslabs(const DecodeParams& p, int32_t b) {
     const int32_t L = clipped_length(p, b);
-    return L == 0 ? 1 : (L + kSlab - 1) / kSlab;
+    return L == 0 ? 1 : (L + SL - 1) / SL;
 }
 
 // CTA whose slice holds slab s (slices: [floor(i S / G), floor((i+1) S / G)) ).
@@ -137,6 +142,11 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 template <bool F8>
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
     if constexpr (F8) return pack_f16x2(lo, hi); else return pack_bf16x2(lo, hi);
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 // Two floats -> two E4M3 codes (nearest even, saturating), the first in the low byte.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
@@ -192,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
     } else if (warp == kGroup) {
         // ================================ producer ================================
         const int32_t B = p.num_seqs, Bs = p.block_size;
-        const int32_t tb = Bs < kSlab ? Bs : kSlab;             // tokens per TMA box
+        constexpr int32_t SL = C::kSlab;
+        const int32_t tb = Bs < SL ? Bs : SL;                   // tokens per TMA box
         const int32_t groups = Hkv / kGroup;
         const int32_t zmax = p.num_blocks * Hkv;                // z extent of the maps
         const uint64_t kv_policy = l2_evict_first_policy();      // K/V are read once
@@ -203,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
         const int32_t c_lo = min(B, lane * cs), c_hi = min(B, c_lo + cs);
         int64_t lane_sum = 0;
 #pragma unroll 4
-        for (int32_t b = c_lo; b < c_hi; ++b) lane_sum += nslabs(p, b);
+        for (int32_t b = c_lo; b < c_hi; ++b) lane_sum += nslabs<SL>(p, b);
         int64_t incl = lane_sum;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -240,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             if (lane == k) {
                 int64_t acc = excl;
                 for (int32_t bb = c_lo; bb < c_hi; ++bb) {
-                    const int32_t n = nslabs(p, bb);
+                    const int32_t n = nslabs<SL>(p, bb);
                     if (r < acc + n) {
                         b = bb;
                         j = (int32_t)(r - acc);
@@ -254,12 +265,12 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
             j = __shfl_sync(0xffffffffu, j, k);
             P = __shfl_sync(0xffffffffu, P, k);
             int32_t L = clipped_length(p, b);
-            int32_t nb = L == 0 ? 1 : (L + kSlab - 1) / kSlab;
+            int32_t nb = L == 0 ? 1 : (L + SL - 1) / SL;
             // segment state
             int32_t seg_nsplit = 1, seg_slot = 0, seg_ifirst = 0, seg_fslot = 0, seg_q = 0;
             const int32_t* table = p.block_tables + (size_t)b * p.max_blocks_per_seq;
             // the first table window, fetched while a prerequisite grid may still run
-            int32_t win_base = (j * kSlab) / Bs, win_entry = -1;
+            int32_t win_base = (j * SL) / Bs, win_entry = -1;
             if (win_base + lane < p.max_blocks_per_seq) win_entry = __ldg(table + win_base + lane);
             // Loads issued ahead so that no copy waits on one: the window after the current one
             // (nx_win2), and, once a slice reaches the next sequence of the stream, that
@@ -299,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 // and the fetched table window) into L2 while the previous kernel finishes
                 const int32_t pf_end = min(min((int64_t)nb, (int64_t)j + (hi - lo)), (int64_t)j + kPrefetchSlabs);
                 for (int32_t jj = j; jj < pf_end && L > 0; ++jj) {
-                    const int32_t t0 = jj * kSlab, valid = min(kSlab, L - t0);
+                    const int32_t t0 = jj * SL, valid = min(SL, L - t0);
                     for (int32_t x = 0; x * tb < valid; ++x) {
                         const int32_t tok = t0 + x * tb, lbk = tok / Bs;
                         if (lbk - win_base >= 32) break;
@@ -364,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 }
                 int st;
                 if (!acquire(empty_bar, gtile, C::kStages, st)) { alive = false; break; }
-                const int32_t t0 = j * kSlab;
-                const int32_t valid = L == 0 ? 0 : min(kSlab, L - t0);
+                const int32_t t0 = j * SL;
+                const int32_t valid = L == 0 ? 0 : min(SL, L - t0);
                 const uint32_t fbar = smem_u32(&full_bar[st]);
                 // fused append: the stage that holds the newest token (position L-1) carries its
                 // physical block; the consumer warps write the new K/V rows to the pool and into
@@ -425,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     }
                     if (s + 1 < hi) {
                         L = clip_length(p, nx_len);
-                        nb = L == 0 ? 1 : (L + kSlab - 1) / kSlab;
+                        nb = L == 0 ? 1 : (L + SL - 1) / SL;
                     }
                 }
             }
@@ -441,7 +452,8 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
         // warp w owns kv head kvh0 + w of every stage
         const int r = lane >> 2, c = lane & 3;
         const int mi = lane >> 3, rr = lane & 7;
-        const int32_t tb = p.block_size < kSlab ? p.block_size : kSlab;
+        constexpr int32_t SL = C::kSlab;
+        const int32_t tb = p.block_size < SL ? p.block_size : SL;
         const float sl2 = p.scale_log2;
         uint32_t qf[NT][C::kKSteps][2];
         float m_run[NT][2], l_run[NT][2];
@@ -452,8 +464,13 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
         // segment starts and written when the stage holding the token arrives
         uint32_t nk[2] = {0u, 0u}, nv[2] = {0u, 0u};
         // rows of this warp's 16 tokens: lane-provided ldmatrix row addresses
-        const int row_a = stage_row(warp, rr + ((mi & 1) << 3), tb);     // K: tokens rr (+8)
-        const int row_b = stage_row(warp, rr + ((mi >> 1) << 3), tb);    // V: tokens rr (+8)
+        // per 16-token M tile u of a stage: K rows of tokens 16u + rr (+8), V rows likewise
+        int row_a[C::kMT], row_b[C::kMT];
+#pragma unroll
+        for (int u = 0; u < C::kMT; ++u) {
+            row_a[u] = stage_row(warp, 16 * u + rr + ((mi & 1) << 3), tb);
+            row_b[u] = stage_row(warp, 16 * u + rr + ((mi >> 1) << 3), tb);
+        }
         for (uint32_t gtile = 0;; ++gtile) {
             const int st = gtile % C::kStages;
             if (!warp_wait(smem_u32(&full_bar[st]), (gtile / C::kStages) & 1, p.status, p.wait_ns)) break;
@@ -593,10 +610,10 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 __syncwarp();
             }
             if constexpr (F8) {
-                if (valid < kSlab) {
+                if (valid < SL) {
                     // tokens past the sequence: zero their V bytes (0-probability rows add nothing)
                     const uint32_t f8v = k_tile + C::kTileBytesIn;
-                    for (int i = lane; i < (kSlab - valid) * (D / 16); i += 32) {
+                    for (int i = lane; i < (SL - valid) * (D / 16); i += 32) {
                         const int t = valid + i / (D / 16), ch = i % (D / 16);
                         *reinterpret_cast<uint4*>(smem_gen + (f8v - smem_base) + f8_off<D>(stage_row(warp, t, tb), ch)) =
                             make_uint4(0, 0, 0, 0);
@@ -604,9 +621,9 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                 }
-            } else if (valid < kSlab) {
+            } else if (valid < SL) {
                 // tokens past the sequence: zero V so that 0-probability rows add nothing
-                for (int i = lane; i < (kSlab - valid) * 8 * C::kHalves; i += 32) {
+                for (int i = lane; i < (SL - valid) * 8 * C::kHalves; i += 32) {
                     const int t = valid + i / (8 * C::kHalves);
                     const int ch = i % (8 * C::kHalves);
                     const int row = stage_row(warp, t, tb);
@@ -617,57 +634,67 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
             }
-            // ---- S = K q^T : 16 tokens x 8 heads per n-tile ----
-            float sacc[NT][4];
+            // ---- S = K q^T : 16 tokens x 8 heads per (M tile, n-tile) ----
+            float sacc[C::kMT][NT][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int u = 0; u < C::kMT; ++u) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-            if constexpr (F8) {
-                // E4M3 K straight from the tile: one ldmatrix.x4 brings 16 tokens x 32 dims of
-                // codes (lane (r, c): 4 codes, dims 4c..4c+3 of a chunk), widened to f16 pairs
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int ks = 0; ks < C::kKSteps; ks += 2) {
-                    uint32_t w[4];
-                    ldmatrix_x4(k_tile + f8_off<D>(row_a, ks + (mi >> 1)), w);
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        uint32_t a[4];
-                        e4m3x4_to_f16x2x2(w[2 * h2], a[0], a[2]);
-                        e4m3x4_to_f16x2x2(w[2 * h2 + 1], a[1], a[3]);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_16816<F8>(sacc[nt], a, qf[nt][ks + h2][0], qf[nt][ks + h2][1]);
+                    for (int e = 0; e < 4; ++e) sacc[u][nt][e] = 0.f;
+                if constexpr (F8) {
+                    // E4M3 K straight from the tile: one ldmatrix.x4 brings 16 tokens x 32 dims of
+                    // codes (lane (r, c): 4 codes, dims 4c..4c+3 of a chunk), widened to f16 pairs
+    #pragma unroll
+                    for (int ks = 0; ks < C::kKSteps; ks += 2) {
+                        uint32_t w[4];
+                        ldmatrix_x4(k_tile + f8_off<D>(row_a[u], ks + (mi >> 1)), w);
+    #pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            uint32_t a[4];
+                            e4m3x4_to_f16x2x2(w[2 * h2], a[0], a[2]);
+                            e4m3x4_to_f16x2x2(w[2 * h2 + 1], a[1], a[3]);
+    #pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                mma_16816<F8>(sacc[u][nt], a, qf[nt][ks + h2][0], qf[nt][ks + h2][1]);
+                        }
                     }
-                }
-            } else {
-#pragma unroll
-                for (int ks = 0; ks < C::kKSteps; ++ks) {
-                    const int ch = 2 * ks + (mi >> 1);
-                    uint32_t a[4];
-                    ldmatrix_x4(swz(k_tile + (ch >> 3) * C::kHalfBytes, row_a, ch), a);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_16816<F8>(sacc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+                } else {
+    #pragma unroll
+                    for (int ks = 0; ks < C::kKSteps; ++ks) {
+                        const int ch = 2 * ks + (mi >> 1);
+                        uint32_t a[4];
+                        ldmatrix_x4(swz(k_tile + (ch >> 3) * C::kHalfBytes, row_a[u], ch), a);
+    #pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_16816<F8>(sacc[u][nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+                    }
                 }
             }
             // ---- online softmax over the 16 rows (tokens) per head column ----
-            const bool v_lo = r < valid, v_hi = (r + 8) < valid;
             // The running max m is kept lazily: while every score of the slab stays within
             // 2^kLazyLog2 of its head's m (log2 domain), the slab is weighted by 2^(s - m) as m
             // stands, with no cross-lane maximum and no rescale of O.  Otherwise (always on a
             // segment's first slab, where m = -inf) m moves to the maximum over the slab.
-            float sv[NT][4], mx[NT][2];
+            float sv[C::kMT][NT][4], mx[NT][2];
             bool need = false;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                sv[nt][0] = v_lo ? sacc[nt][0] * sl2 : -INFINITY;
-                sv[nt][1] = v_lo ? sacc[nt][1] * sl2 : -INFINITY;
-                sv[nt][2] = v_hi ? sacc[nt][2] * sl2 : -INFINITY;
-                sv[nt][3] = v_hi ? sacc[nt][3] * sl2 : -INFINITY;
-                mx[nt][0] = fmaxf(sv[nt][0], sv[nt][2]);
-                mx[nt][1] = fmaxf(sv[nt][1], sv[nt][3]);
-                need |= mx[nt][0] > m_run[nt][0] + kLazyLog2 || mx[nt][1] > m_run[nt][1] + kLazyLog2;
+            for (int nt = 0; nt < NT; ++nt) mx[nt][0] = mx[nt][1] = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < C::kMT; ++u) {
+                const bool v_lo = 16 * u + r < valid, v_hi = 16 * u + r + 8 < valid;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    sv[u][nt][0] = v_lo ? sacc[u][nt][0] * sl2 : -INFINITY;
+                    sv[u][nt][1] = v_lo ? sacc[u][nt][1] * sl2 : -INFINITY;
+                    sv[u][nt][2] = v_hi ? sacc[u][nt][2] * sl2 : -INFINITY;
+                    sv[u][nt][3] = v_hi ? sacc[u][nt][3] * sl2 : -INFINITY;
+                    mx[nt][0] = fmax3(mx[nt][0], sv[u][nt][0], sv[u][nt][2]);
+                    mx[nt][1] = fmax3(mx[nt][1], sv[u][nt][1], sv[u][nt][3]);
+                }
             }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                need |= mx[nt][0] > m_run[nt][0] + kLazyLog2 || mx[nt][1] > m_run[nt][1] + kLazyLog2;
             if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
@@ -692,44 +719,50 @@ __global__ void __launch_bounds__(kThreads, SCfg<D, NT, F8>::kMinBlocks)
                     }
                 }
             }
-            uint32_t pb[NT][2];
+            uint32_t pb[C::kMT][NT][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const float p0 = fast_exp2(sv[nt][0] - m_run[nt][0]), p1 = fast_exp2(sv[nt][1] - m_run[nt][1]);
-                const float p2 = fast_exp2(sv[nt][2] - m_run[nt][0]), p3 = fast_exp2(sv[nt][3] - m_run[nt][1]);
-                l_run[nt][0] += p0 + p2;
-                l_run[nt][1] += p1 + p3;
-                pb[nt][0] = movmatrix_trans(pack_p<F8>(p0, p1));   // tokens 0-7
-                pb[nt][1] = movmatrix_trans(pack_p<F8>(p2, p3));   // tokens 8-15
-            }
-            // ---- O^T += V^T P : 16 head-dim rows x 8 heads per (m-tile, n-tile) ----
-            if constexpr (F8) {
-                // E4M3 V: ldmatrix.trans over byte pairs gives lane (r, c) tokens 2c, 2c+1 of dims
-                // 2r, 2r+1; byte permutes split even and odd dims into two m-tiles (o_acc[2j]:
-                // dims 32j + 2r (+16), o_acc[2j+1]: dims 32j + 2r + 1 (+16))
-                const uint32_t f8v = k_tile + C::kTileBytesIn;
+            for (int u = 0; u < C::kMT; ++u)
 #pragma unroll
-                for (int j = 0; j < D / 32; ++j) {
-                    uint32_t w[4];
-                    ldmatrix_x4_trans(f8v + f8_off<D>(row_b, 2 * j + (mi & 1)), w);
-                    uint32_t ae[4], ao[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)   // bytes 0, 2 (even dims) low, 1, 3 (odd dims) high
-                        e4m3x4_to_f16x2x2(__byte_perm(w[i], 0u, 0x3120u), ae[i], ao[i]);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        mma_16816<F8>(o_acc[nt][2 * j], ae, pb[nt][0], pb[nt][1]);
-                        mma_16816<F8>(o_acc[nt][2 * j + 1], ao, pb[nt][0], pb[nt][1]);
-                    }
+                for (int nt = 0; nt < NT; ++nt) {
+                    const float p0 = fast_exp2(sv[u][nt][0] - m_run[nt][0]), p1 = fast_exp2(sv[u][nt][1] - m_run[nt][1]);
+                    const float p2 = fast_exp2(sv[u][nt][2] - m_run[nt][0]), p3 = fast_exp2(sv[u][nt][3] - m_run[nt][1]);
+                    l_run[nt][0] += p0 + p2;
+                    l_run[nt][1] += p1 + p3;
+                    pb[u][nt][0] = movmatrix_trans(pack_p<F8>(p0, p1));   // tokens 16u + 0-7
+                    pb[u][nt][1] = movmatrix_trans(pack_p<F8>(p2, p3));   // tokens 16u + 8-15
                 }
-            } else {
+            // ---- O^T += V^T P : 16 head-dim rows x 8 heads per (m-tile, n-tile), 16 tokens per
+            // k step (one per M tile of the stage) ----
 #pragma unroll
-                for (int mt = 0; mt < C::kMTiles; ++mt) {
-                    const int ch = 2 * mt + (mi & 1);
-                    uint32_t a[4];
-                    ldmatrix_x4_trans(swz(v_tile + (ch >> 3) * C::kHalfBytes, row_b, ch), a);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_16816<F8>(o_acc[nt][mt], a, pb[nt][0], pb[nt][1]);
+            for (int u = 0; u < C::kMT; ++u) {
+                if constexpr (F8) {
+                    // E4M3 V: ldmatrix.trans over byte pairs gives lane (r, c) tokens 2c, 2c+1 of dims
+                    // 2r, 2r+1; byte permutes split even and odd dims into two m-tiles (o_acc[2j]:
+                    // dims 32j + 2r (+16), o_acc[2j+1]: dims 32j + 2r + 1 (+16))
+                    const uint32_t f8v = k_tile + C::kTileBytesIn;
+    #pragma unroll
+                    for (int j = 0; j < D / 32; ++j) {
+                        uint32_t w[4];
+                        ldmatrix_x4_trans(f8v + f8_off<D>(row_b[u], 2 * j + (mi & 1)), w);
+                        uint32_t ae[4], ao[4];
+    #pragma unroll
+                        for (int i = 0; i < 4; ++i)   // bytes 0, 2 (even dims) low, 1, 3 (odd dims) high
+                            e4m3x4_to_f16x2x2(__byte_perm(w[i], 0u, 0x3120u), ae[i], ao[i]);
+    #pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            mma_16816<F8>(o_acc[nt][2 * j], ae, pb[u][nt][0], pb[u][nt][1]);
+                            mma_16816<F8>(o_acc[nt][2 * j + 1], ao, pb[u][nt][0], pb[u][nt][1]);
+                        }
+                    }
+                } else {
+    #pragma unroll
+                    for (int mt = 0; mt < C::kMTiles; ++mt) {
+                        const int ch = 2 * mt + (mi & 1);
+                        uint32_t a[4];
+                        ldmatrix_x4_trans(swz(v_tile + (ch >> 3) * C::kHalfBytes, row_b[u], ch), a);
+    #pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_16816<F8>(o_acc[nt][mt], a, pb[u][nt][0], pb[u][nt][1]);
+                    }
                 }
             }
             __syncwarp();
@@ -825,6 +858,12 @@ EncodeTiledFn encode_fn() {
 // 3-D view [blocks * Hkv][block_size][head_dim]; box = 64 dims x tb tokens x 8 kv heads.
 // bf16 pools: boxes of 64 dims in 128-byte swizzled rows; E4M3 pools: whole D-byte rows,
 // 64-byte rows (D=64) under the 64B swizzle, 128-byte rows under the 128B one.
+}  // namespace
+
+int stream_slab_tokens(bool fp8, int head_dim) { return fp8 && head_dim == 64 ? 32 : kSlab; }
+
+namespace {
+
 bool make_map(CUtensorMap* map, const void* base, const DecodeParams& p) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -833,9 +872,9 @@ bool make_map(CUtensorMap* map, const void* base, const DecodeParams& p) {
                                 (cuuint64_t)p.num_blocks * p.num_kv_heads};
     const cuuint64_t strides[2] = {(cuuint64_t)p.head_dim * esize,
                                    (cuuint64_t)p.block_size * p.head_dim * esize};
+    const int slab = stream_slab_tokens(p.kv_fp8, p.head_dim);
     const cuuint32_t box[3] = {p.kv_fp8 ? (cuuint32_t)p.head_dim : 64u,
-                               (cuuint32_t)(p.block_size < kSlab ? p.block_size : kSlab),
-                               (cuuint32_t)kGroup};
+                               (cuuint32_t)(p.block_size < slab ? p.block_size : slab), (cuuint32_t)kGroup};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapSwizzle swz_mode = !p.kv_fp8          ? CU_TENSOR_MAP_SWIZZLE_128B
                                         : p.head_dim == 64 ? CU_TENSOR_MAP_SWIZZLE_64B

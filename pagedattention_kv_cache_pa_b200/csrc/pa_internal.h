@@ -127,6 +127,8 @@ bool tensor_kernel_supports(const pa_cache_desc& d);
 // pdl: launch as a programmatic dependent of the previous kernel on the stream.
 cudaError_t launch_decode_stream(const DecodeParams& p, int grid, bool pdl, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeParams& p, bool stream_layout, bool pdl, cudaStream_t stream);
+// Tokens per stage (the unit of the stream partition): 32 for E4M3 pools at head_dim 64, else 16.
+int stream_slab_tokens(bool fp8, int head_dim);
 bool stream_kernel_supports(const pa_cache_desc& d);
 int stream_kernel_grid(const pa_cache_desc& d, int max_ctas, bool fp8);
 

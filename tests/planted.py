@@ -49,11 +49,12 @@ def planted_dims(group: int, head_dim: int) -> list:
     return [g * step for g in range(group)]
 
 
-def stream_partition(lens, num_kv_heads: int, grid: int):
-    """The stream kernel's slices.  Returns (slices, locate) where slices = [(lo, hi)] in slab
-    indices and locate(s) = (kv group, sequence, slab of the sequence)."""
+def stream_partition(lens, num_kv_heads: int, grid: int, slab: int = SLAB):
+    """The stream kernel's slices (slabs of `slab` tokens).  Returns (slices, locate) where
+    slices = [(lo, hi)] in slab indices and locate(s) = (kv group, sequence, slab of the
+    sequence)."""
     lens = np.asarray(lens, dtype=np.int64)
-    n = np.where(lens == 0, 1, -(-lens // SLAB))
+    n = np.where(lens == 0, 1, -(-lens // slab))
     s_seq = int(n.sum())
     groups = num_kv_heads // 8
     S = s_seq * groups
@@ -69,27 +70,27 @@ def stream_partition(lens, num_kv_heads: int, grid: int):
     return slices, locate
 
 
-def stream_pieces(lens, num_kv_heads: int, grid: int):
+def stream_pieces(lens, num_kv_heads: int, grid: int, slab: int = SLAB):
     """Per (kv group, sequence): the list of its pieces as (first slab, end slab) of the
     sequence, one per slice it meets, in order (one piece = the sequence was not cut)."""
-    slices, locate = stream_partition(lens, num_kv_heads, grid)
+    slices, locate = stream_partition(lens, num_kv_heads, grid, slab)
     pieces = {}
     for lo, hi in slices:
         s = lo
         while s < hi:
             gi, b, j = locate(s)
-            n_b = max(1, -(-int(lens[b]) // SLAB))
+            n_b = max(1, -(-int(lens[b]) // slab))
             end = min(n_b, j + (hi - s))
             pieces.setdefault((gi, b), []).append((j, end))
             s += end - j
     return pieces
 
 
-def stream_positions(lens, num_kv_heads: int, grid: int):
+def stream_positions(lens, num_kv_heads: int, grid: int, slab: int = SLAB):
     """(kv group, sequence, token position) of the first token of each slice's first slab,
     the last valid token of its last slab and a middle token of its middle slab."""
     lens = np.asarray(lens, dtype=np.int64)
-    slices, locate = stream_partition(lens, num_kv_heads, grid)
+    slices, locate = stream_partition(lens, num_kv_heads, grid, slab)
     out = []
     for lo, hi in slices:
         for s, where in ((lo, "first"), ((lo + hi - 1) // 2, "mid"), (hi - 1, "last")):
@@ -97,7 +98,7 @@ def stream_positions(lens, num_kv_heads: int, grid: int):
             L = int(lens[b])
             if L == 0:
                 continue
-            t0, t1 = j * SLAB, min(L, (j + 1) * SLAB)
+            t0, t1 = j * slab, min(L, (j + 1) * slab)
             p = t0 if where == "first" else (t1 - 1 if where == "last" else (t0 + t1 - 1) // 2)
             out.append((gi, b, p))
     return out

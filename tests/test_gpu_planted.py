@@ -37,7 +37,8 @@ def _planted(h, b, opts, max_len, split_tokens=0):
     info = pa.pa_decode_describe(b.batch, max_len, h.desc_of(b), opts)
     if info.kernel == pa.PA_KERNEL_TENSOR:
         assert info.ctas > 0
-        pos = pl.stream_positions(lens, b.num_kv_heads, info.ctas)
+        assert info.split_tokens in (16, 32)             # the stream kernel's slab
+        pos = pl.stream_positions(lens, b.num_kv_heads, info.ctas, info.split_tokens)
     else:
         assert info.split_tokens == split_tokens and info.max_splits > 1
         pos = pl.split_positions(lens, b.num_kv_heads, info.split_tokens)
