@@ -486,36 +486,43 @@ def capture_graph(fn, dev):
 
 def run_e2e(E, warm, stream, stage, h_in, h_outs, compute, dist, dev, host_fill=None):
     """Times E end-to-end steps.  Step i copies its inputs from pinned host memory (h_in, or
-    what host_fill(i) returns) into device staging buffer i % 2 on a copy stream, runs compute(i,
-    bufs) on `stream` once that copy has landed, and copies the step's output (the last entry of
-    bufs) back into pinned h_outs[i % 2] on the copy stream.  A staging buffer is refilled only
-    after the step two back has finished with it.  CUDA events on `stream` bracket the whole,
-    max over ranks."""
+    what host_fill(i) returns) into device staging buffer i % 2 on an upload stream, runs
+    compute(i, bufs) on `stream` once that copy has landed, and copies the step's output (the
+    last entry of bufs) back into pinned h_outs[i % 2] on a download stream, so that the two
+    directions overlap each other and the compute.  An input buffer is refilled once the
+    compute two steps back has read it; an output buffer is rewritten once its download two
+    steps back has left.  CUDA events on `stream` bracket the whole, max over ranks."""
     import torch
-    cs = torch.cuda.Stream(device=dev)
+    cs_in = torch.cuda.Stream(device=dev)
+    cs_out = torch.cuda.Stream(device=dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
+    started = [False, False]
 
     def step(i):
         j = i & 1
         d_buf, bufs = stage[j]
         if host_fill is not None:
-            ev_in[j].synchronize()                      # the copy of step i - 2 has left its host buffer
+            ev_in[j].synchronize()                      # the upload of step i - 2 has left its host buffer
             src = host_fill(i)
         else:
             src = h_in
-        with torch.cuda.stream(cs):
-            cs.wait_event(ev_out[j])                    # step i - 2 is done with these buffers
+        with torch.cuda.stream(cs_in):
+            if started[j]:
+                cs_in.wait_event(ev_done[j])            # the compute of step i - 2 has read these inputs
             d_buf.copy_(src, non_blocking=True)
-            ev_in[j].record(cs)
+            ev_in[j].record(cs_in)
         stream.wait_event(ev_in[j])
+        if started[j]:
+            stream.wait_event(ev_out[j])                # the download of step i - 2 has left this output
         compute(i, bufs)
         ev_done[j].record(stream)
-        with torch.cuda.stream(cs):
-            cs.wait_event(ev_done[j])
+        with torch.cuda.stream(cs_out):
+            cs_out.wait_event(ev_done[j])
             h_outs[j].copy_(bufs[-1], non_blocking=True)
-            ev_out[j].record(cs)
+            ev_out[j].record(cs_out)
+        started[j] = True
 
     for i in range(warm):
         step(i)
@@ -525,7 +532,8 @@ def run_e2e(E, warm, stream, stage, h_in, h_outs, compute, dist, dev, host_fill=
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    cs.wait_event(e0)                                   # no copy of the timed steps starts earlier
+    cs_in.wait_event(e0)                                # no copy of the timed steps starts earlier
+    cs_out.wait_event(e0)
     for i in range(E):
         step(warm + i)
     stream.wait_event(ev_out[(warm + E - 1) & 1])       # the last step's output is on the host
@@ -718,7 +726,7 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
         e2e = {"value": world * B * E / (e2e_ms / 1e3), "unit": "seq-steps/s",
                "h2d_bytes_per_step": int(h_buf.numel()), "d2h_bytes_per_step": int(h_outs[0].numel() * 2),
                "copies_per_step": {"h2d": 1, "d2h": 1}, "steps": E,
-               "overlap": "copies on a second stream, one step ahead of the compute"}
+               "overlap": "uploads and downloads on two streams of their own, one step ahead of the compute"}
 
     if rank != 0:
         return None
@@ -998,7 +1006,7 @@ def run_c5(args, rank, world, dist):
                 "d2h_bytes_per_step": int(h_outs[0].numel() * 2),
                 "copies_per_step": {"h2d": 1, "d2h": 1}, "steps": E,
                 "includes": "host block manager (retire, admit, append) per step",
-                "overlap": "copies on a second stream, one step ahead of the compute"},
+                "overlap": "uploads and downloads on two streams of their own, one step ahead of the compute"},
         "gpu_launches": K * NL * (1 if kernel_name == "tensor" else 2),   # one fused call per layer
         "clocks": clk,
     }

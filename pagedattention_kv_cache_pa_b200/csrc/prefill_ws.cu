@@ -153,8 +153,14 @@ struct WsItem {
 // tokens than queries, past the table, or more queries than max_q_len).
 __device__ __forceinline__ int ws_item(const PrefillParams& p, long long i, WsItem& it, bool& tile0) {
     const long long nsh = (long long)p.num_seqs * p.num_kv_heads;
-    const int t_rev = (int)(i / nsh);
-    const int rem = (int)(i - (long long)t_rev * nsh);
+    int t_rev, rem;
+    if (i <= 0x7fffffffLL && nsh <= 0x7fffffffLL) {          // 32-bit division where it fits
+        t_rev = (int)((unsigned)i / (unsigned)nsh);
+        rem = (int)((unsigned)i - (unsigned)t_rev * (unsigned)nsh);
+    } else {
+        t_rev = (int)(i / nsh);
+        rem = (int)(i - (long long)t_rev * nsh);
+    }
     it.b = rem / p.num_kv_heads;
     it.kvh = rem - it.b * p.num_kv_heads;
     tile0 = t_rev == 0 && it.kvh == 0;
@@ -359,14 +365,28 @@ __global__ void __launch_bounds__(kWsThreads, WsCfg<D>::kMinBlocks)
         // Q of an item into buffer k & 1, requested by these warps when the item before it
         // starts (that buffer's last reader, the S MMAs of item k - 2, finished before any
         // score of item k - 1 reached these warps); complete and published when that item ends
+        // thread tid copies chunk tid % kCh of rows tid / kCh + j * (128 / kCh): one division
+        // for its first row, then a carry per step of 128 / kCh rows
+        constexpr int kRowStep = 128 / kCh;
         auto load_q = [&](const WsItem& w, int qb) {
             const uint32_t qbuf = s_q + qb * C::kQBytes;
-            for (int c = tid; c < kWsRows * kCh; c += 128) {
-                const int row = c / kCh, ch = c - row * kCh, R = w.r0 + row;
+            const int tok_step = kRowStep / G, g_step = kRowStep - tok_step * G;
+            const int ch = tid % kCh;
+            int row = tid / kCh, R = w.r0 + row, tok = R / G, gq = R - tok * G;
+#pragma unroll 4
+            for (int j = 0; j < kWsRows / kRowStep; ++j) {
                 const bool live = R < w.rows;
-                const int tok = live ? R / G : 0, gq = live ? R - tok * G : 0;
-                const uint16_t* src = p.q + (((size_t)(w.q0 + tok) * Hq + (size_t)w.kvh * G + gq) * D + ch * 8);
+                const uint16_t* src =
+                    p.q + (((size_t)(w.q0 + (live ? tok : 0)) * Hq + (size_t)w.kvh * G + (live ? gq : 0)) * D + ch * 8);
                 ws_cp_async16(qbuf + ws_sw128<kWsRows>(row, ch), src, live);
+                row += kRowStep;
+                R += kRowStep;
+                tok += tok_step;
+                gq += g_step;
+                if (gq >= G) {
+                    gq -= G;
+                    ++tok;
+                }
             }
         };
         auto publish_q = [&](int qb) {
