@@ -150,3 +150,26 @@ def test_c5_batch_slab_drop_leaves_the_tolerance():
         row, L2 = _without_slabs(d, seq, [slab])
         ok, _ = oracle.within_tolerance(_decode_rows(d, seq, row, L2), full)
         assert not ok
+
+
+@pytest.mark.parametrize("slab", [16, 32])
+def test_stream_partition_mirror_tiles_every_sequence(slab):
+    """The host mirror of the stream partition (16-token slabs, 32 for E4M3 pools at D=64):
+    every (kv group, sequence) is covered by its pieces exactly once and in order, and the
+    slices cut the concatenated slabs into runs that differ by at most one slab."""
+    rng = np.random.default_rng(11 + slab)
+    for trial in range(20):
+        B = int(rng.integers(1, 40))
+        lens = rng.integers(0, 3000, size=B)
+        Hkv = int(rng.choice([8, 16]))
+        grid = int(rng.integers(1, 400))
+        slices, _ = pl.stream_partition(lens, Hkv, grid, slab)
+        sizes = [hi - lo for lo, hi in slices]
+        assert max(sizes) - min(sizes) <= 1
+        assert slices[0][0] == 0 and all(a[1] == b[0] for a, b in zip(slices, slices[1:]))
+        pieces = pl.stream_pieces(lens, Hkv, grid, slab)
+        assert len(pieces) == B * (Hkv // 8)
+        for (gi, b), ps in pieces.items():
+            nb = max(1, -(-int(lens[b]) // slab))
+            assert ps[0][0] == 0 and ps[-1][1] == nb
+            assert all(p[1] == q[0] for p, q in zip(ps, ps[1:]))
