@@ -895,6 +895,7 @@ def run_c5(args, rank, world, dist):
     rc = pa.pa_decode_status(ws)
     if rc != 0:
         raise RuntimeError("decode reported %s" % pa.pa_status_string(rc))
+    first_out = outs[0].float().cpu().numpy()            # layer 0 of trace step 0, for the parity leg
     K, W = args.steps, args.warmup
     settle(trace_step)
     graphs = args.graphs == "on" and pdl
@@ -1012,8 +1013,28 @@ def run_c5(args, rank, world, dist):
     }
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline_c5(t, tables, lens, args.cpu_seconds)
+        if args.rope == 0:
+            res["parity"] = parity_c5(t, tables, lens, first_out)
     del kcs, vcs
     return res
+
+
+def parity_c5(t, tables, lens, gpu_out):
+    """The first trace step's layer-0 output against the oracle on the same inputs: the step's
+    K/V rows appended into the initial pool at each sequence's newest position, then the decode."""
+    import oracle
+    kc, vc = t.pool(0)
+    q, k, v = t.token_inputs(0, 0)
+    L = lens[0].astype(np.int64)
+    B = len(L)
+    slots = tables[0][np.arange(B), (L - 1) // t.block_size].astype(np.int64) * t.block_size + (L - 1) % t.block_size
+    oracle.append_kv(k, v, slots, kc, vc, in_place=True)
+    ref = oracle.paged_decode(q, kc, vc, tables[0], lens[0], t.scale)
+    ok, excess = oracle.within_tolerance(gpu_out, ref)
+    err = np.abs(gpu_out.astype(np.float64) - ref)
+    return {"max_abs_err": float(err.max()), "max_abs_oracle": float(np.abs(ref).max()),
+            "within_tolerance": ok, "worst_excess": excess, "tolerance": "1e-2 + 1e-2 |oracle|",
+            "sample": "layer 0 of trace step 0 (%d sequences x %d heads), fused append + decode" % (B, t.num_q_heads)}
 
 
 def cpu_baseline_c5(t, tables, lens, budget_s):
