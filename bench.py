@@ -484,6 +484,56 @@ def capture_graph(fn, dev):
     return g
 
 
+class _Rt:
+    """The CUDA runtime calls the e2e loop issues per step (copies, event records, stream
+    waits), made straight through ctypes on the libcudart torch has loaded, on raw stream and
+    event handles: a torch copy_ of pinned memory costs several microseconds of host time
+    per call, which at C2's 28 us per step would be the bound."""
+
+    def __init__(self):
+        import ctypes
+        import torch
+        torch.cuda.init()
+        self.lib = ctypes.CDLL("libcudart.so.12")
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        L = self.lib
+        L.cudaMemcpyAsync.argtypes = [vp, vp, sz, ctypes.c_int, vp]
+        L.cudaEventRecord.argtypes = [vp, vp]
+        L.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
+        L.cudaEventSynchronize.argtypes = [vp]
+        L.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(vp), ctypes.c_uint]
+        L.cudaEventDestroy.argtypes = [vp]
+        self.events = []
+
+    def _ok(self, rc, what):
+        if rc != 0:
+            raise RuntimeError("%s returned cudaError %d" % (what, rc))
+
+    def event(self):
+        import ctypes
+        ev = ctypes.c_void_p()
+        self._ok(self.lib.cudaEventCreateWithFlags(ctypes.byref(ev), 2), "cudaEventCreateWithFlags")  # no timing
+        self.events.append(ev.value)
+        return ev.value
+
+    def copy(self, dst, src, nbytes, kind, stream):        # kind 1: host to device, 2: device to host
+        self._ok(self.lib.cudaMemcpyAsync(dst, src, nbytes, kind, stream), "cudaMemcpyAsync")
+
+    def record(self, ev, stream):
+        self._ok(self.lib.cudaEventRecord(ev, stream), "cudaEventRecord")
+
+    def wait(self, stream, ev):
+        self._ok(self.lib.cudaStreamWaitEvent(stream, ev, 0), "cudaStreamWaitEvent")
+
+    def sync(self, ev):
+        self._ok(self.lib.cudaEventSynchronize(ev), "cudaEventSynchronize")
+
+    def close(self):
+        for ev in self.events:
+            self.lib.cudaEventDestroy(ev)
+        self.events = []
+
+
 def run_e2e(E, warm, stream, stage, h_in, h_outs, compute, dist, dev, host_fill=None):
     """Times E end-to-end steps.  Step i copies its inputs from pinned host memory (h_in, or
     what host_fill(i) returns) into device staging buffer i % 2 on an upload stream, runs
@@ -493,36 +543,38 @@ def run_e2e(E, warm, stream, stage, h_in, h_outs, compute, dist, dev, host_fill=
     compute two steps back has read it; an output buffer is rewritten once its download two
     steps back has left.  CUDA events on `stream` bracket the whole, max over ranks."""
     import torch
+    rt = _Rt()
     cs_in = torch.cuda.Stream(device=dev)
     cs_out = torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    started = [False, False]
+    s_main, s_in, s_out = stream.cuda_stream, cs_in.cuda_stream, cs_out.cuda_stream
+    ev_in = [rt.event() for _ in range(2)]
+    ev_done = [rt.event() for _ in range(2)]
+    ev_out = [rt.event() for _ in range(2)]
+    d_ptr = [s[0].data_ptr() for s in stage]
+    o_ptr = [s[1][-1].data_ptr() for s in stage]
+    h_out_ptr = [h.data_ptr() for h in h_outs]
+    n_out = h_outs[0].numel() * h_outs[0].element_size()
+    n_in = stage[0][0].numel() * stage[0][0].element_size()
+    h_in_ptr = h_in.data_ptr() if h_in is not None else None
+    # a wait on an event that was never recorded returns at once: the first two steps need none
 
     def step(i):
         j = i & 1
-        d_buf, bufs = stage[j]
         if host_fill is not None:
-            ev_in[j].synchronize()                      # the upload of step i - 2 has left its host buffer
-            src = host_fill(i)
+            rt.sync(ev_in[j])                               # the upload of step i - 2 has left its host buffer
+            src = host_fill(i).data_ptr()
         else:
-            src = h_in
-        with torch.cuda.stream(cs_in):
-            if started[j]:
-                cs_in.wait_event(ev_done[j])            # the compute of step i - 2 has read these inputs
-            d_buf.copy_(src, non_blocking=True)
-            ev_in[j].record(cs_in)
-        stream.wait_event(ev_in[j])
-        if started[j]:
-            stream.wait_event(ev_out[j])                # the download of step i - 2 has left this output
-        compute(i, bufs)
-        ev_done[j].record(stream)
-        with torch.cuda.stream(cs_out):
-            cs_out.wait_event(ev_done[j])
-            h_outs[j].copy_(bufs[-1], non_blocking=True)
-            ev_out[j].record(cs_out)
-        started[j] = True
+            src = h_in_ptr
+        rt.wait(s_in, ev_done[j])                           # the compute of step i - 2 has read these inputs
+        rt.copy(d_ptr[j], src, n_in, 1, s_in)
+        rt.record(ev_in[j], s_in)
+        rt.wait(s_main, ev_in[j])
+        rt.wait(s_main, ev_out[j])                          # the download of step i - 2 has left this output
+        compute(i, stage[j][1])
+        rt.record(ev_done[j], s_main)
+        rt.wait(s_out, ev_done[j])
+        rt.copy(h_out_ptr[j], o_ptr[j], n_out, 2, s_out)
+        rt.record(ev_out[j], s_out)
 
     for i in range(warm):
         step(i)
@@ -536,9 +588,10 @@ def run_e2e(E, warm, stream, stage, h_in, h_outs, compute, dist, dev, host_fill=
     cs_out.wait_event(e0)
     for i in range(E):
         step(warm + i)
-    stream.wait_event(ev_out[(warm + E - 1) & 1])       # the last step's output is on the host
+    rt.wait(s_main, ev_out[(warm + E - 1) & 1])         # the last step's output is on the host
     e1.record(stream)
     torch.cuda.synchronize()
+    rt.close()
     ms, = max_over_ranks([e0.elapsed_time(e1)], dist, dev)
     return ms
 
@@ -721,12 +774,26 @@ def run_decode(args, rank, world, dist, cfg=None, steps=None, warmup=None, e2e_s
         stage = [(d_buf, resident), (d_buf2, tuple(io2[n][1] for n in ("q", "k", "v", "slots", "tables",
                                                                        "lens")) + (out2,))]
         h_outs = [torch.empty(out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-        e2e_ms = run_e2e(E, min(W, 20), stream, stage, h_buf, h_outs,
-                         lambda i, bufs: call(i % layers, bufs=bufs), dist, dev)
+        compute = lambda i, bufs: call(i % layers, bufs=bufs)    # noqa: E731
+        if fused:
+            # the same library call on raw device pointers (the binding takes ints as well):
+            # its per-tensor dtype, device and contiguity checks passed above for these buffers
+            raw = [tuple(t.data_ptr() for t in s[1]) for s in stage]
+            kc_p, vc_p = [t.data_ptr() for t in kcs], [t.data_ptr() for t in vcs]
+            ws_p, s_h = ws.data_ptr(), stream.cuda_stream
+
+            def compute(i, bufs):
+                qp, kp, vp, _, tp, lp, op = raw[i & 1]
+                L = i % layers
+                pa.pa_append_decode(qp, kp, vp, kc_p[L], vc_p[L], tp, lp, max_len, b.scale, op, ws_p, desc,
+                                    opts, stream=s_h, num_seqs=B, workspace_bytes=wsb)
+        e2e_ms = run_e2e(E, min(W, 20), stream, stage, h_buf, h_outs, compute, dist, dev)
         e2e = {"value": world * B * E / (e2e_ms / 1e3), "unit": "seq-steps/s",
                "h2d_bytes_per_step": int(h_buf.numel()), "d2h_bytes_per_step": int(h_outs[0].numel() * 2),
                "copies_per_step": {"h2d": 1, "d2h": 1}, "steps": E,
-               "overlap": "uploads and downloads on two streams of their own, one step ahead of the compute"}
+               "overlap": "uploads and downloads on two streams of their own, one step ahead of the compute",
+               "host_calls": "cudaMemcpyAsync and event calls on raw handles; the library call on raw pointers"
+                             if fused else "cudaMemcpyAsync and event calls on raw handles"}
 
     if rank != 0:
         return None

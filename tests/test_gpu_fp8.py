@@ -127,6 +127,38 @@ def test_decode_e4m3_shapes(h, shape):
         _decode_case(h, b, 5.0 / 448, 0.02, max_ctas=ctas, fused=fused)
 
 
+# lengths on both sides of every 32-token stage boundary up to a few stages, and past 1024
+SLAB_LENS = sorted({0, 1, 2, 31, 32, 33, 63, 64, 65, 95, 96, 97, 159, 160, 161, 255, 256, 257, 1023,
+                    1024, 1025})
+
+
+@pytest.mark.parametrize("Bs", [8, 16, 32, 64])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_decode_e4m3_32_token_stages(h, Bs, G):
+    """E4M3 pools at head_dim 64 stream K/V in 32-token stages (two bf16-sized 16-token slabs
+    per stage): block sizes below, at and above the stage size, every GQA group the kernel
+    takes, lengths on both sides of each stage boundary; direct, partitioned and fused."""
+    Hkv = 8
+    b = wl.small_batch(7100 + Bs * 32 + G, SLAB_LENS, num_q_heads=Hkv * G, num_kv_heads=Hkv, head_dim=64,
+                       block_size=Bs)
+    opts = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR, kv_dtype=pa.PA_KV_E4M3, k_scale=0.02, v_scale=0.02)
+    plan = pa.pa_decode_describe(b.batch, int(b.context_lens.max()) + 1, h.desc_of(b), opts)
+    assert plan.split_tokens == 32
+    for ctas, fused, pdl in ((0, True, True), (7, False, False), (40, True, False)):
+        _decode_case(h, b, 5.0 / 448, 0.03, max_ctas=ctas, pdl=pdl, fused=fused)
+
+
+@pytest.mark.parametrize("D,want", [(64, 32), (128, 16)])
+def test_e4m3_stage_size_reported(h, D, want):
+    """pa_decode_describe reports the stream kernel's stage: 32 tokens for E4M3 at head_dim 64,
+    16 otherwise (and 16 for bf16 pools at either head_dim)."""
+    b = wl.small_batch(7300 + D, [100, 200], num_q_heads=32, num_kv_heads=8, head_dim=D, block_size=16)
+    f8 = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR, kv_dtype=pa.PA_KV_E4M3, k_scale=0.02, v_scale=0.02)
+    bf = pa.DecodeOptions(kernel=pa.PA_KERNEL_TENSOR)
+    assert pa.pa_decode_describe(2, 201, h.desc_of(b), f8).split_tokens == want
+    assert pa.pa_decode_describe(2, 201, h.desc_of(b), bf).split_tokens == 16
+
+
 def test_e4m3_unsupported_combinations(h):
     b = wl.config1()                                     # Hkv = 1: no whole-group kernel
     desc = h.desc_of(b)
