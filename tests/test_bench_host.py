@@ -21,3 +21,42 @@ def test_pf_cpu_baseline_samples_every_part_of_the_chunks():
     windows = bench.PF_NEW // 64
     seen = {(n % B, (13 * (n // B)) % windows) for n in range(B * windows)}
     assert len(seen) == B * windows
+
+
+def test_unique_kv_bytes_counts_shared_blocks_once():
+    """The roofline's bytes for a shared prefix: a block held by several tables counts once
+    (with the most tokens any sequence uses in it); without sharing they equal the logical
+    K+V bytes."""
+    Bs, Hkv, D = 4, 2, 8
+    # three sequences over one shared 2-block prefix (8 tokens), then private blocks
+    tables = np.array([[0, 1, 2, 3], [0, 1, 4, 0], [0, 1, 5, 6]], dtype=np.int32)
+    lens = np.array([15, 9, 13], dtype=np.int32)
+    row = 2 * Hkv * D * 2                                  # K+V bytes of one token, bf16
+    # prefix 8 tokens once; suffixes 7, 1 and 5 tokens
+    assert bench.unique_kv_bytes(tables, lens, Bs, Hkv, D) == (8 + 7 + 1 + 5) * row
+    assert bench.kv_read_bytes(lens, Hkv, D) == int(lens.sum()) * row
+    # private tables: unique == logical, and E4M3 halves both
+    private = np.array([[0, 1, 2, 3], [4, 5, 6, 7], [8, 9, 10, 11]], dtype=np.int32)
+    assert bench.unique_kv_bytes(private, lens, Bs, Hkv, D) == bench.kv_read_bytes(lens, Hkv, D)
+    assert bench.unique_kv_bytes(private, lens, Bs, Hkv, D, 1) * 2 == bench.kv_read_bytes(lens, Hkv, D)
+    # a partly used shared block counts the longest use: two sequences of 2 and 3 tokens in block 7
+    assert bench.unique_kv_bytes(np.array([[7], [7]]), np.array([2, 3]), Bs, Hkv, D) == 3 * row
+
+
+def test_profiled_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    """A DRAM figure from a profile summary is used only while the kernel sources still hash
+    to the build that was captured; any other hash (an edited kernel) gives null."""
+    import os
+    pkg = tmp_path / "pagedattention_kv_cache_pa_b200"
+    pkg.mkdir()
+    os.symlink(os.path.join(bench.ROOT, "pagedattention_kv_cache_pa_b200", "csrc"), pkg / "csrc")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    good = bench.kernel_source_hash("tensor")
+    (tmp_path / "profiles" / "a.md").write_text(
+        "traffic[c9,tensor]: 12345 bytes/launch source=%s\n"
+        "traffic[c8,tensor]: 999 bytes/launch source=%s\n" % (good, "0" * 16))
+    assert bench.profiled_traffic("c9", "tensor") == 12345
+    assert bench.profiled_traffic("c8", "tensor") is None     # captured on other sources
+    assert bench.profiled_traffic("c7", "tensor") is None     # never captured
+    assert bench.kernel_source_hash("prefill_ws") != good     # each kernel hashes its own files
