@@ -400,8 +400,28 @@ def run_reference(args, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+def single_thread_rate(step, seconds, max_steps=1000):
+    """The same oracle steps on one host thread, for a bounded time (at least one step):
+    (steps, seconds).  The OpenMP thread count is put back afterwards."""
+    import oracle
+    prev = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        n = 0
+        t0 = time.perf_counter()
+        while True:
+            step(n)
+            n += 1
+            dt = time.perf_counter() - t0
+            if dt >= seconds or n >= max_steps:
+                return n, dt
+    finally:
+        oracle.set_num_threads(prev)
+
+
 def cpu_baseline(b, slots, tables, lens, budget_s):
-    """The oracle as it stands on the host's cores, on whole-batch steps until the budget is spent."""
+    """The oracle as it stands on the host's cores, on whole-batch steps until the budget is
+    spent; then the same steps on one thread for a third of the budget."""
     import oracle
     kc, vc = b.k_cache.copy(), b.v_cache.copy()
     n = 0
@@ -413,10 +433,14 @@ def cpu_baseline(b, slots, tables, lens, budget_s):
         dt = time.perf_counter() - t0
         if dt >= budget_s or n >= 1000:
             break
+    n1, dt1 = single_thread_rate(lambda i: oracle.paged_decode(b.q, kc, vc, tables, lens, b.scale),
+                                 budget_s / 3)
     return {"value": n * b.batch / dt, "unit": "seq-steps/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": "%d whole-batch steps of %s (append + decode of all %d sequences x %d heads), %.1f s"
-                      % (n, b.name, b.batch, b.num_q_heads, dt)}
+                      % (n, b.name, b.batch, b.num_q_heads, dt),
+            "single_thread": {"value": n1 * b.batch / dt1, "unit": "seq-steps/s", "cores": 1,
+                              "sample": "%d whole-batch decodes, %.1f s" % (n1, dt1)}}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -1118,11 +1142,16 @@ def cpu_baseline_c5(t, tables, lens, budget_s):
         dt = time.perf_counter() - t0
         if dt >= budget_s:
             break
+    n1, dt1 = single_thread_rate(lambda i: oracle.paged_decode(q, kc, vc, tables[i % t.steps],
+                                                                lens[i % t.steps], t.scale), budget_s / 3)
     # one seq-step = one sequence through all layers: the sample covers 1 of the 16 layers
     return {"value": n * t.batch / dt / t.layers, "unit": "seq-steps/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": "%d trace steps of layer 0 only (256 sequences x 32 heads each), %.1f s; "
-                      "value scaled to all %d layers" % (n, dt, t.layers)}
+                      "value scaled to all %d layers" % (n, dt, t.layers),
+            "single_thread": {"value": n1 * t.batch / dt1 / t.layers, "unit": "seq-steps/s", "cores": 1,
+                              "sample": "%d trace steps of layer 0 on one thread, %.1f s; value scaled "
+                                        "to all %d layers" % (n1, dt1, t.layers)}}
 
 
 def run_pc(args, rank, world, dist):

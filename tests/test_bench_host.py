@@ -60,3 +60,20 @@ def test_profiled_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("c8", "tensor") is None     # captured on other sources
     assert bench.profiled_traffic("c7", "tensor") is None     # never captured
     assert bench.kernel_source_hash("prefill_ws") != good     # each kernel hashes its own files
+
+
+def test_decode_cpu_baseline_reports_parallel_and_single_thread():
+    """The decode CPU baseline times the oracle on the host's threads and again on one thread,
+    and leaves the oracle's thread count as it found it."""
+    import oracle
+    b = wl.small_batch(77, [5, 40, 300], num_q_heads=8, num_kv_heads=2)
+    B, Bs = b.batch, b.block_size
+    lens = b.context_lens.astype(np.int32) + 1
+    slots = np.array([int(b.block_tables[s, (L - 1) // Bs]) * Bs + (L - 1) % Bs for s, L in enumerate(lens)],
+                     dtype=np.int64)
+    before = oracle.num_threads()
+    res = bench.cpu_baseline(b, slots, b.block_tables, lens, 0.05)
+    assert oracle.num_threads() == before
+    assert res["kind"] == "oracle" and res["value"] > 0 and res["cores"] == before
+    st = res["single_thread"]
+    assert st["cores"] == 1 and st["value"] > 0 and st["unit"] == res["unit"]
